@@ -1,0 +1,238 @@
+"""fp64 CPU oracle for the Kimi Delta Attention (KDA) token mixer.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the bench's CPU
+baseline may import this module; the library never does. It shares no code with
+the CUDA path (the seeded input generators are the only common module, and they
+hold none of the mixer's arithmetic).
+
+What it computes (all in float64, from the exact input values upcast):
+
+* ``kda_recurrence`` — the token-by-token definition. The pages' KDA section
+  ("KDA: constant-size memory over a very long context", Ling-3.0-flash article,
+  ai.thesatyajit.com) describes a fixed d_k x d_v state per head that each token
+  first decays per key channel (the gated decay alpha_t, "the erase") and then
+  writes with the delta rule (the write beta_t k_t v_t^T), read by the query. The
+  displayed equation is missing from the extracted page; the reading used is
+
+      S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+      o_t = S_t^T q_t,   alpha_t = exp(log_alpha_t) per key channel,
+
+  i.e. decay acts on the key (row) side and the read happens after the write.
+* ``kda_chunked`` — the chunk-parallel rewrite of the same recurrence (WY/UT
+  form), written in its plainest matrix form per chunk with the pairwise decay
+  factors exp(g_r - g_i) evaluated exactly (no factorisation). It is a
+  self-check of the algebra a chunked kernel follows; it must equal
+  ``kda_recurrence`` to rounding.
+* ``short_conv``, ``l2norm``, ``output_gate`` and ``kda_mixer`` — the fused
+  pre/post stage drawn in the article's KDA panel: a short causal depthwise
+  convolution (kernel 4, from the model's config field short_conv_kernel_size on
+  the llm-architectures-explained page, "Every architecture field") on q, k, v,
+  an L2 norm of q and k, and a final sigmoid output gate.
+* ``kda_decode_step`` — one token of the recurrence for a batch of sequences,
+  updating the state in place (the constant-size state is what makes decode
+  cost independent of context length, same article section).
+
+Readings where the pages are silent (the full list is kept with the design
+notes): no 1/sqrt(d_k) query scale; log_alpha is given directly (natural log,
+<= 0); beta is given in (0, 1); conv tap w[c, 3] multiplies the current token,
+zero history at every sequence start, no bias, identity activation; L2 norm is
+x / sqrt(sum x^2 + 1e-6); the gate is out * sigmoid(g) with no norm before it.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import numpy as np
+from scipy.special import expit
+
+L2NORM_EPS = 1e-6
+CONV_WIDTH = 4
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def _packed(q, k, v, log_alpha, beta, cu_seqlens):
+    """Accept [B, T, H, d] (fixed length) or [sum_T, H, d] (packed with cu_seqlens)."""
+    q, k, v, la, b = _f64(q), _f64(k), _f64(v), _f64(log_alpha), _f64(beta)
+    if cu_seqlens is None:
+        if q.ndim != 4:
+            raise ValueError("fixed-length inputs must be [B, T, H, d]")
+        B, T = q.shape[:2]
+        cu = np.arange(B + 1, dtype=np.int64) * T
+        return (q.reshape(B * T, *q.shape[2:]), k.reshape(B * T, *k.shape[2:]),
+                v.reshape(B * T, *v.shape[2:]), la.reshape(B * T, *la.shape[2:]),
+                b.reshape(B * T, *b.shape[2:]), cu, (B, T))
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    return q, k, v, la, b, cu, None
+
+
+def token_step(S: np.ndarray, q_t, k_t, v_t, la_t, beta_t) -> Tuple[np.ndarray, np.ndarray]:
+    """One token for every head at once. S [H, dk, dv] -> (S_t, o_t [H, dv]).
+
+    Decay the key rows (Diag(alpha) S), form the delta-rule residual of the
+    decayed state at k_t, write beta * k_t (residual)^T, read with q_t.
+    """
+    S = np.exp(la_t)[:, :, None] * S                       # Diag(alpha_t) S_{t-1}
+    pred = np.einsum("hk,hkv->hv", k_t, S)                 # (Diag(alpha) S)^T k_t
+    u = beta_t[:, None] * (v_t - pred)                     # beta_t (v_t - prediction)
+    S = S + k_t[:, :, None] * u[:, None, :]                # + k_t u^T
+    o = np.einsum("hk,hkv->hv", q_t, S)                    # o_t = S_t^T q_t
+    return S, o
+
+
+def kda_recurrence(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
+                   return_states: bool = False):
+    """Token-by-token KDA over packed sequences.
+
+    q, k, log_alpha: [sum_T, H, dk]; v: [sum_T, H, dv]; beta: [sum_T, H];
+    initial_state: [N, H, dk, dv] or None (zeros); cu_seqlens: [N+1] or None
+    with [B, T, H, d] inputs. Returns (out [like v], final_state [N, H, dk, dv]),
+    plus the per-token states [sum_T, H, dk, dv] if ``return_states``.
+    """
+    q, k, v, la, b, cu, fixed = _packed(q, k, v, log_alpha, beta, cu_seqlens)
+    N = len(cu) - 1
+    H, dk = k.shape[1], k.shape[2]
+    dv = v.shape[2]
+    out = np.zeros((q.shape[0], H, dv))
+    final = np.zeros((N, H, dk, dv))
+    states = np.zeros((q.shape[0], H, dk, dv)) if return_states else None
+    for n in range(N):
+        S = np.zeros((H, dk, dv)) if initial_state is None else _f64(initial_state[n]).copy()
+        for t in range(cu[n], cu[n + 1]):
+            S, out[t] = token_step(S, q[t], k[t], v[t], la[t], b[t])
+            if return_states:
+                states[t] = S
+        final[n] = S
+    if fixed is not None:
+        out = out.reshape(fixed[0], fixed[1], H, dv)
+    return (out, final, states) if return_states else (out, final)
+
+
+def kda_chunked(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk: int = 64):
+    """The same result via the chunk-parallel (WY / UT) rewrite.
+
+    Inside a chunk of L tokens that starts from state S0, with g_r the running
+    sum of log_alpha up to and including token r (per key channel):
+      A[r,i]  = beta_r * sum_c k[r,c] k[i,c] exp(g[r,c] - g[i,c])  for i < r
+      T       = (I + A)^-1 Diag(beta)
+      W       = T (K * exp(g)),  U~ = T V,  U = U~ - W S0
+      P[r,i]  = sum_c q[r,c] k[i,c] exp(g[r,c] - g[i,c])          for i <= r
+      O       = (Q * exp(g)) S0 + P U
+      S_L     = Diag(exp(g_last)) S0 + (K * exp(g_last - g))^T U
+    Chunks never cross a sequence boundary; the last chunk may be partial.
+    """
+    q, k, v, la, b, cu, fixed = _packed(q, k, v, log_alpha, beta, cu_seqlens)
+    N = len(cu) - 1
+    H, dk = k.shape[1], k.shape[2]
+    dv = v.shape[2]
+    out = np.zeros((q.shape[0], H, dv))
+    final = np.zeros((N, H, dk, dv))
+    for n in range(N):
+        S = np.zeros((H, dk, dv)) if initial_state is None else _f64(initial_state[n]).copy()
+        for s in range(cu[n], cu[n + 1], chunk):
+            e = min(s + chunk, cu[n + 1])
+            L = e - s
+            Q = q[s:e].transpose(1, 0, 2)                  # [H, L, dk]
+            K = k[s:e].transpose(1, 0, 2)
+            V = v[s:e].transpose(1, 0, 2)                  # [H, L, dv]
+            g = np.cumsum(la[s:e].transpose(1, 0, 2), axis=1)   # [H, L, dk]
+            beta_c = b[s:e].T                               # [H, L]
+            strict = np.tril(np.ones((L, L), dtype=bool), -1)
+            incl = np.tril(np.ones((L, L), dtype=bool), 0)
+            # pairwise decay exp(g_r - g_i), only where i <= r (never overflows)
+            diff = g[:, :, None, :] - g[:, None, :, :]      # [H, r, i, dk]
+            decay = np.where(incl[None, :, :, None], np.exp(np.where(incl[None, :, :, None], diff, 0.0)), 0.0)
+            KK = np.einsum("hrc,hic,hric->hri", K, K, decay)
+            QK = np.einsum("hrc,hic,hric->hri", Q, K, decay)
+            A = beta_c[:, :, None] * np.where(strict, KK, 0.0)
+            P = np.where(incl, QK, 0.0)
+            eye = np.eye(L)
+            Tm = np.linalg.solve(eye[None] + A, np.broadcast_to(eye, (H, L, L))) * beta_c[:, None, :]
+            Gam = np.exp(g)
+            W = Tm @ (K * Gam)
+            Ut = Tm @ V
+            U = Ut - W @ S
+            O = (Q * Gam) @ S + P @ U
+            g_last = g[:, -1, :]                            # [H, dk]
+            Kdec = K * np.exp(g_last[:, None, :] - g)
+            S = np.exp(g_last)[:, :, None] * S + Kdec.transpose(0, 2, 1) @ U
+            out[s:e] = O.transpose(1, 0, 2)
+        final[n] = S
+    if fixed is not None:
+        out = out.reshape(fixed[0], fixed[1], H, dv)
+    return out, final
+
+
+def short_conv(x, w, cu_seqlens) -> np.ndarray:
+    """Causal depthwise convolution of width 4 on packed [sum_T, C] channels.
+
+    y[t, c] = sum_{j=0..3} w[c, j] * x[t - 3 + j, c], with x taken as zero
+    before each sequence's first token; no bias, identity activation.
+    """
+    x, w = _f64(x), _f64(w)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    y = np.zeros_like(x)
+    for n in range(len(cu) - 1):
+        s, e = cu[n], cu[n + 1]
+        for t in range(s, e):
+            for j in range(CONV_WIDTH):
+                src = t - (CONV_WIDTH - 1) + j
+                if src >= s:
+                    y[t] += w[:, j] * x[src]
+    return y
+
+
+def l2norm(x, eps: float = L2NORM_EPS) -> np.ndarray:
+    """x / sqrt(sum(x^2) + eps) over the last axis."""
+    x = _f64(x)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+
+
+def output_gate(o, g) -> np.ndarray:
+    """Final sigmoid output gate: o * sigmoid(g), elementwise."""
+    return _f64(o) * expit(_f64(g))
+
+
+def kda_mixer(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, cu_seqlens,
+              initial_state=None):
+    """Full mixer stage: conv4 on q, k, v -> L2 norm on q, k -> KDA -> sigmoid gate.
+
+    q_raw, k_raw: [sum_T, H, dk]; v_raw: [sum_T, H, dv]; conv_w: [3, H*d, 4]
+    (q, k, v weights); gate: [sum_T, H, dv] or None.
+    """
+    TT, H, dk = np.shape(q_raw)
+    dv = np.shape(v_raw)[2]
+    qc = short_conv(np.reshape(q_raw, (TT, H * dk)), conv_w[0], cu_seqlens).reshape(TT, H, dk)
+    kc = short_conv(np.reshape(k_raw, (TT, H * dk)), conv_w[1], cu_seqlens).reshape(TT, H, dk)
+    vc = short_conv(np.reshape(v_raw, (TT, H * dv)), conv_w[2], cu_seqlens).reshape(TT, H, dv)
+    out, final = kda_recurrence(l2norm(qc), l2norm(kc), vc, log_alpha, beta, initial_state, cu_seqlens)
+    if gate is not None:
+        out = output_gate(out, gate)
+    return out, final
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, state) -> Tuple[np.ndarray, np.ndarray]:
+    """One decode token for N sequences: q, k, log_alpha [N, H, dk]; v [N, H, dv];
+    beta [N, H]; state [N, H, dk, dv]. Returns (out [N, H, dv], new state)."""
+    q, k, v, la, b, S = _f64(q), _f64(k), _f64(v), _f64(log_alpha), _f64(beta), _f64(state)
+    out = np.zeros(v.shape)
+    new = np.zeros(S.shape)
+    for n in range(S.shape[0]):
+        new[n], out[n] = token_step(S[n], q[n], k[n], v[n], la[n], b[n])
+    return out, new
+
+
+def kda_decode_steps(q, k, v, log_alpha, beta, state, seq_subset: Optional[np.ndarray] = None):
+    """Consecutive decode steps: inputs carry a leading [steps] axis. Optionally only
+    a subset of sequences (indices into N) is run. Returns (out [steps, n, H, dv], final)."""
+    idx = np.arange(np.shape(state)[0]) if seq_subset is None else np.asarray(seq_subset)
+    S = _f64(np.asarray(state)[idx])
+    steps = np.shape(q)[0]
+    outs = []
+    for s in range(steps):
+        o, S = kda_decode_step(np.asarray(q[s])[idx], np.asarray(k[s])[idx], np.asarray(v[s])[idx],
+                               np.asarray(log_alpha[s])[idx], np.asarray(beta[s])[idx], S)
+        outs.append(o)
+    return np.stack(outs), S
