@@ -1,0 +1,475 @@
+"""Benchmark of the KDA hot path on B200: prefill tokens/s (headline) with decode
+state GB/s, full-mixer and varlen prefill alongside, each against its roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (one process per GPU)
+
+A step is one kda_chunk_fwd call over the model-shape prefill workload (B=1,
+T=4096, H=32, d_k=d_v=128, bf16 q/k/v, fp32 log_alpha/beta/state). The path is
+independent per (sequence, head), so N GPUs run N replicas of the workload
+("weak" scaling, no data-path collective); each GPU's time comes from CUDA
+events on the launching stream and the job time is the max over ranks.
+Between timed steps the inputs rotate through copies whose total exceeds L2.
+`--impl reference` times the fp64 CPU oracle instead (a deliberately slow
+reference arm on the host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s & decode state GB/s at H=32,d=128 (1 B200, % roofline)"
+H, D, T1 = 32, 128, 4096
+CHUNK = 64
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+# ----------------------------------------------------------------------------------
+# algorithmic work (bytes / flops the method must move or do, per call)
+# ----------------------------------------------------------------------------------
+def prefill_bytes(total_T: int, N: int, Hh: int = H, d: int = D, with_h0: bool = True, mixer: bool = False) -> int:
+    """q, k, v, out (bf16) + log_alpha (fp32) + beta (fp32) + states in/out (fp32).
+    The full mixer adds the gate (bf16) and conv weights; its q, k, v are the raw ones."""
+    tok = total_T * Hh
+    b = tok * d * 2 * 4 + tok * d * 4 + tok * 4
+    b += N * Hh * d * d * 4 * (2 if with_h0 else 1)
+    if mixer:
+        b += tok * d * 2 + 3 * Hh * d * 4 * 4
+    return b
+
+
+def prefill_tc_flops(total_T: int, Hh: int = H, d: int = D, chunk: int = CHUNK) -> int:
+    """Dense tensor-core work per token-head of the chunked form: three d x d state
+    GEMMs (6 d^2) and five chunk-wide GEMMs (10 C d)."""
+    return total_T * Hh * (6 * d * d + 10 * chunk * d)
+
+
+def decode_bytes(N: int, Hh: int = H, d: int = D) -> int:
+    """State read + write (fp32) plus the token's q, k, v, out (bf16), log_alpha, beta."""
+    return N * Hh * (2 * d * d * 4 + 4 * d * 2 + d * 4 + 4)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------------
+# distributed plumbing (replicas): rank info, barrier, max over ranks
+# ----------------------------------------------------------------------------------
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def job_throughput(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Weak scaling: every rank processes `units_per_rank`; the job time is the slowest rank's."""
+    return units_per_rank * world / seconds_max
+
+
+# ----------------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()) if rows else None,
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------------
+# synthetic inputs on the device (timing only; parity runs on the NumPy generator)
+# ----------------------------------------------------------------------------------
+def device_prefill_inputs(total_T, Hh, d, seed, device, normalise=True, state_N=None, mixer=False):
+    import torch
+    g = torch.Generator(device=device).manual_seed(seed)
+    def nrm(*shape):
+        return torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    q, k, v = nrm(total_T, Hh, d), nrm(total_T, Hh, d), nrm(total_T, Hh, d)
+    if normalise:
+        q = q / q.norm(dim=-1, keepdim=True)
+        k = k / k.norm(dim=-1, keepdim=True)
+    la = -torch.nn.functional.softplus(nrm(total_T, Hh, d)) / 16
+    beta = torch.sigmoid(nrm(total_T, Hh))
+    out = dict(q=q.bfloat16(), k=k.bfloat16(), v=v.bfloat16(), log_alpha=la.contiguous(), beta=beta.contiguous())
+    out["initial_state"] = (0.02 * nrm(state_N, Hh, d, d)) if state_N else None
+    if mixer:
+        out["conv_w"] = 0.5 * nrm(3, Hh * d, 4)
+        out["gate"] = nrm(total_T, Hh, d).bfloat16()
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------------
+def time_region(fn, steps, warmup, stream, device):
+    """W untimed calls, then K calls between events; returns per-step ms list (events
+    per step) and the total ms for the K steps, bracketed by barrier + sync."""
+    import torch
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        fn(warmup + i)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    return per, ev[0].elapsed_time(ev[steps])
+
+
+def run_gpu(args):
+    import numpy as np
+    import torch
+
+    import gated_delta_rule_137_b200 as kda
+    from gated_delta_rule_137_b200 import build as kbuild
+    from gated_delta_rule_137_b200 import inputs as I
+
+    rank, local_rank, world = dist_env()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    init_dist(world, "nccl")
+    if rank == 0:
+        kbuild.build()
+    barrier(device)
+    lib = kda.load_library()
+    stream = torch.cuda.current_stream(device)
+    hbm_peak, tc_peak, tc_peak_sus, peak_src = load_peaks()
+    launches = 0
+
+    # ---------------- headline: model-shape prefill, inputs resident in HBM -----------
+    w = I.prefill_model_shape()
+    host = dict(q=torch.from_numpy(w.q).to(torch.bfloat16), k=torch.from_numpy(w.k).to(torch.bfloat16),
+                v=torch.from_numpy(w.v).to(torch.bfloat16), log_alpha=torch.from_numpy(w.log_alpha),
+                beta=torch.from_numpy(w.beta), initial_state=torch.from_numpy(w.initial_state))
+    bytes_call = prefill_bytes(T1, 1)
+    n_sets = max(2, math.ceil(3 * 126e6 / bytes_call) + 1)  # rotate through > 3x L2
+    sets = []
+    for _ in range(n_sets):
+        sets.append({k: t.to(device) for k, t in host.items()})
+    outs = [torch.empty(T1, H, D, dtype=torch.bfloat16, device=device) for _ in range(n_sets)]
+    fins = [torch.empty(1, H, D, D, dtype=torch.float32, device=device) for _ in range(n_sets)]
+    ws_bytes = kda.chunk_fwd_workspace_bytes(T1, 1, H, D, D, kda.KDA_DT_BF16)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
+
+    def step(i):
+        s = sets[i % n_sets]
+        kda.chunk_fwd(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], s["initial_state"], None, N=1,
+                      out=outs[i % n_sets], final_state=fins[i % n_sets], workspace=ws, stream=stream)
+
+    with ClockSampler(device.index) as clk:
+        per, total_ms = time_region(step, args.steps, args.warmup, stream, device)
+    launches += args.steps
+    kda.workspace_status(ws)
+    clocks = clk.summary()
+    total_ms_max = max_over_ranks(total_ms, device)
+    ms_per_step = total_ms_max / args.steps
+    value = job_throughput(T1 * args.steps, world, total_ms_max / 1e3)
+    kern_ms = statistics.mean(per)
+    achieved_gbs = bytes_call / (kern_ms / 1e3) / 1e9
+    tc_tflops = prefill_tc_flops(T1) / (kern_ms / 1e3) / 1e12
+
+    # ---------------- e2e: host buffers through the public API ----------------------
+    pin = {k: t.pin_memory() for k, t in host.items()}
+    dev = {k: torch.empty_like(t, device=device) for k, t in host.items()}
+    h_out = torch.empty(T1, H, D, dtype=torch.bfloat16).pin_memory()
+    h_fin = torch.empty(1, H, D, D, dtype=torch.float32).pin_memory()
+    d_out = torch.empty(T1, H, D, dtype=torch.bfloat16, device=device)
+    d_fin = torch.empty(1, H, D, D, dtype=torch.float32, device=device)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = h_out.numel() * 2 + h_fin.numel() * 4
+
+    def e2e_step(i):
+        for k in pin:
+            dev[k].copy_(pin[k], non_blocking=True)
+        kda.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], dev["initial_state"], None,
+                      N=1, out=d_out, final_state=d_fin, workspace=ws, stream=stream)
+        h_out.copy_(d_out, non_blocking=True)
+        h_fin.copy_(d_fin, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    _, e2e_ms = time_region(e2e_step, e2e_steps, max(1, min(args.warmup, 3)), stream, device)
+    e2e_ms = max_over_ranks(e2e_ms, device)
+    e2e_value = job_throughput(T1 * e2e_steps, world, e2e_ms / 1e3)
+
+    # ---------------- decode: 256 sequences x 32 heads, 64 in-place steps ----------------
+    Nd, dsteps = 256, 64
+    gd = torch.Generator(device=device).manual_seed(1370003)
+    state = 0.02 * torch.randn(Nd, H, D, D, generator=gd, device=device)
+    n_tok_sets = 8
+    toks = []
+    for _ in range(n_tok_sets):
+        q = torch.randn(Nd, H, D, generator=gd, device=device)
+        k = torch.randn(Nd, H, D, generator=gd, device=device)
+        toks.append(dict(q=(q / q.norm(dim=-1, keepdim=True)).bfloat16(), k=(k / k.norm(dim=-1, keepdim=True)).bfloat16(),
+                         v=torch.randn(Nd, H, D, generator=gd, device=device).bfloat16(),
+                         la=(-torch.nn.functional.softplus(torch.randn(Nd, H, D, generator=gd, device=device)) / 16).contiguous(),
+                         b=torch.sigmoid(torch.randn(Nd, H, generator=gd, device=device)).contiguous()))
+    d_outbuf = torch.empty(Nd, H, D, dtype=torch.bfloat16, device=device)
+
+    def dstep(i):
+        t = toks[i % n_tok_sets]
+        kda.decode_step(t["q"], t["k"], t["v"], t["la"], t["b"], state, out=d_outbuf, stream=stream)
+
+    dper, dtot = time_region(dstep, dsteps, 3, stream, device)
+    launches += dsteps
+    dtot = max_over_ranks(dtot, device)
+    dbytes = decode_bytes(Nd)
+    d_us = dtot / dsteps * 1e3
+    decode = {"workload": f"decode N={Nd} H={H} d={D} fp32 state in place, {dsteps} consecutive steps",
+              "us_per_step": d_us, "state_GBps": 2 * Nd * H * D * D * 4 / (d_us * 1e-6) / 1e9,
+              "GBps_all_bytes": dbytes / (d_us * 1e-6) / 1e9,
+              "tokens_per_s": job_throughput(Nd * dsteps, world, dtot / 1e3),
+              "roofline": {"bound": "hbm", "achieved": dbytes / (statistics.mean(dper) * 1e-3) / 1e9, "peak": hbm_peak,
+                           "unit": "GB/s", "frac": dbytes / (statistics.mean(dper) * 1e-3) / 1e9 / hbm_peak,
+                           "algorithmic_bytes_per_launch": dbytes}}
+    del state, toks
+
+    # ---------------- full mixer (conv4 + L2 + KDA + gate), B=2 x T=32768 ----------------
+    mix = None
+    if not args.quick:
+        Bm, Tm = 2, 32768
+        mi = device_prefill_inputs(Bm * Tm, H, D, 1370002, device, normalise=False, mixer=True)
+        mo = torch.empty(Bm * Tm, H, D, dtype=torch.bfloat16, device=device)
+        mf = torch.empty(Bm, H, D, D, dtype=torch.float32, device=device)
+        mws = torch.empty(lib.kda_mixer_fwd_workspace(Bm * Tm, Bm, H, D, D), dtype=torch.uint8, device=device)
+
+        def mstep(i):
+            kda.mixer_fwd(mi["q"], mi["k"], mi["v"], mi["conv_w"], mi["log_alpha"], mi["beta"], mi["gate"], None,
+                          None, N=Bm, out=mo, final_state=mf, workspace=mws, stream=stream)
+
+        msteps = max(3, min(args.steps, 10))
+        mper, mtot = time_region(mstep, msteps, 2, stream, device)
+        launches += 2 * msteps
+        mtot = max_over_ranks(mtot, device)
+        mbytes = prefill_bytes(Bm * Tm, Bm, with_h0=False, mixer=True)
+        mms = statistics.mean(mper)
+        mix = {"workload": f"full mixer B={Bm} T={Tm} H={H} d={D} (conv4 + L2 + KDA + sigmoid gate)",
+               "ms_per_call": mtot / msteps, "tokens_per_s": job_throughput(Bm * Tm * msteps, world, mtot / 1e3),
+               "roofline": {"bound": "hbm", "achieved": mbytes / (mms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": mbytes / (mms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_launch": mbytes}}
+        del mi, mo, mws
+
+    # ---------------- varlen packed prefill, 64 sequences U[256, 8192] ------------------
+    var = None
+    if not args.quick:
+        rng = np.random.default_rng(I.SEED_BASE + 4)
+        lens = [int(x) for x in rng.integers(256, 8193, 64)]
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=device)
+        TT = int(sum(lens))
+        vi = device_prefill_inputs(TT, H, D, 1370004, device, state_N=len(lens))
+        vo = torch.empty(TT, H, D, dtype=torch.bfloat16, device=device)
+        vf = torch.empty(len(lens), H, D, D, dtype=torch.float32, device=device)
+
+        def vstep(i):
+            kda.chunk_fwd(vi["q"], vi["k"], vi["v"], vi["log_alpha"], vi["beta"], vi["initial_state"], cu,
+                          N=len(lens), out=vo, final_state=vf, workspace=ws, stream=stream)
+
+        vsteps = max(3, min(args.steps, 10))
+        vper, vtot = time_region(vstep, vsteps, 2, stream, device)
+        launches += vsteps
+        vtot = max_over_ranks(vtot, device)
+        vbytes = prefill_bytes(TT, len(lens))
+        vms = statistics.mean(vper)
+        var = {"workload": f"varlen prefill 64 seqs (U[256,8192], {TT} tokens) H={H} d={D}",
+               "ms_per_call": vtot / vsteps, "tokens_per_s": job_throughput(TT * vsteps, world, vtot / 1e3),
+               "roofline": {"bound": "hbm", "achieved": vbytes / (vms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": vbytes / (vms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_launch": vbytes},
+               "tensor_tflops": prefill_tc_flops(TT) / (vms * 1e-3) / 1e12}
+        del vi, vo, vf
+
+    cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded NumPy generator; random inputs, no weights)",
+            "config": {"workload": "KDA chunked prefill B=1 T=4096 H=32 d_k=d_v=128 (bf16 q/k/v, fp32 log_alpha/beta/state)",
+                       "global_batch": world, "seq_len": T1, "heads": H, "head_dim": D, "chunk": CHUNK,
+                       "parallelism": f"replicas x{world} (independent (sequence, head) chains, no collective)",
+                       "l2": f"inputs rotate through {n_sets} device copies ({n_sets * bytes_call / 1e6:.0f} MB > L2)"},
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved_gbs / hbm_peak, "traffic": args.traffic,
+                         "kernel": "kda_prefill_kernel<32>", "algorithmic_bytes_per_launch": bytes_call,
+                         "kernel_us": kern_ms * 1e3, "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src}, burst copy)",
+                         "tensor": {"achieved_tflops": tc_tflops, "peak_tflops": tc_peak,
+                                    "frac": tc_tflops / tc_peak, "flops_per_launch": prefill_tc_flops(T1)}},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "decode": decode, "mixer": mix, "varlen": var,
+            "clocks": clocks, "gpu_launches": launches, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(device)
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------------
+# CPU oracle: the reported baseline and the reference arm
+# ----------------------------------------------------------------------------------
+def oracle_sample(heads: int = 2, T: int = T1):
+    """Times the fp64 oracle on `heads` of the 32 heads over T tokens of the
+    model-shape prefill; returns (token-equivalents/s at H=32, seconds, description)."""
+    from gated_delta_rule_137_b200 import inputs as I
+    from oracle import kda_oracle as O
+    w = I.prefill_model_shape(T)
+    hs = list(range(heads))
+    t0 = time.perf_counter()
+    O.kda_recurrence(w.q[:, hs], w.k[:, hs], w.v[:, hs], w.log_alpha[:, hs], w.beta[:, hs],
+                     w.initial_state[:, hs], w.cu_seqlens)
+    dt = time.perf_counter() - t0
+    tok_equiv = T * heads / H
+    return tok_equiv / dt, dt, f"fp64 NumPy oracle, {heads} of {H} heads x {T} tokens of the B=1 T=4096 workload (scaled to all heads)"
+
+
+def cpu_baseline(args):
+    v, dt, desc = oracle_sample(heads=args.cpu_heads)
+    return {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc, "seconds": dt}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        oracle_sample(heads=1, T=256)
+    per = []
+    for _ in range(args.steps):
+        v, dt, desc = oracle_sample(heads=1, T=1024)
+        per.append(dt)
+    total = sum(per)
+    tok_equiv = args.steps * 1024 * 1 / H
+    value = tok_equiv / total
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded NumPy generator)",
+        "config": {"workload": "KDA chunked prefill B=1 T=4096 H=32 d_k=d_v=128 (bf16 q/k/v, fp32 log_alpha/beta/state)",
+                   "global_batch": 1, "seq_len": T1, "parallelism": "host CPU, 1 core"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": "each step: 1 of 32 heads x the first 1024 tokens (scaled to all heads)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--quick", action="store_true", help="headline and decode only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=32)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch of the prefill kernel from an ncu capture (reported as given)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+"""Python binding of libkda.so — a B200 (sm_100a) implementation of the Kimi Delta
+Attention (KDA) token mixer.
+
+The binding only marshals arguments: torch tensors supply device memory and the
+current CUDA stream, and every step of the computation runs in the library's CUDA
+kernels. There is no CPU fallback: if libkda.so is missing or fails to load, the
+calls raise.
+
+    out, final = chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+    out        = decode_step(q, k, v, log_alpha, beta, state)      # state in place
+    out, final = mixer_fwd(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, ...)
+
+Shapes (token-major, packed): q, k, log_alpha [total_T, H, dk]; v [total_T, H, dv];
+beta [total_T, H]; states [N, H, dk, dv]; cu_seqlens int32 [N+1] (device).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "kda.h")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_RANGE = range(6)
+KDA_DT_F32, KDA_DT_BF16 = 0, 1
+DEVFLAG_BAD_SEQLENS = 0x1
+DEVFLAG_DECAY_RANGE = 0x2
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_WORKSPACE",
+                 4: "KDA_ERR_CUDA", 5: "KDA_ERR_RANGE"}
+
+_vp, _i32, _i64, _sz, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)
+
+_SIGNATURES = {
+    "kda_status_string": (ctypes.c_char_p, [_i32]),
+    "kda_last_error": (ctypes.c_char_p, []),
+    "kda_version": (ctypes.c_char_p, []),
+    "kda_chunk_fwd_workspace": (_sz, [_i64, _i32, _i32, _i32, _i32, _i32]),
+    "kda_chunk_fwd": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
+                             _vp, _vp, _vp, _sz, _vp]),
+    "kda_decode_step": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "kda_mixer_fwd_workspace": (_sz, [_i64, _i32, _i32, _i32, _i32]),
+    "kda_mixer_fwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
+                             _vp, _vp, _vp, _sz, _vp]),
+    "kda_workspace_status": (_i32, [_vp, _vp, _u32p]),
+}
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libkda.so and declare its C signatures. Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"{path} is missing: build it with `python -m gated_delta_rule_137_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def header_functions(path: str = HEADER_PATH) -> list:
+    """Names of the functions include/kda.h declares."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(status: int) -> None:
+    if status != KDA_OK:
+        raise KdaError(status, load_library().kda_last_error().decode())
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return KDA_DT_BF16
+    if t.dtype == torch.float32:
+        return KDA_DT_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return _torch().cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def chunk_fwd_workspace_bytes(total_T: int, N: int, H: int, dk: int, dv: int, dtype_code: int) -> int:
+    return int(load_library().kda_chunk_fwd_workspace(total_T, N, H, dk, dv, dtype_code))
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *, N: Optional[int] = None,
+              out=None, final_state=None, output_final_state: bool = True, workspace=None, stream=None,
+              check_status: bool = False) -> Tuple[object, object]:
+    """Chunked KDA prefill (kda_chunk_fwd). q, k, log_alpha [T, H, dk] or [B, T, H, dk]."""
+    torch = _torch()
+    lib = load_library()
+    if q.dim() == 4:  # fixed-length [B, T, H, d]
+        B, T = q.shape[:2]
+        q, k, v, log_alpha = (x.reshape(B * T, *x.shape[2:]) for x in (q, k, v, log_alpha))
+        beta = beta.reshape(B * T, -1)
+        N = B
+        shape_back = (B, T)
+    else:
+        shape_back = None
+    total_T, H, dk = q.shape
+    dv = v.shape[-1]
+    if N is None:
+        if cu_seqlens is None:
+            raise ValueError("N is needed when cu_seqlens is not given")
+        N = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((total_T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = int(lib.kda_chunk_fwd_workspace(total_T, N, H, dk, dv, dt))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+                             _ptr(cu_seqlens), total_T, N, H, dk, dv, _ptr(out), _ptr(final_state),
+                             _ptr(workspace), workspace.numel(), _stream(stream)))
+    if check_status:
+        workspace_status(workspace, stream)
+    if shape_back is not None:
+        out = out.reshape(*shape_back, H, dv)
+    return out, final_state
+
+
+def decode_step(q, k, v, log_alpha, beta, state, *, out=None, stream=None):
+    """One decode token per (sequence, head); `state` [N, H, dk, dv] fp32 is updated in place."""
+    torch = _torch()
+    lib = load_library()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    _check(lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
+                               _ptr(state), N, H, dk, dv, _ptr(out), _stream(stream)))
+    return out
+
+
+def mixer_fwd(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate=None, initial_state=None, cu_seqlens=None, *,
+              N: Optional[int] = None, out=None, final_state=None, output_final_state: bool = True,
+              workspace=None, stream=None, check_status: bool = False):
+    """Full mixer prefill (kda_mixer_fwd): conv4 -> L2 norm -> KDA -> sigmoid gate."""
+    torch = _torch()
+    lib = load_library()
+    total_T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    if N is None:
+        if cu_seqlens is None:
+            raise ValueError("N is needed when cu_seqlens is not given")
+        N = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((total_T, H, dv), dtype=torch.bfloat16, device=q_raw.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q_raw.device)
+    need = int(lib.kda_mixer_fwd_workspace(total_T, N, H, dk, dv))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q_raw.device)
+    _check(lib.kda_mixer_fwd(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w), _ptr(log_alpha), _ptr(beta),
+                             _ptr(gate), _ptr(initial_state), _ptr(cu_seqlens), total_T, N, H, dk, dv, _ptr(out),
+                             _ptr(final_state), _ptr(workspace), workspace.numel(), _stream(stream)))
+    if check_status:
+        workspace_status(workspace, stream)
+    return out, final_state
+
+
+def workspace_status(workspace, stream=None) -> int:
+    """Reads and clears the device status word; raises KdaError(KDA_ERR_RANGE) if set."""
+    lib = load_library()
+    flags = ctypes.c_uint32(0)
+    st = lib.kda_workspace_status(_ptr(workspace), _stream(stream), ctypes.byref(flags))
+    if st not in (KDA_OK, KDA_ERR_RANGE):
+        _check(st)
+    if st == KDA_ERR_RANGE:
+        raise KdaError(st, f"device status flags 0x{flags.value:08x}")
+    return flags.value

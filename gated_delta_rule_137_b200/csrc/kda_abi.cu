@@ -1,0 +1,276 @@
+// kda_abi.cu — the extern "C" boundary of libkda.so: argument validation on the
+// host, workspace sizing, status strings, and dispatch to the kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "kda_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+kda_status fail(kda_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+kda_status ok() {
+  g_last_error[0] = '\0';
+  return KDA_OK;
+}
+
+kda_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(KDA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(kda_dtype dt) { return dt == KDA_DT_F32 ? 4 : 2; }
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Staging buffers of kda_chunk_fwd when a head dim is below 128 (zero padding in
+// the input dtype; element size es).
+struct StageLayout {
+  size_t q, k, v, la, h0, out, ht, total;
+};
+
+StageLayout stage_layout(int64_t total_T, int N, int H, size_t es) {
+  StageLayout L{};
+  const size_t tok = static_cast<size_t>(total_T) * H * kda::kD;
+  const size_t st = static_cast<size_t>(N) * H * kda::kD * kda::kD * sizeof(float);
+  size_t off = kda::kStatusBytes;
+  L.q = off;   off = kda::align256(off + tok * es);
+  L.k = off;   off = kda::align256(off + tok * es);
+  L.v = off;   off = kda::align256(off + tok * es);
+  L.la = off;  off = kda::align256(off + tok * 4);
+  L.h0 = off;  off = kda::align256(off + st);
+  L.out = off; off = kda::align256(off + tok * es);
+  L.ht = off;  off = kda::align256(off + st);
+  L.total = off;
+  return L;
+}
+
+bool needs_staging(int dk, int dv) { return dk != kda::kD || dv != kda::kD; }
+
+kda_status check_common(int64_t total_T, int N, int H, int dk, int dv) {
+  if (total_T < 0 || total_T > (int64_t{1} << 31) - 1024)
+    return fail(KDA_ERR_INVALID_ARG, "total_T=%lld out of range [0, 2^31-1024]", static_cast<long long>(total_T));
+  if (N < 0) return fail(KDA_ERR_INVALID_ARG, "N=%d must be >= 0", N);
+  if (H < 1 || H > 65535) return fail(KDA_ERR_INVALID_ARG, "H=%d must be in [1, 65535]", H);
+  if (dk < 1 || dk > KDA_MAX_HEAD_DIM || dv < 1 || dv > KDA_MAX_HEAD_DIM)
+    return fail(KDA_ERR_INVALID_ARG, "dk=%d, dv=%d must be in [1, %d]", dk, dv, KDA_MAX_HEAD_DIM);
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(kda_status s) {
+  switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_RANGE: return "KDA_ERR_RANGE";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+const char* kda_last_error(void) { return g_last_error; }
+
+const char* kda_version(void) { return "0.1.0"; }
+
+size_t kda_chunk_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv, kda_dtype qkv_dtype) {
+  if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
+  if (qkv_dtype != KDA_DT_F32 && qkv_dtype != KDA_DT_BF16) return 0;
+  if (!needs_staging(dk, dv)) return kda::kStatusBytes;
+  return stage_layout(total_T, N, H, elem_size(qkv_dtype)).total;
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype qkv_dtype, const float* log_alpha,
+                         const float* beta, const float* initial_state, const int32_t* cu_seqlens, int64_t total_T,
+                         int N, int H, int dk, int dv, void* out, float* final_state, void* workspace,
+                         size_t workspace_bytes, kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  kda_status st = check_common(total_T, N, H, dk, dv);
+  if (st != KDA_OK) return st;
+  if (qkv_dtype != KDA_DT_F32 && qkv_dtype != KDA_DT_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "qkv_dtype=%d is neither KDA_DT_F32 nor KDA_DT_BF16", static_cast<int>(qkv_dtype));
+  if (N == 0) {
+    if (total_T != 0) return fail(KDA_ERR_INVALID_ARG, "N=0 with total_T=%lld", static_cast<long long>(total_T));
+    return ok();
+  }
+  if (!cu_seqlens && total_T % N != 0)
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL but total_T=%lld is not a multiple of N=%d",
+                static_cast<long long>(total_T), N);
+  if (total_T > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
+    return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta and out must be non-NULL");
+  const void* ptrs[] = {q, k, v, log_alpha, beta, initial_state, out, final_state, workspace};
+  const char* names[] = {"q", "k", "v", "log_alpha", "beta", "initial_state", "out", "final_state", "workspace"};
+  for (int i = 0; i < 9; ++i)
+    if (ptrs[i] && !aligned16(ptrs[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+  const size_t es = elem_size(qkv_dtype);
+  const size_t n_out = static_cast<size_t>(total_T) * H * dv * es;
+  const size_t n_st = static_cast<size_t>(N) * H * dk * dv * sizeof(float);
+  if (final_state && initial_state && final_state != initial_state &&
+      ranges_overlap(final_state, n_st, initial_state, n_st))
+    return fail(KDA_ERR_INVALID_ARG, "final_state partially overlaps initial_state");
+  if (ranges_overlap(out, n_out, q, static_cast<size_t>(total_T) * H * dk * es) ||
+      ranges_overlap(out, n_out, k, static_cast<size_t>(total_T) * H * dk * es) ||
+      ranges_overlap(out, n_out, v, static_cast<size_t>(total_T) * H * dv * es) ||
+      ranges_overlap(out, n_out, final_state, n_st) || ranges_overlap(out, n_out, initial_state, n_st))
+    return fail(KDA_ERR_INVALID_ARG, "out overlaps an input or a state buffer");
+  const size_t need = kda_chunk_fwd_workspace(total_T, N, H, dk, dv, qkv_dtype);
+  if (!workspace || workspace_bytes < need)
+    return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? workspace_bytes : 0, need);
+
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+
+  kda::PrefillArgs a{};
+  a.beta = beta;
+  a.cu = cu_seqlens;
+  a.status = status;
+  a.total_T = total_T;
+  a.N = N;
+  a.H = H;
+  a.in_f32 = a.out_f32 = (qkv_dtype == KDA_DT_F32);
+  if (!needs_staging(dk, dv)) {
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.h0 = initial_state;
+    a.out = out; a.ht = final_state;
+    e = kda::launch_prefill_d128(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+    return ok();
+  }
+  const StageLayout L = stage_layout(total_T, N, H, es);
+  a.q = ws + L.q; a.k = ws + L.k; a.v = ws + L.v;
+  a.log_alpha = reinterpret_cast<float*>(ws + L.la);
+  a.h0 = initial_state ? reinterpret_cast<float*>(ws + L.h0) : nullptr;
+  a.out = ws + L.out;
+  a.ht = final_state ? reinterpret_cast<float*>(ws + L.ht) : nullptr;
+  e = kda::launch_stage_in(q, k, v, qkv_dtype == KDA_DT_BF16, log_alpha, initial_state, total_T, N, H, dk, dv,
+                           ws + L.q, ws + L.k, ws + L.v, reinterpret_cast<float*>(ws + L.la),
+                           initial_state ? reinterpret_cast<float*>(ws + L.h0) : nullptr, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "staging kernel launch");
+  e = kda::launch_prefill_d128(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+  e = kda::launch_stage_out(ws + L.out, a.ht, qkv_dtype == KDA_DT_BF16, total_T, N, H, dk, dv, out, final_state,
+                            stream);
+  if (e != cudaSuccess) return cuda_fail(e, "unstaging kernel launch");
+  return ok();
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, kda_dtype qkv_dtype, const float* log_alpha,
+                           const float* beta, float* state, int N, int H, int dk, int dv, void* out,
+                           kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  kda_status st = check_common(0, N, H, dk, dv);
+  if (st != KDA_OK) return st;
+  if (qkv_dtype != KDA_DT_F32 && qkv_dtype != KDA_DT_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "qkv_dtype=%d is neither KDA_DT_F32 nor KDA_DT_BF16", static_cast<int>(qkv_dtype));
+  if (dv % 4 != 0) return fail(KDA_ERR_UNSUPPORTED, "decode needs dv %% 4 == 0 (dv=%d)", dv);
+  if (N == 0) return ok();
+  if (!q || !k || !v || !log_alpha || !beta || !state || !out)
+    return fail(KDA_ERR_INVALID_ARG, "all pointers must be non-NULL");
+  if (!aligned16(state) || !aligned16(out)) return fail(KDA_ERR_INVALID_ARG, "state and out must be 16-byte aligned");
+  const void* small[] = {q, k, v, log_alpha, beta};
+  for (const void* p : small)
+    if (reinterpret_cast<uintptr_t>(p) & 3u) return fail(KDA_ERR_INVALID_ARG, "q/k/v/log_alpha/beta must be 4-byte aligned");
+  const size_t n_st = static_cast<size_t>(N) * H * dk * dv * sizeof(float);
+  const size_t n_out = static_cast<size_t>(N) * H * dv * elem_size(qkv_dtype);
+  if (ranges_overlap(out, n_out, state, n_st)) return fail(KDA_ERR_INVALID_ARG, "out overlaps state");
+  cudaError_t e = kda::launch_decode_step(q, k, v, qkv_dtype == KDA_DT_BF16, log_alpha, beta, state, N, H, dk, dv,
+                                          out, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  return ok();
+}
+
+size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv) {
+  if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
+  if (dk != kda::kD || dv != kda::kD) return 0;
+  const size_t tok = static_cast<size_t>(total_T) * H * kda::kD * sizeof(float);
+  return kda::kStatusBytes + 3 * kda::align256(tok);
+}
+
+kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                         const float* log_alpha, const float* beta, const void* gate, const float* initial_state,
+                         const int32_t* cu_seqlens, int64_t total_T, int N, int H, int dk, int dv, void* out,
+                         float* final_state, void* workspace, size_t workspace_bytes, kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  kda_status st = check_common(total_T, N, H, dk, dv);
+  if (st != KDA_OK) return st;
+  if (dk != kda::kD || dv != kda::kD)
+    return fail(KDA_ERR_UNSUPPORTED, "the fused mixer is built for dk = dv = 128 (got %d, %d)", dk, dv);
+  if (N == 0) {
+    if (total_T != 0) return fail(KDA_ERR_INVALID_ARG, "N=0 with total_T=%lld", static_cast<long long>(total_T));
+    return ok();
+  }
+  if (!cu_seqlens && total_T % N != 0)
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL but total_T=%lld is not a multiple of N=%d",
+                static_cast<long long>(total_T), N);
+  if (total_T > 0 && (!q_raw || !k_raw || !v_raw || !conv_w || !log_alpha || !beta || !out))
+    return fail(KDA_ERR_INVALID_ARG, "q_raw, k_raw, v_raw, conv_w, log_alpha, beta and out must be non-NULL");
+  const void* ptrs[] = {q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, out, final_state, workspace};
+  const char* names[] = {"q_raw", "k_raw", "v_raw", "conv_w", "log_alpha", "beta", "gate",
+                         "initial_state", "out", "final_state", "workspace"};
+  for (int i = 0; i < 11; ++i)
+    if (ptrs[i] && !aligned16(ptrs[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+  const size_t n_st = static_cast<size_t>(N) * H * dk * dv * sizeof(float);
+  if (final_state && initial_state && final_state != initial_state &&
+      ranges_overlap(final_state, n_st, initial_state, n_st))
+    return fail(KDA_ERR_INVALID_ARG, "final_state partially overlaps initial_state");
+  const size_t need = kda_mixer_fwd_workspace(total_T, N, H, dk, dv);
+  if (!workspace || workspace_bytes < need)
+    return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? workspace_bytes : 0, need);
+
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  const size_t tok = kda::align256(static_cast<size_t>(total_T) * H * kda::kD * sizeof(float));
+  char* qn = ws + kda::kStatusBytes;
+  char* kn = qn + tok;
+  char* vn = kn + tok;
+  e = kda::launch_conv_l2(q_raw, k_raw, v_raw, conv_w, cu_seqlens, total_T, N, H, kda::kD, qn, kn, vn, status, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "conv/L2 kernel launch");
+  kda::PrefillArgs a{};
+  a.q = qn; a.k = kn; a.v = vn; a.log_alpha = log_alpha; a.beta = beta; a.h0 = initial_state; a.cu = cu_seqlens;
+  a.gate = gate; a.out = out; a.ht = final_state; a.status = status; a.total_T = total_T; a.N = N; a.H = H;
+  a.in_f32 = true;   // conv/L2 outputs stay fp32
+  a.out_f32 = false;
+  e = kda::launch_prefill_d128(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+  return ok();
+}
+
+kda_status kda_workspace_status(void* workspace, kda_stream_t stream_, uint32_t* flags) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!workspace) return fail(KDA_ERR_INVALID_ARG, "workspace is NULL");
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(word), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  if (flags) *flags = word;
+  if (word) return fail(KDA_ERR_RANGE, "device status word 0x%08x", word);
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+// kda_internal.h — declarations shared by the library's translation units (not
+// part of the public C ABI, which is include/kda.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/kda.h"
+#include "sm100_ptx.cuh"
+
+namespace kda {
+
+// Head dimension the tensor-core prefill kernel is built for; other sizes are
+// zero-padded to it (exact: padded channels carry log_alpha = 0 and zero data).
+constexpr int kD = 128;
+// Tokens per chunk of the chunked prefill.
+constexpr int kChunk = 64;
+
+// Workspace layout of kda_chunk_fwd / kda_mixer_fwd: the first 256 bytes hold the
+// device status word; staging buffers (if any) follow at 256-byte boundaries.
+constexpr size_t kStatusBytes = 256;
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct PrefillArgs {
+  const void* q;          // [total_T, H, 128], bf16 or fp32 (in_f32)
+  const void* k;          // [total_T, H, 128]
+  const void* v;          // [total_T, H, 128]
+  const float* log_alpha; // fp32 [total_T, H, 128]
+  const float* beta;      // fp32 [total_T, H]
+  const float* h0;        // fp32 [N, H, 128, 128] or null
+  const int32_t* cu;      // int32 [N+1] or null (equal lengths)
+  const void* gate;       // bf16 [total_T, H, 128] or null (sigmoid output gate)
+  void* out;              // [total_T, H, 128], bf16 or fp32 (out_f32)
+  float* ht;              // fp32 [N, H, 128, 128] or null
+  uint32_t* status;       // device status word
+  int64_t total_T;
+  int N, H;
+  bool in_f32;            // q, k, v are fp32 (else bf16)
+  bool out_f32;           // out is fp32 (else bf16)
+};
+
+cudaError_t launch_decode_step(const void* q, const void* k, const void* v, bool bf16, const float* log_alpha,
+                               const float* beta, float* state, int N, int H, int dk, int dv, void* out,
+                               cudaStream_t stream);
+
+// Tensor-core chunked prefill on d = 128 operands (bf16 or fp32 q/k/v/out).
+cudaError_t launch_prefill_d128(const PrefillArgs& a, cudaStream_t stream);
+
+// Staging for head dims below 128: zero-pads q/k/v (in their own dtype), log_alpha
+// and the initial state to d = 128, and copies the results back.
+cudaError_t launch_stage_in(const void* q, const void* k, const void* v, bool bf16, const float* log_alpha,
+                            const float* h0, int64_t total_T, int N, int H, int dk, int dv, void* q_p, void* k_p,
+                            void* v_p, float* la_p, float* h0_p, cudaStream_t stream);
+cudaError_t launch_stage_out(const void* out_p, const float* ht_p, bool bf16, int64_t total_T, int N, int H, int dk,
+                             int dv, void* out, float* ht, cudaStream_t stream);
+
+// Pre-stage of the full mixer: causal depthwise conv (width 4) on q, k, v, L2 norm
+// of q and k, written in fp32 (no intermediate rounding).
+cudaError_t launch_conv_l2(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                           const int32_t* cu, int64_t total_T, int N, int H, int d, void* q_o, void* k_o, void* v_o,
+                           uint32_t* status, cudaStream_t stream);
+
+}  // namespace kda

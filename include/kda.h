@@ -1,0 +1,184 @@
+/*
+ * kda.h — C ABI of libkda.so, a B200 (sm_100a) implementation of the Kimi Delta
+ * Attention (KDA) token mixer.
+ *
+ * The operation (page "Ling-3.0-flash: a 124B open MoE that runs like a 5B and
+ * reaches for 1M tokens", section "KDA: constant-size memory over a very long
+ * context"): a gated delta-rule linear attention that keeps one fixed d_k x d_v
+ * state S per head. Each token decays S per key channel (alpha_t, the erase),
+ * then writes the key/value association with the delta rule (beta_t k_t v_t^T),
+ * and the query reads the state. The displayed equation is missing from that
+ * page; the library implements
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t                      alpha_t = exp(log_alpha_t) per key channel
+ *
+ * Head geometry of the model (page "Ling 3.0 Flash", table "Every architecture
+ * field"): 32 key heads = 32 value heads, head dim 128, short-conv kernel 4.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named "device" are CUDA device memory owned by the caller; the
+ *   library never frees or retains them past the call. Nothing persistent is
+ *   allocated: scratch comes from the caller's `workspace`.
+ * - Layouts are row-major, last index fastest, token-major packed:
+ *     q, k, log_alpha   [total_T, H, dk]      v, out, gate   [total_T, H, dv]
+ *     beta              [total_T, H]          states         [N, H, dk, dv]
+ *   Fixed-length batches B x T are the same memory with total_T = B*T, N = B.
+ * - Sequences: `cu_seqlens` is a device int32 array [N+1] with cu[0] = 0,
+ *   cu[N] = total_T and cu[n] <= cu[n+1] (zero-length sequences allowed). NULL
+ *   means N equal sequences of total_T / N tokens.
+ * - No query scale is applied (o is linear in q: pre-scale q if wanted).
+ * - All calls are asynchronous on `stream` (0 = legacy default stream). Argument
+ *   checks are synchronous on the host and return before any launch. A launch
+ *   failure returns KDA_ERR_CUDA. The library never aborts, traps or prints.
+ * - Problems that only the device can see (a cu_seqlens that is not
+ *   non-decreasing or overruns total_T; a chunk whose per-channel decay exceeds
+ *   the documented range) set bits in a status word held in `workspace`; the
+ *   affected (sequence, head) pairs are skipped and their outputs left
+ *   unspecified. Read the word with kda_workspace_status() after the stream
+ *   has run the call.
+ * - Thread safety: calls may be issued from several host threads; the message
+ *   returned by kda_last_error() is thread-local.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kda_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1, /* NULL pointer, bad size, dtype, or misalignment   */
+  KDA_ERR_UNSUPPORTED = 2, /* valid request outside what this build implements  */
+  KDA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than the query returned  */
+  KDA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed        */
+  KDA_ERR_RANGE = 5        /* device-detected range violation (status word set)  */
+} kda_status;
+
+typedef enum { KDA_DT_F32 = 0, KDA_DT_BF16 = 1 } kda_dtype;
+
+/* Bits of the device status word (kda_workspace_status). */
+#define KDA_DEVFLAG_BAD_SEQLENS 0x1u  /* cu_seqlens not monotone / out of range */
+#define KDA_DEVFLAG_DECAY_RANGE 0x2u  /* chunk decay beyond the supported range  */
+
+/* Largest head dimensions this build accepts (d_k, d_v <= 128; the model uses 128). */
+#define KDA_MAX_HEAD_DIM 128
+
+/* Human-readable name of a status code (static string). */
+KDA_API const char* kda_status_string(kda_status s);
+
+/* Detail of the last non-OK status returned on this host thread ("" if none). */
+KDA_API const char* kda_last_error(void);
+
+/* Library version, "major.minor.patch". */
+KDA_API const char* kda_version(void);
+
+/*
+ * Workspace, in bytes, that kda_chunk_fwd needs for these sizes (a multiple of
+ * 256; never 0, the status word always lives there). Returns 0 for sizes the
+ * library rejects.
+ */
+KDA_API size_t kda_chunk_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv, kda_dtype qkv_dtype);
+
+/*
+ * Chunked prefill: runs the recurrence above over every packed sequence.
+ *
+ * Defining passage: the KDA section cited at the top (the gated decay, the
+ * delta-rule write, the read with the query, a state whose size does not
+ * depend on T). The chunk-parallel form used on the device (64-token chunks,
+ * the WY/UT triangular solve, tensor-core GEMMs, fp32 state carried between
+ * chunks) computes the same result up to rounding.
+ *
+ *   q, k       device, [total_T, H, dk], dtype qkv_dtype (bf16 or fp32)
+ *   v          device, [total_T, H, dv], dtype qkv_dtype
+ *   log_alpha  device fp32 [total_T, H, dk]: natural log of the per-channel
+ *              decay, <= 0. Supported range: the decay summed over any 64-token
+ *              chunk (aligned to the sequence start) must stay within 80 nats per
+ *              channel; beyond it KDA_DEVFLAG_DECAY_RANGE is set.
+ *   beta       device fp32 [total_T, H], the write strength (sigmoid output).
+ *   initial_state  device fp32 [N, H, dk, dv] or NULL (zero state).
+ *   cu_seqlens device int32 [N+1] or NULL (equal lengths; total_T % N == 0).
+ *   out        device [total_T, H, dv], dtype qkv_dtype; rows of zero-length
+ *              sequences are not written.
+ *   final_state device fp32 [N, H, dk, dv] or NULL (not written). It may alias
+ *              initial_state exactly (same pointer); partial overlap is an error.
+ *   workspace  device, >= kda_chunk_fwd_workspace(...) bytes, 256-byte aligned;
+ *              its contents on entry are ignored.
+ *
+ * Alignment: every tensor pointer must be 16-byte aligned. Returns KDA_OK once
+ * the work is enqueued.
+ */
+KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype qkv_dtype,
+                         const float* log_alpha, const float* beta, const float* initial_state,
+                         const int32_t* cu_seqlens, int64_t total_T, int N, int H, int dk, int dv,
+                         void* out, float* final_state, void* workspace, size_t workspace_bytes,
+                         kda_stream_t stream);
+
+/*
+ * Decode step: one token per (sequence, head), state updated in place.
+ *
+ * Defining passage: the same KDA section (each token updates the fixed-size
+ * state in place; decode does not grow with context). Per (n, h):
+ *     S' = Diag(exp(log_alpha)) S;  u = beta (v - S'^T k);  S <- S' + k u^T;
+ *     out = S^T q  (= S'^T q + u (k . q)).
+ *
+ *   q, k       device [N, H, dk], dtype qkv_dtype;  v device [N, H, dv]
+ *   log_alpha  device fp32 [N, H, dk];  beta device fp32 [N, H]
+ *   state      device fp32 [N, H, dk, dv], read and overwritten in place
+ *   out        device [N, H, dv], dtype qkv_dtype; must not overlap state
+ * Alignment: state and out 16-byte aligned; other pointers 4-byte aligned.
+ */
+KDA_API kda_status kda_decode_step(const void* q, const void* k, const void* v, kda_dtype qkv_dtype,
+                           const float* log_alpha, const float* beta, float* state,
+                           int N, int H, int dk, int dv, void* out, kda_stream_t stream);
+
+/* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes). */
+KDA_API size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv);
+
+/*
+ * Full mixer prefill: the KDA panel of the same article — q and k pass through
+ * a short causal depthwise conv and an L2 norm, v through a conv, then the KDA
+ * recurrence, then a sigmoid output gate.
+ *   conv (kernel 4, page "Ling 3.0 Flash", field short_conv_kernel_size):
+ *     y[t, c] = sum_{j=0..3} w[c, j] x[t-3+j, c], zero history at each sequence
+ *     start, no bias, identity activation;
+ *   L2 norm per (token, head) of q and k: x / sqrt(sum x^2 + 1e-6), in fp32;
+ *   gate: out = o * sigmoid(g) (skipped when gate is NULL).
+ *
+ *   q_raw, k_raw  device bf16 [total_T, H, dk];  v_raw device bf16 [total_T, H, dv]
+ *   conv_w        device fp32 [3, H*d, 4] (q, k, v weights; requires dk == dv = d)
+ *   gate          device bf16 [total_T, H, dv] or NULL
+ *   log_alpha, beta, initial_state, cu_seqlens, out (bf16), final_state,
+ *   workspace, stream: as for kda_chunk_fwd.
+ */
+KDA_API kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                         const float* log_alpha, const float* beta, const void* gate,
+                         const float* initial_state, const int32_t* cu_seqlens, int64_t total_T,
+                         int N, int H, int dk, int dv, void* out, float* final_state,
+                         void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * Reads the device status word kept in `workspace` (KDA_DEVFLAG_* bits) after
+ * synchronising `stream`, and clears it. Returns KDA_ERR_RANGE when any bit
+ * was set, KDA_OK otherwise; *flags (if not NULL) receives the bits.
+ */
+KDA_API kda_status kda_workspace_status(void* workspace, kda_stream_t stream, uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,130 @@
+"""The C-ABI library: it loads, exports every function include/kda.h declares, and
+rejects bad arguments on the host before touching the GPU (CPU tests), plus
+device-side error paths (GPU tests)."""
+import ctypes
+import subprocess
+
+import numpy as np
+import pytest
+
+import gated_delta_rule_137_b200 as kda
+
+FAKE = 0x10000  # 16-byte aligned non-null address; never dereferenced by host checks
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_137_b200 import build
+    build.build()
+    return kda.load_library()
+
+
+def test_exports_match_header(lib):
+    declared = kda.header_functions()
+    assert set(declared) >= {"kda_chunk_fwd", "kda_decode_step", "kda_mixer_fwd", "kda_chunk_fwd_workspace",
+                             "kda_mixer_fwd_workspace", "kda_workspace_status", "kda_status_string",
+                             "kda_last_error", "kda_version"}
+    out = subprocess.run(["nm", "-D", "--defined-only", kda.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [f for f in declared if f not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    # nothing else of ours leaks out of the library
+    ours = {s for s in exported if s.startswith("kda")}
+    assert ours == set(declared)
+    for f in declared:
+        assert getattr(lib, f) is not None
+
+
+def test_status_strings(lib):
+    for code, name in [(0, b"KDA_OK"), (1, b"KDA_ERR_INVALID_ARG"), (2, b"KDA_ERR_UNSUPPORTED"),
+                       (3, b"KDA_ERR_WORKSPACE"), (4, b"KDA_ERR_CUDA"), (5, b"KDA_ERR_RANGE")]:
+        assert lib.kda_status_string(code) == name
+    assert lib.kda_version().decode().count(".") == 2
+
+
+def test_workspace_query(lib):
+    ws = lib.kda_chunk_fwd_workspace(4096, 1, 32, 128, 128, kda.KDA_DT_BF16)
+    assert ws >= 4 and ws % 256 == 0
+    small = lib.kda_chunk_fwd_workspace(64, 1, 2, 16, 16, kda.KDA_DT_F32)
+    assert small > ws  # staging buffers for fp32 / d < 128
+    assert lib.kda_chunk_fwd_workspace(64, 1, 2, 0, 16, kda.KDA_DT_F32) == 0
+    assert lib.kda_chunk_fwd_workspace(64, 1, 2, 129, 16, kda.KDA_DT_BF16) == 0
+    assert lib.kda_chunk_fwd_workspace(64, 1, 2, 16, 16, 7) == 0
+    assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 128, 128) >= 3 * 1000 * 32 * 128 * 2
+    assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 64, 64) == 0
+
+
+def _chunk(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=kda.KDA_DT_BF16, la=FAKE, beta=FAKE, h0=None, cu=None, total_T=128, N=1,
+             H=2, dk=128, dv=128, out=FAKE * 2, ht=None, ws=FAKE * 3, ws_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return lib.kda_chunk_fwd(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"], a["h0"], a["cu"], a["total_T"],
+                             a["N"], a["H"], a["dk"], a["dv"], a["out"], a["ht"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(dk=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(dv=129), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(total_T=-5), kda.KDA_ERR_INVALID_ARG),
+    (dict(dt=3), kda.KDA_ERR_INVALID_ARG),
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(out=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(beta=FAKE + 4), kda.KDA_ERR_INVALID_ARG),           # misaligned
+    (dict(N=3, total_T=128), kda.KDA_ERR_INVALID_ARG),        # equal lengths need T % N == 0
+    (dict(N=0, total_T=64), kda.KDA_ERR_INVALID_ARG),
+    (dict(cu=FAKE + 2), kda.KDA_ERR_INVALID_ARG),             # cu_seqlens not 4-byte aligned
+    (dict(ws=None), kda.KDA_ERR_WORKSPACE),
+    (dict(ws_bytes=16), kda.KDA_ERR_WORKSPACE),
+    (dict(h0=FAKE * 8, ht=FAKE * 8 + 1024), kda.KDA_ERR_INVALID_ARG),  # partial state overlap
+    (dict(out=FAKE), kda.KDA_ERR_INVALID_ARG),                # out aliases q
+])
+def test_chunk_fwd_rejects_bad_arguments(lib, bad, status):
+    assert _chunk(lib, **bad) == status
+    assert lib.kda_last_error()  # a message explains it
+
+
+def test_chunk_fwd_empty_batch_is_a_no_op(lib):
+    assert _chunk(lib, N=0, total_T=0) == kda.KDA_OK
+    assert lib.kda_last_error() == b""
+
+
+def test_decode_rejects_bad_arguments(lib):
+    args = [FAKE, FAKE, FAKE, kda.KDA_DT_BF16, FAKE, FAKE, FAKE * 4, 4, 2, 128, 128, FAKE * 16, None]
+    bad = list(args); bad[9] = 0
+    assert lib.kda_decode_step(*bad) == kda.KDA_ERR_INVALID_ARG
+    bad = list(args); bad[10] = 30  # dv not a multiple of 4
+    assert lib.kda_decode_step(*bad) == kda.KDA_ERR_UNSUPPORTED
+    bad = list(args); bad[6] = FAKE * 4 + 8  # state misaligned
+    assert lib.kda_decode_step(*bad) == kda.KDA_ERR_INVALID_ARG
+    bad = list(args); bad[11] = FAKE * 4  # out overlaps state
+    assert lib.kda_decode_step(*bad) == kda.KDA_ERR_INVALID_ARG
+    bad = list(args); bad[0] = None
+    assert lib.kda_decode_step(*bad) == kda.KDA_ERR_INVALID_ARG
+    ok = list(args); ok[7] = 0  # N = 0: nothing to do
+    assert lib.kda_decode_step(*ok) == kda.KDA_OK
+
+
+def test_mixer_rejects_bad_arguments(lib):
+    base = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 128, 1, 2, 128, 128, FAKE * 2, None, FAKE * 3,
+            1 << 24, None]
+    bad = list(base); bad[12] = 64; bad[13] = 64
+    assert lib.kda_mixer_fwd(*bad) == kda.KDA_ERR_UNSUPPORTED
+    bad = list(base); bad[3] = None
+    assert lib.kda_mixer_fwd(*bad) == kda.KDA_ERR_INVALID_ARG
+    bad = list(base); bad[17] = 100
+    assert lib.kda_mixer_fwd(*bad) == kda.KDA_ERR_WORKSPACE
+    assert lib.kda_workspace_status(None, None, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    import importlib
+    mod = importlib.import_module("gated_delta_rule_137_b200")
+    saved = mod._lib
+    try:
+        mod._lib = None
+        with pytest.raises(OSError):
+            mod.load_library(str(tmp_path / "nope.so"))
+    finally:
+        mod._lib = saved

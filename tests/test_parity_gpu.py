@@ -1,0 +1,261 @@
+"""GPU parity: libkda.so (through the C ABI) against the fp64 oracle on the same
+seeded inputs. Small cases are compared element by element; the full-size
+workloads are compared on sampled (sequence, head) chains that the oracle runs
+in full. Tolerances: prefill max|err| <= 2e-2 * RMS per tensor; decode fp32
+state max|err| <= 1e-4 * max|ref| (bf16 outputs also get their rounding)."""
+import numpy as np
+import pytest
+
+from gated_delta_rule_137_b200 import inputs as I
+from oracle import kda_oracle as O
+from tests.helpers import (assert_decode_out_close, assert_decode_state_close, assert_prefill_close, to_device,
+                           to_host)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kda():
+    import torch
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    from gated_delta_rule_137_b200 import build
+    build.build()
+    import gated_delta_rule_137_b200 as m
+    m.load_library()
+    return m
+
+
+def _upload(w):
+    dt = w.qkv_dtype
+    return dict(q=to_device(w.q, dt), k=to_device(w.k, dt), v=to_device(w.v, dt),
+                log_alpha=to_device(w.log_alpha, "f32"), beta=to_device(w.beta, "f32"),
+                initial_state=None if w.initial_state is None else to_device(w.initial_state, "f32"),
+                cu_seqlens=to_device(w.cu_seqlens, "i32"))
+
+
+def _run_prefill(kda, w, varlen=True):
+    import torch
+    d = _upload(w)
+    out, fin = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                             d["cu_seqlens"] if varlen else None, N=w.N, check_status=True)
+    torch.cuda.synchronize()
+    return to_host(out), to_host(fin)
+
+
+def _oracle_heads(w, heads):
+    hs = list(heads)
+    s0 = None if w.initial_state is None else w.initial_state[:, hs]
+    return O.kda_recurrence(w.q[:, hs], w.k[:, hs], w.v[:, hs], w.log_alpha[:, hs], w.beta[:, hs], s0, w.cu_seqlens)
+
+
+# --------------------------------------------------------------------------- decode
+
+def test_decode_small_bf16(kda):
+    import torch
+    w = I.make_decode(3, 2, 128, 128, 5, seed=11)
+    st = to_device(w.state, "f32")
+    outs = []
+    for s in range(w.steps):
+        outs.append(to_host(kda.decode_step(to_device(w.q[s], "bf16"), to_device(w.k[s], "bf16"),
+                                            to_device(w.v[s], "bf16"), to_device(w.log_alpha[s], "f32"),
+                                            to_device(w.beta[s], "f32"), st)))
+    torch.cuda.synchronize()
+    ref_o, ref_s = O.kda_decode_steps(w.q, w.k, w.v, w.log_alpha, w.beta, w.state)
+    assert_decode_out_close(np.stack(outs), ref_o, "decode out")
+    assert_decode_state_close(to_host(st), ref_s, "decode state")
+
+
+def test_decode_small_dims_f32(kda):
+    import torch
+    rng = np.random.default_rng(12)
+    N, H, dk, dv, steps = 2, 3, 16, 8, 4
+    q = rng.standard_normal((steps, N, H, dk)).astype(np.float32)
+    k = (rng.standard_normal((steps, N, H, dk)) / 4).astype(np.float32)
+    v = rng.standard_normal((steps, N, H, dv)).astype(np.float32)
+    la = (-rng.random((steps, N, H, dk)) / 4).astype(np.float32)
+    b = rng.random((steps, N, H)).astype(np.float32)
+    s0 = rng.standard_normal((N, H, dk, dv)).astype(np.float32)
+    st = to_device(s0, "f32")
+    outs = []
+    for s in range(steps):
+        outs.append(to_host(kda.decode_step(to_device(q[s], "f32"), to_device(k[s], "f32"), to_device(v[s], "f32"),
+                                            to_device(la[s], "f32"), to_device(b[s], "f32"), st)))
+    torch.cuda.synchronize()
+    ref_o, ref_s = O.kda_decode_steps(q, k, v, la, b, s0)
+    assert_decode_state_close(np.stack(outs), ref_o, "decode out (fp32)")
+    assert_decode_state_close(to_host(st), ref_s, "decode state (fp32)")
+
+
+def test_decode_model_shape_64_steps(kda):
+    """256 sequences x 32 heads x 128 x 128 fp32 state in place, 64 consecutive steps;
+    the oracle follows every 32nd sequence (all heads, all steps)."""
+    import torch
+    w = I.decode_batch()
+    st = to_device(w.state, "f32")
+    subset = np.arange(0, w.N, 32)
+    outs = []
+    for s in range(w.steps):
+        o = kda.decode_step(to_device(w.q[s], "bf16"), to_device(w.k[s], "bf16"), to_device(w.v[s], "bf16"),
+                            to_device(w.log_alpha[s], "f32"), to_device(w.beta[s], "f32"), st)
+        outs.append(to_host(o[torch.as_tensor(subset, device=o.device)]))
+    torch.cuda.synchronize()
+    ref_o, ref_s = O.kda_decode_steps(w.q, w.k, w.v, w.log_alpha, w.beta, w.state, seq_subset=subset)
+    assert_decode_out_close(np.stack(outs), ref_o, "decode out")
+    assert_decode_state_close(to_host(st)[subset], ref_s, "decode state")
+
+
+# --------------------------------------------------------------------------- prefill
+
+def test_prefill_tiny_fp32_d16(kda):
+    """B=1, T=64, H=2, d=16 fp32 (zero-padded to the d=128 kernel), chunk-aligned."""
+    w = I.tiny_recurrence()
+    out, fin = _run_prefill(kda, w, varlen=False)
+    ro, rf = O.kda_recurrence(w.q, w.k, w.v, w.log_alpha, w.beta, None, w.cu_seqlens)
+    assert_prefill_close(out, ro, "out", stored_bf16=False)
+    assert_prefill_close(fin, rf, "final_state")
+
+
+@pytest.mark.parametrize("lens,H,dk,dv,dtype", [
+    ([200], 2, 128, 128, "bf16"),                 # ragged tail, 32-column slices
+    ([64, 1, 130, 0, 63, 129], 3, 128, 128, "bf16"),  # varlen, empty and 1-token sequences
+    ([150], 1, 128, 128, "f32"),                  # fp32 q/k/v through the staging path
+    ([70, 33], 2, 64, 32, "bf16"),                # dk, dv below 128 (zero padding)
+    ([96] * 4, 25, 128, 128, "bf16"),             # 100 chains -> 64-column slices
+    ([70] * 10, 32, 128, 128, "bf16"),            # 320 chains -> full 128-column CTAs
+])
+def test_prefill_small_cases(kda, lens, H, dk, dv, dtype):
+    w = I.make_prefill(lens, H, dk, dv, seed=sum(lens) + H, qkv_dtype=dtype)
+    out, fin = _run_prefill(kda, w)
+    ro, rf = O.kda_recurrence(w.q, w.k, w.v, w.log_alpha, w.beta, w.initial_state, w.cu_seqlens)
+    assert_prefill_close(out, ro, "out", stored_bf16=(dtype == "bf16"))
+    assert_prefill_close(fin, rf, "final_state")
+
+
+def test_prefill_model_shape_sampled_heads(kda):
+    """B=1, T=4096, H=32, d=128 bf16 with N(0, 0.02^2) initial state; oracle on 4 heads."""
+    w = I.prefill_model_shape()
+    out, fin = _run_prefill(kda, w, varlen=False)
+    heads = [0, 11, 22, 31]
+    ro, rf = _oracle_heads(w, heads)
+    assert_prefill_close(out[:, heads], ro, "out", stored_bf16=True)
+    assert_prefill_close(fin[:, heads], rf, "final_state")
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(fin))
+
+
+def test_prefill_varlen_sampled(kda):
+    """64 packed sequences, lengths U[256, 8192], per-sequence initial states."""
+    w = I.varlen_prefill()
+    out, fin = _run_prefill(kda, w)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(fin))
+    lens = np.diff(w.cu_seqlens)
+    picks = [int(np.argmin(lens)), int(np.argmax(lens)), 17]
+    for n, h in zip(picks, [5, 30, 12]):
+        s, e = int(w.cu_seqlens[n]), int(w.cu_seqlens[n + 1])
+        ro, rf = O.kda_recurrence(w.q[s:e, h:h + 1], w.k[s:e, h:h + 1], w.v[s:e, h:h + 1],
+                                  w.log_alpha[s:e, h:h + 1], w.beta[s:e, h:h + 1],
+                                  w.initial_state[n:n + 1, h:h + 1], np.array([0, e - s]))
+        assert_prefill_close(out[s:e, h:h + 1], ro, f"out seq {n} head {h}", stored_bf16=True)
+        assert_prefill_close(fin[n:n + 1, h:h + 1], rf, f"final seq {n} head {h}")
+
+
+def test_prefill_split_and_state_alias(kda):
+    """run(T) == run(T1) then run(T - T1) from the carried state, with final_state
+    written over initial_state in place; and prefill then one decode step equals
+    the prefill of one more token."""
+    import torch
+    w = I.make_prefill([301], 4, 128, 128, seed=5)
+    d = _upload(w)
+    T, T1 = 300, 100
+    part = lambda x, a, b: x[a:b].contiguous()
+    ro, rf = O.kda_recurrence(w.q[:T], w.k[:T], w.v[:T], w.log_alpha[:T], w.beta[:T], w.initial_state,
+                              np.array([0, T]))
+    out, fin = kda.chunk_fwd(part(d["q"], 0, T), part(d["k"], 0, T), part(d["v"], 0, T),
+                             part(d["log_alpha"], 0, T), part(d["beta"], 0, T), d["initial_state"], None, N=1)
+    st = d["initial_state"].clone()
+    outs = []
+    for a, b in ((0, T1), (T1, T)):
+        o, _ = kda.chunk_fwd(part(d["q"], a, b), part(d["k"], a, b), part(d["v"], a, b),
+                             part(d["log_alpha"], a, b), part(d["beta"], a, b), st, None, N=1, final_state=st)
+        outs.append(to_host(o))
+    torch.cuda.synchronize()
+    assert_prefill_close(to_host(out), ro, "whole out", stored_bf16=True)
+    assert_prefill_close(to_host(fin), rf, "whole final")
+    assert_prefill_close(np.concatenate(outs), ro, "split out", stored_bf16=True)
+    assert_prefill_close(to_host(st), rf, "split final (in place)")
+    # one more token through the decode kernel, from the prefill's final state
+    ro2, rf2 = O.kda_recurrence(w.q, w.k, w.v, w.log_alpha, w.beta, w.initial_state, w.cu_seqlens)
+    sl = slice(T, T + 1)  # one sequence (N=1) of H=4 heads
+    od = kda.decode_step(d["q"][sl], d["k"][sl], d["v"][sl], d["log_alpha"][sl], d["beta"][sl], fin)
+    torch.cuda.synchronize()
+    assert_prefill_close(to_host(od)[0], ro2[T], "decode after prefill", stored_bf16=True)
+    assert_prefill_close(to_host(fin), rf2, "state after decode")
+
+
+def test_prefill_zero_tokens_copies_state(kda):
+    import torch
+    s0 = torch.randn(2, 3, 128, 128, device="cuda")
+    e = torch.empty(0, 3, 128, device="cuda", dtype=torch.bfloat16)
+    la = torch.empty(0, 3, 128, device="cuda")
+    b = torch.empty(0, 3, device="cuda")
+    cu = torch.zeros(3, dtype=torch.int32, device="cuda")
+    out, fin = kda.chunk_fwd(e, e, e, la, b, s0, cu, N=2)
+    torch.cuda.synchronize()
+    assert torch.equal(fin, s0)
+
+
+def test_device_status_flags(kda):
+    import torch
+    w = I.make_prefill([100, 100], 2, 128, 128, seed=9)
+    d = _upload(w)
+    bad_cu = torch.tensor([0, 150, 120], dtype=torch.int32, device="cuda")  # not monotone
+    with pytest.raises(kda.KdaError):
+        kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, bad_cu, N=2, check_status=True)
+    strong = d["log_alpha"] * 0 - 3.0  # 64 tokens x 3 nats > the supported chunk range
+    with pytest.raises(kda.KdaError):
+        kda.chunk_fwd(d["q"], d["k"], d["v"], strong, d["beta"], None, d["cu_seqlens"], N=2, check_status=True)
+    # a valid call afterwards reports a clean status
+    kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, d["cu_seqlens"], N=2, check_status=True)
+
+
+# --------------------------------------------------------------------------- mixer
+
+def _mixer_oracle_heads(w, heads):
+    outs, fins = [], []
+    d = w.dk
+    for h in heads:
+        sl = slice(h * d, (h + 1) * d)
+        cw = w.conv_w[:, sl]
+        o, f = O.kda_mixer(w.q[:, h:h + 1], w.k[:, h:h + 1], w.v[:, h:h + 1], cw, w.log_alpha[:, h:h + 1],
+                           w.beta[:, h:h + 1], w.gate[:, h:h + 1], w.cu_seqlens)
+        outs.append(o)
+        fins.append(f)
+    return np.concatenate(outs, axis=1), np.concatenate(fins, axis=1)
+
+
+def _run_mixer(kda, w):
+    import torch
+    dt = "bf16"
+    out, fin = kda.mixer_fwd(to_device(w.q, dt), to_device(w.k, dt), to_device(w.v, dt), to_device(w.conv_w, "f32"),
+                             to_device(w.log_alpha, "f32"), to_device(w.beta, "f32"), to_device(w.gate, dt), None,
+                             to_device(w.cu_seqlens, "i32"), N=w.N, check_status=True)
+    torch.cuda.synchronize()
+    return to_host(out), to_host(fin)
+
+
+def test_mixer_small(kda):
+    w = I.make_prefill([300, 77], 4, 128, 128, seed=21, state_std=0.0, normalise_qk=False, mixer=True)
+    out, fin = _run_mixer(kda, w)
+    ro, rf = _mixer_oracle_heads(w, range(4))
+    assert_prefill_close(out, ro, "mixer out", stored_bf16=True)
+    assert_prefill_close(fin, rf, "mixer final")
+
+
+def test_mixer_full_size_sampled_heads(kda):
+    """B=2, T=32768, H=32, d=128: conv4 + L2 + KDA + sigmoid gate; oracle on 2 heads."""
+    w = I.mixer_prefill()
+    out, fin = _run_mixer(kda, w)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(fin))
+    heads = [3, 28]
+    ro, rf = _mixer_oracle_heads(w, heads)
+    assert_prefill_close(out[:, heads], ro, "mixer out", stored_bf16=True)
+    assert_prefill_close(fin[:, heads], rf, "mixer final")
