@@ -55,6 +55,8 @@ _SIGNATURES = {
     "kda_mixer_fwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
                              _vp, _vp, _vp, _sz, _vp]),
     "kda_workspace_status": (_i32, [_vp, _vp, _u32p]),
+    "kda_mixer_fwd_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
+                                     _vp, _vp, _vp]),
 }
 
 

@@ -73,6 +73,10 @@ kda_status check_common(int64_t total_T, int N, int H, int dk, int dv) {
 
 }  // namespace
 
+namespace kda {
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+}  // namespace kda
+
 extern "C" {
 
 const char* kda_status_string(kda_status s) {

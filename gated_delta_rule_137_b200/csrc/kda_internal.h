@@ -41,6 +41,9 @@ struct PrefillArgs {
   bool out_f32;           // out is fp32 (else bf16)
 };
 
+// Sets the message kda_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, bool bf16, const float* log_alpha,
                                const float* beta, float* state, int N, int H, int dk, int dv, void* out,
                                cudaStream_t stream);

@@ -171,6 +171,28 @@ KDA_API kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const voi
                          void* workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * Full mixer prefill without a workspace, for callers that cannot allocate device
+ * memory where they run the mixer (a plugin whose host framework owns every device
+ * allocation, a serving loop that may not call cudaMalloc). The paper has no
+ * counterpart: this is a packaging of kda_mixer_fwd, same arguments minus the
+ * workspace, same results.
+ *
+ * Scratch is a fixed array in the library's device memory (about 24 MiB per GPU
+ * that loads the library, held until the process exits). Limit: total_T * H <=
+ * 16384 token-heads; larger calls return KDA_ERR_UNSUPPORTED before any launch.
+ * The first call on a device looks the array up (cudaGetSymbolAddress) with that
+ * device current; make it before any stream capture. All calls on a device share
+ * the array, which keeps the last call's contents (the status word is cleared at
+ * the start of each call); calls that overlap on the GPU race and give undefined
+ * results. Device-detected range flags are not reported. Allocates nothing.
+ */
+KDA_API kda_status kda_mixer_fwd_noalloc(const void* q_raw, const void* k_raw, const void* v_raw,
+                                         const float* conv_w, const float* log_alpha, const float* beta,
+                                         const void* gate, const float* initial_state, const int32_t* cu_seqlens,
+                                         int64_t total_T, int N, int H, int dk, int dv, void* out,
+                                         float* final_state, kda_stream_t stream);
+
+/*
  * Reads the device status word kept in `workspace` (KDA_DEVFLAG_* bits) after
  * synchronising `stream`, and clears it. Returns KDA_ERR_RANGE when any bit
  * was set, KDA_OK otherwise; *flags (if not NULL) receives the bits.
