@@ -51,7 +51,7 @@ namespace kda {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // 8 warps; warps w and w+4 share TMEM lane quarter w
 constexpr float kMaxChunkDecay = 80.f;
 constexpr int kLd = 68;  // row stride (floats) of the fp32 solve scratch (16-B aligned rows)
 
@@ -74,6 +74,7 @@ struct Smem {
   static constexpr int kST = kKH;                    // DV*512 <= 64 KB, spans KH and KTT
   static constexpr int kStage = kTP;                 // 64 x DV bf16
   static constexpr int kScratch = kKH;               // A/X [64][kLd] + Y [32][kLd]
+  static constexpr int kTot = kVT;                   // per-warp decay totals [8][128] (gate pass only)
   static constexpr int kBeta = kVT + DV * 256;       // fp32 [64]
   static constexpr int kBar = kBeta + 256;           // 2 mbarriers
   static constexpr int kTmemSlot = kBar + 16;
@@ -104,6 +105,18 @@ __device__ __forceinline__ float ld_in(const __nv_bfloat16* p) { return __bfloat
 __device__ __forceinline__ float ld_in(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float as_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ float as_f32(float x) { return x; }
+
+// 4 consecutive input elements (8-byte bf16 or 16-byte fp32 read-only load)
+__device__ __forceinline__ void ld4_in(const __nv_bfloat16* p, float* o) {
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p));
+  const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
+  o[0] = __bfloat162float(b[0]); o[1] = __bfloat162float(b[1]);
+  o[2] = __bfloat162float(b[2]); o[3] = __bfloat162float(b[3]);
+}
+__device__ __forceinline__ void ld4_in(const float* p, float* o) {
+  const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+  o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+}
 
 // 16 consecutive output values of one row (TOut = bf16 or fp32)
 __device__ __forceinline__ void store16(__nv_bfloat16* dst, const float* o) {
@@ -165,7 +178,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   using SM = Smem<DV>;
   using TM = Tmem<DV>;
   constexpr int kSlices = kD / DV;
-  constexpr int kBatch = 16;  // tokens whose loads are in flight together in the gate pass
   static_assert(64 * DV * sizeof(TIn) <= 32768, "V staging must fit in the TP region");
 
   extern __shared__ uint8_t smem_raw[];
@@ -174,18 +186,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sA = reinterpret_cast<float*>(sm + SM::kScratch);    // [64][kLd]: A, then X in place
   float* sY = sA + 64 * kLd;                                  // [32][kLd]
   float* sBeta = reinterpret_cast<float*>(sm + SM::kBeta);
+  float* sTot = reinterpret_cast<float*>(sm + SM::kTot);      // [8][128]
   uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + SM::kBar);
   uint64_t* bar_tma = bar_mma + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmemSlot);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int lq = warp & 3;          // TMEM lane quarter this warp may access
+  const int half = warp >> 2;       // which half of a row's columns this warp handles
+  const int row = lq * 32 + lane;   // TMEM lane = accumulator row of this thread
+  const bool owner = warp < 4;      // warps 0-3 own the state rows (row == tid)
   const int slice = blockIdx.x % kSlices;
   const int nh = blockIdx.x / kSlices;
   const int H = a.H;
   const int h = nh % H;
   const int n = nh / H;
-  const int col0 = slice * DV;  // first value column owned by this CTA
+  const int col0 = slice * DV;      // first value column owned by this CTA
 
   // ---- sequence bounds ------------------------------------------------------------
   int64_t bos, eos;
@@ -217,15 +235,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_off = static_cast<uint32_t>(lq * 32) << 16;
 
-  // ---- the state slice in registers: thread c holds S[c][col0 .. col0+DV) ----------
+  // ---- the state slice in registers of warps 0-3: thread c holds S[c][col0 .. col0+DV)
   float S[DV];
-  {
-    const float* h0 = a.h0 ? a.h0 + ((static_cast<size_t>(n) * H + h) * kD + tid) * kD + col0 : nullptr;
+#pragma unroll
+  for (int j = 0; j < DV; ++j) S[j] = 0.f;
+  if (owner && a.h0) {
+    const float* h0 = a.h0 + ((static_cast<size_t>(n) * H + h) * kD + tid) * kD + col0;
 #pragma unroll
     for (int j = 0; j < DV; j += 4) {
-      const float4 x = h0 ? *reinterpret_cast<const float4*>(h0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 x = *reinterpret_cast<const float4*>(h0 + j);
       S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
     }
   }
@@ -256,53 +276,101 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int64_t t0 = bos; t0 < eos && !failed; t0 += kChunk) {
     const int len = static_cast<int>(eos - t0 < kChunk ? eos - t0 : kChunk);
 
-    // -- 1. V tile (bf16) by TMA into the staging area -----------------------------------
+    // -- 1. V tile by TMA into the staging area (the TP region, free until step 5) -----
     if (tid == 0) {
       mbar_arrive_expect_tx(bar_tma, 64u * DV * static_cast<uint32_t>(sizeof(TIn)));
       tma_load_3d(sm + SM::kStage, &tm_v, col0, h, static_cast<int>(t0), bar_tma);
     }
+    // warm L2 with the next chunk's q, k, log_alpha rows
+    if (t0 + kChunk < eos && lane < 8) {
+      const int64_t nt = t0 + kChunk;
+      const int r = warp * 8 + lane;
+      if (nt + r < eos) {
+        const size_t o = static_cast<size_t>(nt + r) * tok_stride + static_cast<size_t>(h) * kD;
+#pragma unroll
+        for (int c = 0; c < kD; c += 32) prefetch_l2(lag + o + c);
+        prefetch_l2(kg + o);
+        prefetch_l2(kg + o + 64);
+        prefetch_l2(qg + o);
+        prefetch_l2(qg + o + 64);
+      }
+    }
 
-    // -- 2. gates: thread c walks the chunk's tokens for key channel c ---------------
-    // Loads of kBatch tokens are issued together (rows past the sequence end read
-    // the chunk's first row, always in bounds, and are then replaced by zero).
-    float gamma_last;
+    // -- 2. gates. Warp w takes tokens 8w..8w+7, lane l key channels 4l..4l+3 ----------
+    float gamma_last = 1.f;  // e^{g_last} of key channel `tid` (owner warps)
     {
-      const int c = tid;
       if (tid < 64) sBeta[tid] = tid < len ? __ldg(a.beta + (t0 + tid) * H + h) : 0.f;
-      float g = 0.f;
-      const size_t base = static_cast<size_t>(t0) * tok_stride + static_cast<size_t>(h) * kD + c;
-#pragma unroll 1
-      for (int r0 = 0; r0 < kChunk; r0 += kBatch) {
-        float la[kBatch], kv[kBatch], qv[kBatch];
+      const int c0 = lane * 4, r0 = warp * 8;
+      float la[8][4], kv[8][4], qv[8][4];
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          const bool in = r0 + i < len;
-          const size_t o = base + static_cast<size_t>(in ? r0 + i : 0) * tok_stride;
-          const float l = __ldg(lag + o), kx = ld_in(kg + o), qx = ld_in(qg + o);
-          la[i] = in ? l : 0.f;
-          kv[i] = in ? kx : 0.f;
-          qv[i] = in ? qx : 0.f;
-        }
+      for (int i = 0; i < 8; ++i) {
+        const bool in = r0 + i < len;
+        const size_t o = static_cast<size_t>(t0 + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
+        const float4 l4 = __ldg(reinterpret_cast<const float4*>(lag + o));
+        float k4[4], q4[4];
+        ld4_in(kg + o, k4);
+        ld4_in(qg + o, q4);
+        la[i][0] = in ? l4.x : 0.f; la[i][1] = in ? l4.y : 0.f; la[i][2] = in ? l4.z : 0.f; la[i][3] = in ? l4.w : 0.f;
 #pragma unroll
-        for (int i = 0; i < kBatch; i += 4) {
-          float kt[4], kh[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = r0 + i + e;
-            g += la[i + e];
-            const float eg = __expf(g), eng = __expf(-g);
-            kt[e] = kv[i + e] * eg;
-            kh[e] = kv[i + e] * eng;
-            st_tf32(sm + SM::kKQ, f32_offset(r, c, 128), kt[e]);              // Kt   [tok][ch]
-            st_tf32(sm + SM::kKQ, f32_offset(64 + r, c, 128), qv[i + e] * eg);  // Qt   [tok][ch]
-            st_tf32(sm + SM::kKH, f32_offset(r, c, 64), kh[e]);               // Kh   [tok][ch]
-          }
-          st4_tf32(sm + SM::kKTT, f32_offset(c, r0 + i, 128), kt[0], kt[1], kt[2], kt[3]);  // Kt^T [ch][tok]
-          st4_tf32(sm + SM::kKHT, f32_offset(c, r0 + i, 128), kh[0], kh[1], kh[2], kh[3]);  // Kh^T [ch][tok]
+        for (int e = 0; e < 4; ++e) {
+          kv[i][e] = in ? k4[e] : 0.f;
+          qv[i][e] = in ? q4[e] : 0.f;
         }
       }
-      if (-g > kMaxChunkDecay) atomicOr(a.status, kFlagDecayRange);
-      gamma_last = __expf(g);
+      // running sums within this warp's 8 tokens, then the other warps' totals before them
+      float tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) { tot[e] += la[i][e]; la[i][e] = tot[e]; }
+      *reinterpret_cast<float4*>(sTot + warp * kD + c0) = make_float4(tot[0], tot[1], tot[2], tot[3]);
+      __syncthreads();
+      float pre[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int w = 0; w < warp; ++w) {
+        const float4 t4 = *reinterpret_cast<const float4*>(sTot + w * kD + c0);
+        pre[0] += t4.x; pre[1] += t4.y; pre[2] += t4.z; pre[3] += t4.w;
+      }
+      if (owner) {
+        float gl = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) gl += sTot[w * kD + tid];
+        if (-gl > kMaxChunkDecay) atomicOr(a.status, kFlagDecayRange);
+        gamma_last = __expf(gl);
+      }
+      float kt[8][4], kh[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float qt[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float g = pre[e] + la[i][e];
+          const float eg = __expf(g), eng = __expf(-g);
+          kt[i][e] = kv[i][e] * eg;
+          kh[i][e] = kv[i][e] * eng;
+          qt[e] = qv[i][e] * eg;
+        }
+        const int r = r0 + i;
+        st4_tf32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[i][0], kt[i][1], kt[i][2], kt[i][3]);   // Kt [tok][ch]
+        st4_tf32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);          // Qt [tok][ch]
+        st4_tf32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);    // Kh [tok][ch]
+      }
+      // channel-major copies: channel c0+e, tokens r0..r0+7; lanes rotate e so that one
+      // store instruction touches 8 different swizzle rows (no 16-way bank conflict)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = (j + lane) & 3;
+        float x[8], y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          x[i] = e == 0 ? kt[i][0] : e == 1 ? kt[i][1] : e == 2 ? kt[i][2] : kt[i][3];
+          y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
+        }
+        const int c = c0 + e;
+        st4_tf32(sm + SM::kKTT, f32_offset(c, r0, 128), x[0], x[1], x[2], x[3]);       // Kt^T [ch][tok]
+        st4_tf32(sm + SM::kKTT, f32_offset(c, r0 + 4, 128), x[4], x[5], x[6], x[7]);
+        st4_tf32(sm + SM::kKHT, f32_offset(c, r0, 128), y[0], y[1], y[2], y[3]);       // Kh^T [ch][tok]
+        st4_tf32(sm + SM::kKHT, f32_offset(c, r0 + 4, 128), y[4], y[5], y[6], y[7]);
+      }
     }
 
     // -- 3. V landed: widen/transpose to V^T fp32 (rows past the sequence end -> 0) -------
@@ -332,27 +400,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!wait_mma()) { failed = true; break; }
 
-    // -- 5. A (rows 0..63: beta-scaled, strictly lower) and P (rows 64..127: lower) ------
+    // -- 5. A (rows 0..63: beta-scaled, strictly lower), P (rows 64..127: lower) ---------
+    //       each warp takes 32 of the 64 columns of its rows
     {
-      float d[64];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        tmem_ld16(tmem + lane_off + TM::kD0 + 16 * j, *reinterpret_cast<float(*)[16]>(d + 16 * j));
+      const int cb = half * 32;
+      float d[32];
+      tmem_ld16(tmem + lane_off + TM::kD0 + cb, *reinterpret_cast<float(*)[16]>(d));
+      tmem_ld16(tmem + lane_off + TM::kD0 + cb + 16, *reinterpret_cast<float(*)[16]>(d + 16));
       tmem_ld_wait();
-      if (warp < 2) {
-        const int r = tid;
+      if (lq < 2) {
+        const int r = row;
         const float br = sBeta[r];
 #pragma unroll
-        for (int i = 0; i < 64; i += 4)
-          *reinterpret_cast<float4*>(sA + r * kLd + i) =
-              make_float4(i < r ? br * d[i] : 0.f, i + 1 < r ? br * d[i + 1] : 0.f, i + 2 < r ? br * d[i + 2] : 0.f,
-                          i + 3 < r ? br * d[i + 3] : 0.f);
+        for (int i = 0; i < 32; i += 4) {
+          const int c = cb + i;
+          *reinterpret_cast<float4*>(sA + r * kLd + c) =
+              make_float4(c < r ? br * d[i] : 0.f, c + 1 < r ? br * d[i + 1] : 0.f, c + 2 < r ? br * d[i + 2] : 0.f,
+                          c + 3 < r ? br * d[i + 3] : 0.f);
+        }
       } else {
-        const int r = tid - 64;
+        const int r = row - 64;
 #pragma unroll
-        for (int i = 0; i < 64; i += 4)
-          st4_tf32(sm + SM::kTP, f32_offset(64 + r, i, 128), i <= r ? d[i] : 0.f, i + 1 <= r ? d[i + 1] : 0.f,
-                   i + 2 <= r ? d[i + 2] : 0.f, i + 3 <= r ? d[i + 3] : 0.f);
+        for (int i = 0; i < 32; i += 4) {
+          const int c = cb + i;
+          st4_tf32(sm + SM::kTP, f32_offset(64 + r, c, 128), c <= r ? d[i] : 0.f, c + 1 <= r ? d[i + 1] : 0.f,
+                   c + 2 <= r ? d[i + 2] : 0.f, c + 3 <= r ? d[i + 3] : 0.f);
+        }
       }
     }
     tc_fence_before_sync();
@@ -404,10 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
       }
     }
-    if (tid < 64) {
-      const int r = tid;
+    if (tid < 128) {  // T row r, columns 32*hc .. +31
+      const int r = tid & 63, hc = tid >> 6;
 #pragma unroll
-      for (int i = 0; i < 64; i += 4) {
+      for (int i = 32 * hc; i < 32 * hc + 32; i += 4) {
         const float4 xr = *reinterpret_cast<const float4*>(sA + r * kLd + i);
         st4_tf32(sm + SM::kTP, f32_offset(r, i, 128), i <= r ? xr.x * sBeta[i] : 0.f,
                  i + 1 <= r ? xr.y * sBeta[i + 1] : 0.f, i + 2 <= r ? xr.z * sBeta[i + 2] : 0.f,
@@ -430,21 +503,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!wait_mma()) { failed = true; break; }
 
-    // -- 8. -W -> rows 0..63 of KQ (over Kt);  S -> S^T operand ------------------------------
-    if (warp < 2) {
-      const int r = tid;
+    // -- 8. -W -> rows 0..63 of KQ (over Kt), 64 columns per warp;  S -> S^T operand ------
+    if (lq < 2) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < 4; ++j) {
+        const int cb = half * 64 + 16 * j;
         float w[16];
-        tmem_ld16(tmem + lane_off + TM::kD0 + 16 * j, w);
+        tmem_ld16(tmem + lane_off + TM::kD0 + cb, w);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; e += 4)
-          st4_tf32(sm + SM::kKQ, f32_offset(r, 16 * j + e, 128), -w[e], -w[e + 1], -w[e + 2], -w[e + 3]);
+          st4_tf32(sm + SM::kKQ, f32_offset(row, cb + e, 128), -w[e], -w[e + 1], -w[e + 2], -w[e + 3]);
       }
     }
+    if (owner) {
 #pragma unroll
-    for (int j = 0; j < DV; ++j) st_tf32(sm + SM::kST, f32_offset(j, tid, DV), S[j]);
+      for (int j = 0; j < DV; ++j) st_tf32(sm + SM::kST, f32_offset(j, tid, DV), S[j]);
+    }
     fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
@@ -459,17 +534,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!wait_mma()) { failed = true; break; }
 
-    // -- 10. U = U~ - W S -> U^T operand (over V^T) --------------------------------------------
-    if (warp < 2) {
-      const int r = tid;
+    // -- 10. U = U~ - W S -> U^T operand (over V^T), DV/2 columns per warp ----------------------
+    if (lq < 2) {
 #pragma unroll
-      for (int j = 0; j < DV; j += 16) {
+      for (int j = 0; j < DV / 2; j += 16) {
+        const int cb = half * (DV / 2) + j;
         float ut[16], ws[16];
-        tmem_ld16(tmem + lane_off + TM::kD3 + j, ut);
-        tmem_ld16(tmem + lane_off + TM::kD1 + j, ws);
+        tmem_ld16(tmem + lane_off + TM::kD3 + cb, ut);
+        tmem_ld16(tmem + lane_off + TM::kD1 + cb, ws);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) st_tf32(sm + SM::kVT, f32_offset(j + e, r, DV), ut[e] + ws[e]);
+        for (int e = 0; e < 16; ++e) st_tf32(sm + SM::kVT, f32_offset(cb + e, row, DV), ut[e] + ws[e]);
       }
     }
     fence_proxy_async_smem();
@@ -489,24 +564,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!wait_mma()) { failed = true; break; }
 
-    // -- 12. S <- e^{g_last} (S + D2);  out rows <- O (* sigmoid(gate)) ----------------
-#pragma unroll
-    for (int j = 0; j < DV; j += 16) {
-      float d2[16];
-      tmem_ld16(tmem + lane_off + TM::kD2 + j, d2);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) S[j + i] = gamma_last * (S[j + i] + d2[i]);
-    }
-    if (warp >= 2) {
-      const int r = tid - 64;
+    // -- 12. S <- e^{g_last} (S + D2) (owners);  out rows <- O (* sigmoid(gate)) ---------
+    if (owner) {
 #pragma unroll
       for (int j = 0; j < DV; j += 16) {
+        float d2[16];
+        tmem_ld16(tmem + lane_off + TM::kD2 + j, d2);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) S[j + i] = gamma_last * (S[j + i] + d2[i]);
+      }
+    }
+    if (lq >= 2) {
+      const int r = row - 64;
+#pragma unroll
+      for (int j = 0; j < DV / 2; j += 16) {
+        const int cb = half * (DV / 2) + j;
         float o[16];
-        tmem_ld16(tmem + lane_off + TM::kD1 + j, o);
+        tmem_ld16(tmem + lane_off + TM::kD1 + cb, o);
         tmem_ld_wait();
         if (r < len) {
-          const size_t off = static_cast<size_t>(t0 + r) * tok_stride + static_cast<size_t>(h) * kD + col0 + j;
+          const size_t off = static_cast<size_t>(t0 + r) * tok_stride + static_cast<size_t>(h) * kD + col0 + cb;
           if (gateg) {
             const uint4 g0 = *reinterpret_cast<const uint4*>(gateg + off);
             const uint4 g1 = *reinterpret_cast<const uint4*>(gateg + off + 8);
@@ -527,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- final state -------------------------------------------------------------------
-  if (!failed && a.ht) {
+  if (!failed && a.ht && owner) {
     float* ht = a.ht + ((static_cast<size_t>(n) * H + h) * kD + tid) * kD + col0;
 #pragma unroll
     for (int j = 0; j < DV; j += 4) *reinterpret_cast<float4*>(ht + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);

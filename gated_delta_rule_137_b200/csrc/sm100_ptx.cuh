@@ -91,6 +91,11 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Bring one global cache line into L2 ahead of its use.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ---------------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor) loads — plain, never multicast
 // ---------------------------------------------------------------------------------
