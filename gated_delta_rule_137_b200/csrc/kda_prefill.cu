@@ -51,7 +51,7 @@ namespace kda {
 
 namespace {
 
-constexpr int kThreads = 256;  // 8 warps; warps w and w+4 share TMEM lane quarter w
+constexpr int kThreads = 512;  // 16 warps; warp w reads TMEM lanes 32*(w%4).. and column part w/4
 constexpr float kMaxChunkDecay = 80.f;
 constexpr int kLd = 68;  // row stride (floats) of the fp32 solve scratch (16-B aligned rows)
 
@@ -74,14 +74,16 @@ struct Smem {
   static constexpr int kST = kKH;                    // DV*512 <= 64 KB, spans KH and KTT
   static constexpr int kStage = kTP;                 // 64 x DV bf16
   static constexpr int kScratch = kKH;               // A/X [64][kLd] + Y [32][kLd]
-  static constexpr int kTot = kVT;                   // per-warp decay totals [8][128] (gate pass only)
+  static constexpr int kTot = kVT;                   // per-warp decay totals [16][128] (gate pass only)
   static constexpr int kBeta = kVT + DV * 256;       // fp32 [64]
-  static constexpr int kBar = kBeta + 256;           // 2 mbarriers
+  static constexpr int kGamma = kBeta + 256;         // fp32 [2][128]: e^{g_last} of the last two chunks
+  static constexpr int kBar = kGamma + 1024;         // 2 mbarriers
   static constexpr int kTmemSlot = kBar + 16;
   static constexpr int kTotal = kTmemSlot + 16;
   static constexpr int kAlloc = kTotal + 1024;       // slack for the 1024-B alignment
   static_assert(DV * 512 <= 65536, "S^T must fit in KH + KTT");
   static_assert((64 + 32) * kLd * 4 <= 32768, "solve scratch must fit in KH");
+  static_assert(16 * 128 * 4 <= DV * 256, "decay totals must fit in VT");
 };
 
 template <int DV>
@@ -89,7 +91,7 @@ struct Tmem {
   static constexpr uint32_t kCols = (128 + 3 * DV) <= 256 ? 256u : 512u;
   static constexpr uint32_t kD0 = 0;                 // [A; P], then [W; -]   (128 cols)
   static constexpr uint32_t kD1 = 128;               // [-W S; Qt S] -> O     (DV cols)
-  static constexpr uint32_t kD2 = 128 + DV;          // Kh^T U                (DV cols)
+  static constexpr uint32_t kD2 = 128 + DV;          // the state S (+= Kh^T U) (DV cols)
   static constexpr uint32_t kD3 = 128 + 2 * DV;      // [U~; -]               (DV cols)
 };
 
@@ -118,6 +120,18 @@ __device__ __forceinline__ void ld4_in(const float* p, float* o) {
   o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
 }
 
+// 8 consecutive output values of one row (TOut = bf16 or fp32)
+__device__ __forceinline__ void store8(__nv_bfloat16* dst, const float* o) {
+  uint4 p;
+  p.x = pack_bf16x2(o[0], o[1]); p.y = pack_bf16x2(o[2], o[3]);
+  p.z = pack_bf16x2(o[4], o[5]); p.w = pack_bf16x2(o[6], o[7]);
+  *reinterpret_cast<uint4*>(dst) = p;
+}
+__device__ __forceinline__ void store8(float* dst, const float* o) {
+  *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+  *reinterpret_cast<float4*>(dst + 4) = make_float4(o[4], o[5], o[6], o[7]);
+}
+
 // 16 consecutive output values of one row (TOut = bf16 or fp32)
 __device__ __forceinline__ void store16(__nv_bfloat16* dst, const float* o) {
   uint4 p0, p1;
@@ -144,32 +158,41 @@ __device__ __forceinline__ void st4_tf32(uint8_t* base, uint32_t off, float a, f
 // CTA-wide OR of a predicate (every thread gets the same answer).
 __device__ __forceinline__ bool cta_any(bool x) { return __syncthreads_or(x ? 1 : 0) != 0; }
 
-// C (n x n, row stride kLd) = scale * A (n x n) * B (n x n), all fp32 in shared
-// memory; n in {16, 32}; `count` independent products are spread over the CTA.
-// Thread tile: 2 rows x 4 columns.
-__device__ __forceinline__ void small_gemm(int n, int count, const float* const* As, const float* const* Bs,
-                                           float* const* Cs, float scale) {
-  const int tiles_per = (n / 2) * (n / 4);
-  for (int w = threadIdx.x; w < count * tiles_per; w += kThreads) {
-    const int p = w / tiles_per, t = w % tiles_per;
-    const int r0 = (t / (n / 4)) * 2, c0 = (t % (n / 4)) * 4;
-    const float* A = As[p];
-    const float* B = Bs[p];
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    for (int k = 0; k < n; ++k) {
-      const float a0 = A[r0 * kLd + k], a1 = A[(r0 + 1) * kLd + k];
-      const float4 b = *reinterpret_cast<const float4*>(B + k * kLd + c0);
-      acc[0][0] = fmaf(a0, b.x, acc[0][0]); acc[0][1] = fmaf(a0, b.y, acc[0][1]);
-      acc[0][2] = fmaf(a0, b.z, acc[0][2]); acc[0][3] = fmaf(a0, b.w, acc[0][3]);
-      acc[1][0] = fmaf(a1, b.x, acc[1][0]); acc[1][1] = fmaf(a1, b.y, acc[1][1]);
-      acc[1][2] = fmaf(a1, b.z, acc[1][2]); acc[1][3] = fmaf(a1, b.w, acc[1][3]);
-    }
-    float* C = Cs[p];
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-      *reinterpret_cast<float4*>(C + (r0 + i) * kLd + c0) =
-          make_float4(scale * acc[i][0], scale * acc[i][1], scale * acc[i][2], scale * acc[i][3]);
+// ---- small fp32-accurate products for the triangular solve (warp-level mma.sync) ----
+// x = hi + lo with hi, lo representable in tf32; the 3-term product hi*hi + hi*lo + lo*hi
+// keeps close to fp32 accuracy on the tensor pipe.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  const float h = to_tf32(x);
+  hi = __float_as_uint(h);
+  lo = __float_as_uint(to_tf32(x - h));
+}
+
+__device__ __forceinline__ void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// One warp: C (16 x 8) = scale * A (16 x K, row stride kLd) * B (K x 8, row stride kLd),
+// fp32 in shared memory, K a multiple of 8; C stored with row stride kLd.
+__device__ __forceinline__ void warp_gemm_16x8(const float* A, const float* B, int K, float* C, float scale) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k = 0; k < K; k += 8) {
+    uint32_t ah[4], al[4], bh[2], bl[2];
+    split_tf32(A[g * kLd + k + t], ah[0], al[0]);
+    split_tf32(A[(g + 8) * kLd + k + t], ah[1], al[1]);
+    split_tf32(A[g * kLd + k + t + 4], ah[2], al[2]);
+    split_tf32(A[(g + 8) * kLd + k + t + 4], ah[3], al[3]);
+    split_tf32(B[(k + t) * kLd + g], bh[0], bl[0]);
+    split_tf32(B[(k + t + 4) * kLd + g], bh[1], bl[1]);
+    mma_m16n8k8_tf32(acc, al, bh);
+    mma_m16n8k8_tf32(acc, ah, bl);
+    mma_m16n8k8_tf32(acc, ah, bh);
   }
+  *reinterpret_cast<float2*>(C + g * kLd + 2 * t) = make_float2(scale * acc[0], scale * acc[1]);
+  *reinterpret_cast<float2*>(C + (g + 8) * kLd + 2 * t) = make_float2(scale * acc[2], scale * acc[3]);
 }
 
 template <int DV, typename TIn, typename TOut>
@@ -178,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using SM = Smem<DV>;
   using TM = Tmem<DV>;
   constexpr int kSlices = kD / DV;
+  constexpr int kPart = DV / 4;     // value columns per warp in the TMEM epilogues
   static_assert(64 * DV * sizeof(TIn) <= 32768, "V staging must fit in the TP region");
 
   extern __shared__ uint8_t smem_raw[];
@@ -186,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sA = reinterpret_cast<float*>(sm + SM::kScratch);    // [64][kLd]: A, then X in place
   float* sY = sA + 64 * kLd;                                  // [32][kLd]
   float* sBeta = reinterpret_cast<float*>(sm + SM::kBeta);
-  float* sTot = reinterpret_cast<float*>(sm + SM::kTot);      // [8][128]
+  float* sGamma = reinterpret_cast<float*>(sm + SM::kGamma);  // [2][128]
+  float* sTot = reinterpret_cast<float*>(sm + SM::kTot);      // [16][128]
   uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + SM::kBar);
   uint64_t* bar_tma = bar_mma + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmemSlot);
@@ -195,9 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int lq = warp & 3;          // TMEM lane quarter this warp may access
-  const int half = warp >> 2;       // which half of a row's columns this warp handles
+  const int cp = warp >> 2;         // which quarter of a row's columns this warp handles
   const int row = lq * 32 + lane;   // TMEM lane = accumulator row of this thread
-  const bool owner = warp < 4;      // warps 0-3 own the state rows (row == tid)
   const int slice = blockIdx.x % kSlices;
   const int nh = blockIdx.x / kSlices;
   const int H = a.H;
@@ -231,23 +255,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, TM::kCols);
     tmem_relinquish();
   }
+  if (tid < 128) sGamma[128 + tid] = 1.f;  // "previous chunk" scale for the first chunk
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = static_cast<uint32_t>(lq * 32) << 16;
 
-  // ---- the state slice in registers of warps 0-3: thread c holds S[c][col0 .. col0+DV)
-  float S[DV];
+  // ---- the state slice lives in TMEM (D2): lane c = key row c, DV columns ----------
+  {
+    const float* h0 = a.h0 ? a.h0 + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0 : nullptr;
 #pragma unroll
-  for (int j = 0; j < DV; ++j) S[j] = 0.f;
-  if (owner && a.h0) {
-    const float* h0 = a.h0 + ((static_cast<size_t>(n) * H + h) * kD + tid) * kD + col0;
+    for (int j = 0; j < kPart; j += 8) {
+      const int c = cp * kPart + j;
+      float x[8];
+      if (h0) {
+        const float4 u = *reinterpret_cast<const float4*>(h0 + c);
+        const float4 w = *reinterpret_cast<const float4*>(h0 + c + 4);
+        x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
+      } else {
 #pragma unroll
-    for (int j = 0; j < DV; j += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(h0 + j);
-      S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+      }
+      tmem_st8(tmem + lane_off + TM::kD2 + c, x);
     }
+    tmem_st_wait();
   }
 
   const TIn* __restrict__ qg = static_cast<const TIn*>(a.q);
@@ -263,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t mma_phase = 0, tma_phase = 0;
   bool failed = false;
+  int gslot = 1;  // sGamma slot of the last chunk's e^{g_last} (slot 1 holds 1.0 initially)
 
   // all threads wait for the last commit; false (everywhere) if it never came
   auto wait_mma = [&]() -> bool {
@@ -273,8 +306,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     return true;
   };
 
+  // Gate inputs of one chunk for this thread (warp w: tokens 4w..4w+3, lane l: key
+  // channels 4l..4l+3). The next chunk's are loaded while this chunk's MMAs run.
+  const int c0 = lane * 4, r0 = warp * 4;
+  float4 la4[4];   // raw loads, masked where used (keeps the loads in flight)
+  uint32_t kraw[4][sizeof(TIn)], qraw[4][sizeof(TIn)];  // 4 elements: 2 words (bf16) or 4 (fp32)
+  auto load_gate = [&](int64_t tc, int lc) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool in = r0 + i < lc;  // rows past the sequence end read the chunk's first row
+      const size_t o = static_cast<size_t>(tc + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
+      la4[i] = __ldg(reinterpret_cast<const float4*>(lag + o));
+      if constexpr (sizeof(TIn) == 2) {
+        const uint2 kk2 = __ldg(reinterpret_cast<const uint2*>(kg + o));
+        const uint2 qq2 = __ldg(reinterpret_cast<const uint2*>(qg + o));
+        kraw[i][0] = kk2.x; kraw[i][1] = kk2.y; qraw[i][0] = qq2.x; qraw[i][1] = qq2.y;
+      } else {
+        const uint4 kk4 = __ldg(reinterpret_cast<const uint4*>(kg + o));
+        const uint4 qq4 = __ldg(reinterpret_cast<const uint4*>(qg + o));
+        kraw[i][0] = kk4.x; kraw[i][1] = kk4.y; kraw[i][2] = kk4.z; kraw[i][3] = kk4.w;
+        qraw[i][0] = qq4.x; qraw[i][1] = qq4.y; qraw[i][2] = qq4.z; qraw[i][3] = qq4.w;
+      }
+    }
+  };
+  // element e (0..3) of a raw 4-element load
+  auto unpack = [&](const uint32_t* w, int e) -> float {
+    if constexpr (sizeof(TIn) == 2) {
+      const uint32_t x = w[e >> 1];
+      return __uint_as_float((e & 1) ? (x & 0xFFFF0000u) : (x << 16));
+    } else {
+      return __uint_as_float(w[e]);
+    }
+  };
+  if (bos < eos) load_gate(bos, static_cast<int>(eos - bos < kChunk ? eos - bos : kChunk));
+
   for (int64_t t0 = bos; t0 < eos && !failed; t0 += kChunk) {
     const int len = static_cast<int>(eos - t0 < kChunk ? eos - t0 : kChunk);
+    const int gnew = gslot ^ 1;  // slot for this chunk's e^{g_last}
 
     // -- 1. V tile by TMA into the staging area (the TP region, free until step 5) -----
     if (tid == 0) {
@@ -282,9 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sm + SM::kStage, &tm_v, col0, h, static_cast<int>(t0), bar_tma);
     }
     // warm L2 with the next chunk's q, k, log_alpha rows
-    if (t0 + kChunk < eos && lane < 8) {
+    if (t0 + kChunk < eos && lane < 4) {
       const int64_t nt = t0 + kChunk;
-      const int r = warp * 8 + lane;
+      const int r = warp * 4 + lane;
       if (nt + r < eos) {
         const size_t o = static_cast<size_t>(nt + r) * tok_stride + static_cast<size_t>(h) * kD;
 #pragma unroll
@@ -296,31 +364,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
-    // -- 2. gates. Warp w takes tokens 8w..8w+7, lane l key channels 4l..4l+3 ----------
-    float gamma_last = 1.f;  // e^{g_last} of key channel `tid` (owner warps)
+    // -- 2. gates. Warp w takes tokens 4w..4w+3, lane l key channels 4l..4l+3 ----------
     {
       if (tid < 64) sBeta[tid] = tid < len ? __ldg(a.beta + (t0 + tid) * H + h) : 0.f;
-      const int c0 = lane * 4, r0 = warp * 8;
-      float la[8][4], kv[8][4], qv[8][4];
+      float la[4][4], kv[4][4], qv[4][4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 4; ++i) {
         const bool in = r0 + i < len;
-        const size_t o = static_cast<size_t>(t0 + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
-        const float4 l4 = __ldg(reinterpret_cast<const float4*>(lag + o));
-        float k4[4], q4[4];
-        ld4_in(kg + o, k4);
-        ld4_in(qg + o, q4);
-        la[i][0] = in ? l4.x : 0.f; la[i][1] = in ? l4.y : 0.f; la[i][2] = in ? l4.z : 0.f; la[i][3] = in ? l4.w : 0.f;
+        la[i][0] = in ? la4[i].x : 0.f; la[i][1] = in ? la4[i].y : 0.f;
+        la[i][2] = in ? la4[i].z : 0.f; la[i][3] = in ? la4[i].w : 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          kv[i][e] = in ? k4[e] : 0.f;
-          qv[i][e] = in ? q4[e] : 0.f;
+          kv[i][e] = in ? unpack(kraw[i], e) : 0.f;
+          qv[i][e] = in ? unpack(qraw[i], e) : 0.f;
         }
       }
-      // running sums within this warp's 8 tokens, then the other warps' totals before them
+      // running sums within this warp's 4 tokens, then the totals of the warps before it
       float tot[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int e = 0; e < 4; ++e) { tot[e] += la[i][e]; la[i][e] = tot[e]; }
       *reinterpret_cast<float4*>(sTot + warp * kD + c0) = make_float4(tot[0], tot[1], tot[2], tot[3]);
@@ -330,16 +392,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 t4 = *reinterpret_cast<const float4*>(sTot + w * kD + c0);
         pre[0] += t4.x; pre[1] += t4.y; pre[2] += t4.z; pre[3] += t4.w;
       }
-      if (owner) {
+      if (tid < 128) {
         float gl = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) gl += sTot[w * kD + tid];
+        for (int w = 0; w < 16; ++w) gl += sTot[w * kD + tid];
         if (-gl > kMaxChunkDecay) atomicOr(a.status, kFlagDecayRange);
-        gamma_last = __expf(gl);
+        sGamma[gnew * 128 + tid] = __expf(gl);
       }
-      float kt[8][4], kh[8][4];
+      float kt[4][4], kh[4][4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 4; ++i) {
         float qt[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -354,22 +416,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         st4_tf32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);          // Qt [tok][ch]
         st4_tf32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);    // Kh [tok][ch]
       }
-      // channel-major copies: channel c0+e, tokens r0..r0+7; lanes rotate e so that one
-      // store instruction touches 8 different swizzle rows (no 16-way bank conflict)
+      // channel-major copies: channel c0+e, tokens r0..r0+3; lanes rotate e so that one
+      // store instruction touches different swizzle rows
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int e = (j + lane) & 3;
-        float x[8], y[8];
+        float x[4], y[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
           x[i] = e == 0 ? kt[i][0] : e == 1 ? kt[i][1] : e == 2 ? kt[i][2] : kt[i][3];
           y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
         }
-        const int c = c0 + e;
-        st4_tf32(sm + SM::kKTT, f32_offset(c, r0, 128), x[0], x[1], x[2], x[3]);       // Kt^T [ch][tok]
-        st4_tf32(sm + SM::kKTT, f32_offset(c, r0 + 4, 128), x[4], x[5], x[6], x[7]);
-        st4_tf32(sm + SM::kKHT, f32_offset(c, r0, 128), y[0], y[1], y[2], y[3]);       // Kh^T [ch][tok]
-        st4_tf32(sm + SM::kKHT, f32_offset(c, r0 + 4, 128), y[4], y[5], y[6], y[7]);
+        st4_tf32(sm + SM::kKTT, f32_offset(c0 + e, r0, 128), x[0], x[1], x[2], x[3]);   // Kt^T [ch][tok]
+        st4_tf32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);   // Kh^T [ch][tok]
       }
     }
 
@@ -401,18 +460,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!wait_mma()) { failed = true; break; }
 
     // -- 5. A (rows 0..63: beta-scaled, strictly lower), P (rows 64..127: lower) ---------
-    //       each warp takes 32 of the 64 columns of its rows
     {
-      const int cb = half * 32;
-      float d[32];
-      tmem_ld16(tmem + lane_off + TM::kD0 + cb, *reinterpret_cast<float(*)[16]>(d));
-      tmem_ld16(tmem + lane_off + TM::kD0 + cb + 16, *reinterpret_cast<float(*)[16]>(d + 16));
+      const int cb = cp * 16;
+      float d[16];
+      tmem_ld16(tmem + lane_off + TM::kD0 + cb, d);
       tmem_ld_wait();
       if (lq < 2) {
         const int r = row;
         const float br = sBeta[r];
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
+        for (int i = 0; i < 16; i += 4) {
           const int c = cb + i;
           *reinterpret_cast<float4*>(sA + r * kLd + c) =
               make_float4(c < r ? br * d[i] : 0.f, c + 1 < r ? br * d[i + 1] : 0.f, c + 2 < r ? br * d[i + 2] : 0.f,
@@ -421,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const int r = row - 64;
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
+        for (int i = 0; i < 16; i += 4) {
           const int c = cb + i;
           st4_tf32(sm + SM::kTP, f32_offset(64 + r, c, 128), c <= r ? d[i] : 0.f, c + 1 <= r ? d[i + 1] : 0.f,
                    c + 2 <= r ? d[i + 2] : 0.f, c + 3 <= r ? d[i + 3] : 0.f);
@@ -432,55 +489,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     // -- 6. X = (I + A)^-1 in fp32 (in place over A), T = X Diag(beta) ---------------------
-    {
-      float x[16];
-      if (tid < 64) {  // 16x16 diagonal blocks: thread (b, j) solves column j of block b
-        const int b = tid >> 4, j = tid & 15;
-        const float* Ab = sA + (16 * b) * kLd + 16 * b;
+    // 6a. 16x16 diagonal blocks by forward substitution in registers: warp b < 4 owns
+    //     block b, lane (r = lane % 16, half hh) holds row r, columns 8hh..8hh+7.
+    if (warp < 4) {
+      const int b = warp, r = lane & 15, hh = lane >> 4;
+      float* Arow = sA + (16 * b + r) * kLd + 16 * b;
+      float av[16], x[8];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          float acc = (r == j) ? 1.f : 0.f;
+      for (int i = 0; i < 16; ++i) av[i] = Arow[i];
 #pragma unroll
-          for (int i = 0; i < r; ++i) acc = fmaf(-Ab[r * kLd + i], x[i], acc);
-          x[r] = acc;
-        }
-      }
-      __syncthreads();
-      if (tid < 64) {
-        const int b = tid >> 4, j = tid & 15;
+      for (int j = 0; j < 8; ++j) x[j] = (8 * hh + j == r) ? 1.f : 0.f;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sA[(16 * b + r) * kLd + 16 * b + j] = x[r];
+      for (int i = 0; i < 15; ++i) {  // row i is final: rows below subtract A[r][i] * row i
+        const float c = (r > i) ? av[i] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = fmaf(-c, __shfl_sync(0xffffffffu, x[j], i + 16 * hh), x[j]);
       }
-      __syncthreads();
-      // doubling: for each diagonal pair [[X1, 0], [A21, X2]] -> X21 = -X2 (A21 X1)
-#pragma unroll 1
-      for (int s = 16; s < 64; s *= 2) {
-        const int pairs = 64 / (2 * s);
-        const float* As_[2];
-        const float* Bs_[2];
-        float* Cs_[2];
-        for (int p = 0; p < pairs; ++p) {
-          const int o = 2 * s * p;
-          As_[p] = sA + (o + s) * kLd + o;   // A21
-          Bs_[p] = sA + o * kLd + o;         // X1
-          Cs_[p] = sY + p * 16;              // Y (pairs of 16 side by side, or one 32)
-        }
-        small_gemm(s, pairs, As_, Bs_, Cs_, 1.f);
-        __syncthreads();
-        for (int p = 0; p < pairs; ++p) {
-          const int o = 2 * s * p;
-          As_[p] = sA + (o + s) * kLd + o + s;  // X2
-          Bs_[p] = sY + p * 16;                 // Y
-          Cs_[p] = sA + (o + s) * kLd + o;      // X21 over A21
-        }
-        small_gemm(s, pairs, As_, Bs_, Cs_, -1.f);
-        __syncthreads();
-      }
+      __syncwarp();
+      *reinterpret_cast<float4*>(Arow + 8 * hh) = make_float4(x[0], x[1], x[2], x[3]);
+      *reinterpret_cast<float4*>(Arow + 8 * hh + 4) = make_float4(x[4], x[5], x[6], x[7]);
     }
-    if (tid < 128) {  // T row r, columns 32*hc .. +31
-      const int r = tid & 63, hc = tid >> 6;
+    __syncthreads();
+    // 6b. doubling, [[X1, 0], [A21, X2]]^-1 has lower-left block -X2 (A21 X1):
+    //     16 -> 32 on the two diagonal pairs (warp = pair * 2 + 8-column tile) ...
+    if (warp < 4) {
+      const int p = warp >> 1, nt = warp & 1, o = 32 * p;
+      warp_gemm_16x8(sA + (o + 16) * kLd + o, sA + o * kLd + o + 8 * nt, 16, sY + 16 * p + 8 * nt, 1.f);
+    }
+    __syncthreads();
+    if (warp < 4) {
+      const int p = warp >> 1, nt = warp & 1, o = 32 * p;
+      warp_gemm_16x8(sA + (o + 16) * kLd + o + 16, sY + 16 * p + 8 * nt, 16, sA + (o + 16) * kLd + o + 8 * nt, -1.f);
+    }
+    __syncthreads();
+    //     ... then 32 -> 64 (warp = 16-row tile * 4 + 8-column tile)
+    if (warp < 8) {
+      const int mt = warp >> 2, nt = warp & 3;
+      warp_gemm_16x8(sA + (32 + 16 * mt) * kLd, sA + 8 * nt, 32, sY + (16 * mt) * kLd + 8 * nt, 1.f);
+    }
+    __syncthreads();
+    if (warp < 8) {
+      const int mt = warp >> 2, nt = warp & 3;
+      warp_gemm_16x8(sA + (32 + 16 * mt) * kLd + 32, sY + 8 * nt, 32, sA + (32 + 16 * mt) * kLd + 8 * nt, -1.f);
+    }
+    __syncthreads();
+    {  // T row r, columns 8*part .. +7
+      const int r = tid & 63, c = (tid >> 6) * 8;
 #pragma unroll
-      for (int i = 32 * hc; i < 32 * hc + 32; i += 4) {
+      for (int i = c; i < c + 8; i += 4) {
         const float4 xr = *reinterpret_cast<const float4*>(sA + r * kLd + i);
         st4_tf32(sm + SM::kTP, f32_offset(r, i, 128), i <= r ? xr.x * sBeta[i] : 0.f,
                  i + 1 <= r ? xr.y * sBeta[i + 1] : 0.f, i + 2 <= r ? xr.z * sBeta[i + 2] : 0.f,
@@ -503,11 +559,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!wait_mma()) { failed = true; break; }
 
-    // -- 8. -W -> rows 0..63 of KQ (over Kt), 64 columns per warp;  S -> S^T operand ------
+    // -- 8. -W -> rows 0..63 of KQ (over Kt);  S <- e^{g_last}(previous chunk) S in TMEM
+    //       and as the S^T operand -------------------------------------------------------
     if (lq < 2) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int cb = half * 64 + 16 * j;
+      for (int j = 0; j < 2; ++j) {
+        const int cb = cp * 32 + 16 * j;
         float w[16];
         tmem_ld16(tmem + lane_off + TM::kD0 + cb, w);
         tmem_ld_wait();
@@ -516,9 +573,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           st4_tf32(sm + SM::kKQ, f32_offset(row, cb + e, 128), -w[e], -w[e + 1], -w[e + 2], -w[e + 3]);
       }
     }
-    if (owner) {
+    {
+      const float gm = sGamma[gslot * 128 + row];
 #pragma unroll
-      for (int j = 0; j < DV; ++j) st_tf32(sm + SM::kST, f32_offset(j, tid, DV), S[j]);
+      for (int j = 0; j < kPart; j += 8) {
+        const int c = cp * kPart + j;
+        float x[8];
+        tmem_ld8(tmem + lane_off + TM::kD2 + c, x);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x[e] *= gm;
+          st_tf32(sm + SM::kST, f32_offset(c + e, row, DV), x[e]);
+        }
+        tmem_st8(tmem + lane_off + TM::kD2 + c, x);
+      }
+      tmem_st_wait();
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
@@ -532,71 +602,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_tf32(tmem + TM::kD1, kdesc(sb + SM::kKQ, kk, 128), kdesc(sb + SM::kST, kk, DV), kIdV, kk > 0);
       umma_commit(bar_mma);
     }
+    if (t0 + kChunk < eos) {  // next chunk's gate inputs, in flight during the MMAs
+      const int64_t nt = t0 + kChunk;
+      load_gate(nt, static_cast<int>(eos - nt < kChunk ? eos - nt : kChunk));
+    }
     if (!wait_mma()) { failed = true; break; }
 
-    // -- 10. U = U~ - W S -> U^T operand (over V^T), DV/2 columns per warp ----------------------
+    // -- 10. U = U~ - W S -> U^T operand (over V^T) ---------------------------------------------
     if (lq < 2) {
 #pragma unroll
-      for (int j = 0; j < DV / 2; j += 16) {
-        const int cb = half * (DV / 2) + j;
-        float ut[16], ws[16];
-        tmem_ld16(tmem + lane_off + TM::kD3 + cb, ut);
-        tmem_ld16(tmem + lane_off + TM::kD1 + cb, ws);
+      for (int j = 0; j < kPart; j += 8) {
+        const int c = cp * kPart + j;
+        float ut[8], ws[8];
+        tmem_ld8(tmem + lane_off + TM::kD3 + c, ut);
+        tmem_ld8(tmem + lane_off + TM::kD1 + c, ws);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) st_tf32(sm + SM::kVT, f32_offset(cb + e, row, DV), ut[e] + ws[e]);
+        for (int e = 0; e < 8; ++e) st_tf32(sm + SM::kVT, f32_offset(c + e, row, DV), ut[e] + ws[e]);
       }
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
 
-    // -- 11. D2 = Kh^T U ;  D1 += [T; P] U  ->  O = Qt S + P U in rows 64..127 ----------------
+    // -- 11. D2 = S + Kh^T U ;  D1 += [T; P] U  ->  O = Qt S + P U in rows 64..127 ------------
     if (tid == 0) {
       tc_fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_tf32(tmem + TM::kD2, kdesc(sb + SM::kKHT, kk, 128), kdesc(sb + SM::kVT, kk, DV), kIdV, kk > 0);
+        umma_tf32(tmem + TM::kD2, kdesc(sb + SM::kKHT, kk, 128), kdesc(sb + SM::kVT, kk, DV), kIdV, 1u);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
         umma_tf32(tmem + TM::kD1, kdesc(sb + SM::kTP, kk, 128), kdesc(sb + SM::kVT, kk, DV), kIdV, 1u);
       umma_commit(bar_mma);
     }
     if (!wait_mma()) { failed = true; break; }
+    gslot = gnew;
 
-    // -- 12. S <- e^{g_last} (S + D2) (owners);  out rows <- O (* sigmoid(gate)) ---------
-    if (owner) {
-#pragma unroll
-      for (int j = 0; j < DV; j += 16) {
-        float d2[16];
-        tmem_ld16(tmem + lane_off + TM::kD2 + j, d2);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) S[j + i] = gamma_last * (S[j + i] + d2[i]);
-      }
-    }
+    // -- 12. out rows <- O (* sigmoid(gate)) ------------------------------------------------------
     if (lq >= 2) {
       const int r = row - 64;
 #pragma unroll
-      for (int j = 0; j < DV / 2; j += 16) {
-        const int cb = half * (DV / 2) + j;
-        float o[16];
-        tmem_ld16(tmem + lane_off + TM::kD1 + cb, o);
+      for (int j = 0; j < kPart; j += 8) {
+        const int c = cp * kPart + j;
+        float o[8];
+        tmem_ld8(tmem + lane_off + TM::kD1 + c, o);
         tmem_ld_wait();
         if (r < len) {
-          const size_t off = static_cast<size_t>(t0 + r) * tok_stride + static_cast<size_t>(h) * kD + col0 + cb;
+          const size_t off = static_cast<size_t>(t0 + r) * tok_stride + static_cast<size_t>(h) * kD + col0 + c;
           if (gateg) {
             const uint4 g0 = *reinterpret_cast<const uint4*>(gateg + off);
-            const uint4 g1 = *reinterpret_cast<const uint4*>(gateg + off + 8);
             const __nv_bfloat16* gb0 = reinterpret_cast<const __nv_bfloat16*>(&g0);
-            const __nv_bfloat16* gb1 = reinterpret_cast<const __nv_bfloat16*>(&g1);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              o[i] *= 1.f / (1.f + __expf(-bf2f(gb0[i])));
-              o[8 + i] *= 1.f / (1.f + __expf(-bf2f(gb1[i])));
-            }
+            for (int i = 0; i < 8; ++i) o[i] *= 1.f / (1.f + __expf(-bf2f(gb0[i])));
           }
-          store16(outg + off, o);
+          store8(outg + off, o);
         }
       }
     }
@@ -604,11 +664,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   }
 
-  // ---- final state -------------------------------------------------------------------
-  if (!failed && a.ht && owner) {
-    float* ht = a.ht + ((static_cast<size_t>(n) * H + h) * kD + tid) * kD + col0;
+  // ---- final state: e^{g_last} of the last chunk times D2 --------------------------------
+  if (!failed && a.ht) {
+    const float gm = sGamma[gslot * 128 + row];
+    float* ht = a.ht + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0;
 #pragma unroll
-    for (int j = 0; j < DV; j += 4) *reinterpret_cast<float4*>(ht + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    for (int j = 0; j < kPart; j += 8) {
+      const int c = cp * kPart + j;
+      float x[8];
+      tmem_ld8(tmem + lane_off + TM::kD2 + c, x);
+      tmem_ld_wait();
+      *reinterpret_cast<float4*>(ht + c) = make_float4(gm * x[0], gm * x[1], gm * x[2], gm * x[3]);
+      *reinterpret_cast<float4*>(ht + c + 4) = make_float4(gm * x[4], gm * x[5], gm * x[6], gm * x[7]);
+    }
   }
 
   // ---- teardown ----------------------------------------------------------------------
@@ -681,11 +749,11 @@ cudaError_t launch_dv(const PrefillArgs& a, cudaStream_t stream) {
 
 template <typename TIn, typename TOut>
 cudaError_t launch_types(const PrefillArgs& a, cudaStream_t stream) {
-  // value-column slices per chain: split more when there are few (sequence, head)
-  // chains, so that the grid still covers the 148 SMs
+  // value-column slices per chain: split when there are few (sequence, head) chains,
+  // as far as a single wave of CTAs over the 148 SMs allows (one CTA per SM)
   const int64_t chains = static_cast<int64_t>(a.N) * a.H;
-  if (chains <= 74) return launch_dv<32, TIn, TOut>(a, stream);
-  if (chains <= 296) return launch_dv<64, TIn, TOut>(a, stream);
+  if (4 * chains <= 148) return launch_dv<32, TIn, TOut>(a, stream);
+  if (2 * chains <= 148) return launch_dv<64, TIn, TOut>(a, stream);
   return launch_dv<128, TIn, TOut>(a, stream);
 }
 
