@@ -155,6 +155,12 @@ __device__ __forceinline__ void st4_tf32(uint8_t* base, uint32_t off, float a, f
   *reinterpret_cast<float4*>(base + off) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
 }
 
+// 4 consecutive fp32 of one row as one 16-byte store, not rounded: operands whose
+// tf32 truncation costs no accuracy (Kt, W, S) skip the rounding.
+__device__ __forceinline__ void st4_f32(uint8_t* base, uint32_t off, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(base + off) = make_float4(a, b, c, d);
+}
+
 // CTA-wide OR of a predicate (every thread gets the same answer).
 __device__ __forceinline__ bool cta_any(bool x) { return __syncthreads_or(x ? 1 : 0) != 0; }
 
@@ -297,13 +303,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool failed = false;
   int gslot = 1;  // sGamma slot of the last chunk's e^{g_last} (slot 1 holds 1.0 initially)
 
-  // all threads wait for the last commit; false (everywhere) if it never came
-  auto wait_mma = [&]() -> bool {
-    const bool ok = mbar_wait(bar_mma, mma_phase, a.status);
+  // Every thread waits for the last commit on its own. A wait that runs out of time
+  // raises the status flag and marks this thread; the CTA agrees on it once per chunk
+  // and stops (after draining the tensor pipe, see the teardown).
+  bool lost = false;
+  auto wait_mma = [&]() {
+    if (!lost && !mbar_wait(bar_mma, mma_phase, a.status)) lost = true;
     mma_phase ^= 1u;
-    if (cta_any(!ok)) return false;
     tc_fence_after_sync();
-    return true;
   };
 
   // Gate inputs of one chunk for this thread (warp w: tokens 4w..4w+3, lane l: key
@@ -408,13 +415,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float g = pre[e] + la[i][e];
           const float eg = __expf(g), eng = __expf(-g);
           kt[i][e] = kv[i][e] * eg;
-          kh[i][e] = kv[i][e] * eng;
+          kh[i][e] = to_tf32(kv[i][e] * eng);
           qt[e] = qv[i][e] * eg;
         }
         const int r = r0 + i;
-        st4_tf32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[i][0], kt[i][1], kt[i][2], kt[i][3]);   // Kt [tok][ch]
+        st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[i][0], kt[i][1], kt[i][2], kt[i][3]);    // Kt [tok][ch]
         st4_tf32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);          // Qt [tok][ch]
-        st4_tf32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);    // Kh [tok][ch]
+        st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);     // Kh [tok][ch]
       }
       // channel-major copies: channel c0+e, tokens r0..r0+3; lanes rotate e so that one
       // store instruction touches different swizzle rows
@@ -427,16 +434,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           x[i] = e == 0 ? kt[i][0] : e == 1 ? kt[i][1] : e == 2 ? kt[i][2] : kt[i][3];
           y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
         }
-        st4_tf32(sm + SM::kKTT, f32_offset(c0 + e, r0, 128), x[0], x[1], x[2], x[3]);   // Kt^T [ch][tok]
-        st4_tf32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);   // Kh^T [ch][tok]
+        st4_f32(sm + SM::kKTT, f32_offset(c0 + e, r0, 128), x[0], x[1], x[2], x[3]);    // Kt^T [ch][tok]
+        st4_f32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);    // Kh^T [ch][tok]
       }
     }
 
     // -- 3. V landed: widen/transpose to V^T fp32 (rows past the sequence end -> 0) -------
     {
-      const bool ok = mbar_wait(bar_tma, tma_phase, a.status);
+      if (!lost && !mbar_wait(bar_tma, tma_phase, a.status)) lost = true;
       tma_phase ^= 1u;
-      if (cta_any(!ok)) { failed = true; break; }
+      __syncthreads();  // every thread is done with the decay totals (they share V^T's space)
       const TIn* st = reinterpret_cast<const TIn*>(sm + SM::kStage);
       for (int i = tid; i < DV * 16; i += kThreads) {
         const int j = i % DV, t4 = (i / DV) * 4;
@@ -457,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_tf32(tmem + TM::kD0, kdesc(sb + SM::kKQ, kk, 128), kdesc(sb + SM::kKH, kk, 64), kIdAP, kk > 0);
       umma_commit(bar_mma);
     }
-    if (!wait_mma()) { failed = true; break; }
+    wait_mma();
 
     // -- 5. A (rows 0..63: beta-scaled, strictly lower), P (rows 64..127: lower) ---------
     {
@@ -557,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_tf32(tmem + TM::kD3, kdesc(sb + SM::kTP, kk, 128), kdesc(sb + SM::kVT, kk, DV), kIdV, kk > 0);
       umma_commit(bar_mma);
     }
-    if (!wait_mma()) { failed = true; break; }
+    wait_mma();
 
     // -- 8. -W -> rows 0..63 of KQ (over Kt);  S <- e^{g_last}(previous chunk) S in TMEM
     //       and as the S^T operand -------------------------------------------------------
@@ -570,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; e += 4)
-          st4_tf32(sm + SM::kKQ, f32_offset(row, cb + e, 128), -w[e], -w[e + 1], -w[e + 2], -w[e + 3]);
+          st4_f32(sm + SM::kKQ, f32_offset(row, cb + e, 128), -w[e], -w[e + 1], -w[e + 2], -w[e + 3]);
       }
     }
     {
@@ -584,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           x[e] *= gm;
-          st_tf32(sm + SM::kST, f32_offset(c + e, row, DV), x[e]);
+          *reinterpret_cast<float*>(sm + SM::kST + f32_offset(c + e, row, DV)) = x[e];
         }
         tmem_st8(tmem + lane_off + TM::kD2 + c, x);
       }
@@ -606,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t nt = t0 + kChunk;
       load_gate(nt, static_cast<int>(eos - nt < kChunk ? eos - nt : kChunk));
     }
-    if (!wait_mma()) { failed = true; break; }
+    wait_mma();
 
     // -- 10. U = U~ - W S -> U^T operand (over V^T) ---------------------------------------------
     if (lq < 2) {
@@ -636,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_tf32(tmem + TM::kD1, kdesc(sb + SM::kTP, kk, 128), kdesc(sb + SM::kVT, kk, DV), kIdV, 1u);
       umma_commit(bar_mma);
     }
-    if (!wait_mma()) { failed = true; break; }
+    wait_mma();
     gslot = gnew;
 
     // -- 12. out rows <- O (* sigmoid(gate)) ------------------------------------------------------
@@ -661,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     tc_fence_before_sync();
-    __syncthreads();
+    failed = cta_any(lost);
   }
 
   // ---- final state: e^{g_last} of the last chunk times D2 --------------------------------
@@ -679,7 +686,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ---- teardown ----------------------------------------------------------------------
+  // ---- teardown: after a lost wait, let the tensor pipe and the TMA unit drain (bounded)
+  //      before the TMEM goes back -------------------------------------------------------
+  if (failed && tid == 0) {
+    umma_commit(bar_mma);
+    mbar_wait(bar_mma, mma_phase, a.status);
+    mbar_wait(bar_tma, tma_phase, a.status);
+  }
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 0) {
