@@ -75,6 +75,11 @@ kda_status check_common(int64_t total_T, int N, int H, int dk, int dv) {
 
 namespace kda {
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
+kda_status mixer_fwd_staged(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                            const float* log_alpha, const float* beta, const void* gate, const float* initial_state,
+                            const int32_t* cu_seqlens, int64_t total_T, int N, int H, void* out, float* final_state,
+                            void* scratch, cudaStream_t stream);
 }  // namespace kda
 
 extern "C" {
@@ -207,32 +212,30 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, kda_dtyp
 size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv) {
   if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
   if (dk != kda::kD || dv != kda::kD) return 0;
-  const size_t tok = static_cast<size_t>(total_T) * H * kda::kD * sizeof(float);
-  return kda::kStatusBytes + 3 * kda::align256(tok);
+  return kda::kStatusBytes;  // the conv/L2 stage runs inside the prefill kernel
 }
 
-kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
-                         const float* log_alpha, const float* beta, const void* gate, const float* initial_state,
-                         const int32_t* cu_seqlens, int64_t total_T, int N, int H, int dk, int dv, void* out,
-                         float* final_state, void* workspace, size_t workspace_bytes, kda_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+namespace {
+
+// Checks shared by the fused and the two-stage mixer entry points.
+kda_status check_mixer(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                       const float* log_alpha, const float* beta, const void* gate, const float* initial_state,
+                       const int32_t* cu_seqlens, int64_t total_T, int N, int H, int dk, int dv, void* out,
+                       float* final_state) {
   kda_status st = check_common(total_T, N, H, dk, dv);
   if (st != KDA_OK) return st;
   if (dk != kda::kD || dv != kda::kD)
     return fail(KDA_ERR_UNSUPPORTED, "the fused mixer is built for dk = dv = 128 (got %d, %d)", dk, dv);
-  if (N == 0) {
-    if (total_T != 0) return fail(KDA_ERR_INVALID_ARG, "N=0 with total_T=%lld", static_cast<long long>(total_T));
-    return ok();
-  }
-  if (!cu_seqlens && total_T % N != 0)
+  if (N == 0 && total_T != 0) return fail(KDA_ERR_INVALID_ARG, "N=0 with total_T=%lld", static_cast<long long>(total_T));
+  if (N > 0 && !cu_seqlens && total_T % N != 0)
     return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL but total_T=%lld is not a multiple of N=%d",
                 static_cast<long long>(total_T), N);
   if (total_T > 0 && (!q_raw || !k_raw || !v_raw || !conv_w || !log_alpha || !beta || !out))
     return fail(KDA_ERR_INVALID_ARG, "q_raw, k_raw, v_raw, conv_w, log_alpha, beta and out must be non-NULL");
-  const void* ptrs[] = {q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, out, final_state, workspace};
+  const void* ptrs[] = {q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, out, final_state};
   const char* names[] = {"q_raw", "k_raw", "v_raw", "conv_w", "log_alpha", "beta", "gate",
-                         "initial_state", "out", "final_state", "workspace"};
-  for (int i = 0; i < 11; ++i)
+                         "initial_state", "out", "final_state"};
+  for (int i = 0; i < 10; ++i)
     if (ptrs[i] && !aligned16(ptrs[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
   if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
     return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
@@ -240,24 +243,32 @@ kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   if (final_state && initial_state && final_state != initial_state &&
       ranges_overlap(final_state, n_st, initial_state, n_st))
     return fail(KDA_ERR_INVALID_ARG, "final_state partially overlaps initial_state");
+  return KDA_OK;
+}
+
+}  // namespace
+
+kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                         const float* log_alpha, const float* beta, const void* gate, const float* initial_state,
+                         const int32_t* cu_seqlens, int64_t total_T, int N, int H, int dk, int dv, void* out,
+                         float* final_state, void* workspace, size_t workspace_bytes, kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  kda_status st = check_mixer(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, cu_seqlens,
+                              total_T, N, H, dk, dv, out, final_state);
+  if (st != KDA_OK) return st;
+  if (N == 0) return ok();
+  if (workspace && !aligned16(workspace)) return fail(KDA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
   const size_t need = kda_mixer_fwd_workspace(total_T, N, H, dk, dv);
   if (!workspace || workspace_bytes < need)
     return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? workspace_bytes : 0, need);
-
-  char* ws = static_cast<char*>(workspace);
-  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
-  const size_t tok = kda::align256(static_cast<size_t>(total_T) * H * kda::kD * sizeof(float));
-  char* qn = ws + kda::kStatusBytes;
-  char* kn = qn + tok;
-  char* vn = kn + tok;
-  e = kda::launch_conv_l2(q_raw, k_raw, v_raw, conv_w, cu_seqlens, total_T, N, H, kda::kD, qn, kn, vn, status, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "conv/L2 kernel launch");
   kda::PrefillArgs a{};
-  a.q = qn; a.k = kn; a.v = vn; a.log_alpha = log_alpha; a.beta = beta; a.h0 = initial_state; a.cu = cu_seqlens;
-  a.gate = gate; a.out = out; a.ht = final_state; a.status = status; a.total_T = total_T; a.N = N; a.H = H;
-  a.in_f32 = true;   // conv/L2 outputs stay fp32
+  a.q = q_raw; a.k = k_raw; a.v = v_raw; a.log_alpha = log_alpha; a.beta = beta; a.h0 = initial_state;
+  a.cu = cu_seqlens; a.gate = gate; a.conv_w = conv_w; a.out = out; a.ht = final_state; a.status = status;
+  a.total_T = total_T; a.N = N; a.H = H;
+  a.in_f32 = false;  // raw bf16 q, k, v
   a.out_f32 = false;
   e = kda::launch_prefill_d128(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
@@ -278,3 +289,38 @@ kda_status kda_workspace_status(void* workspace, kda_stream_t stream_, uint32_t*
 }
 
 }  // extern "C"
+
+namespace kda {
+
+// Two-stage form of the full mixer (conv4 + L2 pre-stage into fp32 buffers in
+// `scratch`, then the recurrence on them). `scratch` holds
+// mixer_staged_scratch_bytes(total_T, H) bytes.
+kda_status mixer_fwd_staged(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                            const float* log_alpha, const float* beta, const void* gate, const float* initial_state,
+                            const int32_t* cu_seqlens, int64_t total_T, int N, int H, void* out, float* final_state,
+                            void* scratch, cudaStream_t stream) {
+  kda_status st = check_mixer(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, cu_seqlens,
+                              total_T, N, H, kD, kD, out, final_state);
+  if (st != KDA_OK) return st;
+  if (N == 0) return ok();
+  char* ws = static_cast<char*>(scratch);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  const size_t tok = align256(static_cast<size_t>(total_T) * H * kD * sizeof(float));
+  char* qn = ws + kStatusBytes;
+  char* kn = qn + tok;
+  char* vn = kn + tok;
+  e = launch_conv_l2(q_raw, k_raw, v_raw, conv_w, cu_seqlens, total_T, N, H, kD, qn, kn, vn, status, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "conv/L2 kernel launch");
+  PrefillArgs a{};
+  a.q = qn; a.k = kn; a.v = vn; a.log_alpha = log_alpha; a.beta = beta; a.h0 = initial_state; a.cu = cu_seqlens;
+  a.gate = gate; a.out = out; a.ht = final_state; a.status = status; a.total_T = total_T; a.N = N; a.H = H;
+  a.in_f32 = true;   // conv/L2 outputs stay fp32
+  a.out_f32 = false;
+  e = launch_prefill_d128(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+  return ok();
+}
+
+}  // namespace kda

@@ -32,6 +32,8 @@ struct PrefillArgs {
   const float* h0;        // fp32 [N, H, 128, 128] or null
   const int32_t* cu;      // int32 [N+1] or null (equal lengths)
   const void* gate;       // bf16 [total_T, H, 128] or null (sigmoid output gate)
+  const float* conv_w;    // fp32 [3, H*128, 4] or null: q, k, v are the raw mixer inputs and
+                          // go through conv4 (+ L2 norm of q, k) inside the kernel
   void* out;              // [total_T, H, 128], bf16 or fp32 (out_f32)
   float* ht;              // fp32 [N, H, 128, 128] or null
   uint32_t* status;       // device status word
@@ -59,8 +61,18 @@ cudaError_t launch_stage_in(const void* q, const void* k, const void* v, bool bf
 cudaError_t launch_stage_out(const void* out_p, const float* ht_p, bool bf16, int64_t total_T, int N, int H, int dk,
                              int dv, void* out, float* ht, cudaStream_t stream);
 
-// Pre-stage of the full mixer: causal depthwise conv (width 4) on q, k, v, L2 norm
-// of q and k, written in fp32 (no intermediate rounding).
+// Two-stage form of the full mixer: conv4 + L2 pre-stage into fp32 scratch buffers,
+// then the recurrence (used where the scratch is provided by the caller's side).
+kda_status mixer_fwd_staged(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                            const float* log_alpha, const float* beta, const void* gate, const float* initial_state,
+                            const int32_t* cu_seqlens, int64_t total_T, int N, int H, void* out, float* final_state,
+                            void* scratch, cudaStream_t stream);
+inline size_t mixer_staged_scratch_bytes(int64_t total_T, int H) {
+  return kStatusBytes + 3 * align256(static_cast<size_t>(total_T) * H * kD * sizeof(float));
+}
+
+// Pre-stage of the two-stage mixer: causal depthwise conv (width 4) on q, k, v, L2
+// norm of q and k, written in fp32 (no intermediate rounding).
 cudaError_t launch_conv_l2(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
                            const int32_t* cu, int64_t total_T, int N, int H, int d, void* q_o, void* k_o, void* v_o,
                            uint32_t* status, cudaStream_t stream);

@@ -5,9 +5,10 @@
 // run the mixer: a plugin inside a host framework that owns every device
 // allocation through its own pool, or a latency-critical serving loop where a
 // cudaMalloc (and the device-wide synchronisation it can imply) is not acceptable.
-// This entry point takes only inputs and outputs. Its scratch (the fp32 conv/L2
-// outputs and the device status word) lives in one file-scope __device__ array of
-// fixed size that every GPU which loads the library keeps until the process exits.
+// This entry point takes only inputs and outputs. It runs the two-stage form of the
+// mixer, whose scratch (the fp32 conv/L2 outputs and the device status word) lives in
+// one file-scope __device__ array of fixed size that every GPU which loads the
+// library keeps until the process exits.
 //
 // Contract:
 //   * scratch capacity: total_T * H <= kNoallocMaxTokenHeads (16384 token-heads,
@@ -80,11 +81,10 @@ extern "C" KDA_API kda_status kda_mixer_fwd_noalloc(const void* q_raw, const voi
              kNoallocScratchBytes);
     return noalloc_fail(total_T < 0 || H < 1 ? KDA_ERR_INVALID_ARG : KDA_ERR_UNSUPPORTED, msg);
   }
-  // Same host-side argument checks as kda_mixer_fwd, through that entry point's
-  // own validation: ask it for the workspace it would need and compare.
-  const size_t need = kda_mixer_fwd_workspace(total_T, N, H, dk, dv);
-  if (need == 0) return noalloc_fail(KDA_ERR_INVALID_ARG, "kda_mixer_fwd_noalloc: sizes rejected (dk = dv = 128 required)");
-  if (need > kNoallocScratchBytes) return noalloc_fail(KDA_ERR_UNSUPPORTED, "kda_mixer_fwd_noalloc: scratch too small");
+  if (dk != kda::kD || dv != kda::kD || kda_mixer_fwd_workspace(total_T, N, H, dk, dv) == 0)
+    return noalloc_fail(KDA_ERR_INVALID_ARG, "kda_mixer_fwd_noalloc: sizes rejected (dk = dv = 128 required)");
+  if (kda::mixer_staged_scratch_bytes(total_T, H) > kNoallocScratchBytes)
+    return noalloc_fail(KDA_ERR_UNSUPPORTED, "kda_mixer_fwd_noalloc: scratch too small");
   unsigned char* scratch = nullptr;
   const cudaError_t e = scratch_on_current_device(&scratch);
   if (e != cudaSuccess) {
@@ -92,8 +92,8 @@ extern "C" KDA_API kda_status kda_mixer_fwd_noalloc(const void* q_raw, const voi
     snprintf(msg, sizeof(msg), "kda_mixer_fwd_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
     return noalloc_fail(KDA_ERR_CUDA, msg);
   }
-  // kda_mixer_fwd clears the status word and lays its fp32 buffers out exactly as
-  // the workspace query describes; the static array stands in for the workspace.
-  return kda_mixer_fwd(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, cu_seqlens, total_T, N, H,
-                       dk, dv, out, final_state, scratch, kNoallocScratchBytes, stream_);
+  // The two-stage form of the mixer (conv/L2 outputs kept in fp32 in the static array,
+  // then the recurrence); it computes what kda_mixer_fwd computes, within rounding.
+  return kda::mixer_fwd_staged(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, cu_seqlens,
+                               total_T, N, H, out, final_state, scratch, reinterpret_cast<cudaStream_t>(stream_));
 }

@@ -201,14 +201,20 @@ __device__ __forceinline__ void warp_gemm_16x8(const float* A, const float* B, i
   *reinterpret_cast<float2*>(C + (g + 8) * kLd + 2 * t) = make_float2(scale * acc[2], scale * acc[3]);
 }
 
-template <int DV, typename TIn, typename TOut>
+// kConv: q, k, v are the raw inputs of the full mixer; the kernel applies the causal
+// depthwise conv of width 4 (zero history at each sequence start) to all three and
+// the L2 norm x / sqrt(sum x^2 + 1e-6) to q and k, in fp32, before the recurrence.
+template <int DV, typename TIn, typename TOut, bool kConv>
 __global__ void __launch_bounds__(kThreads, 1)
     kda_prefill_kernel(const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
   using SM = Smem<DV>;
   using TM = Tmem<DV>;
   constexpr int kSlices = kD / DV;
-  constexpr int kPart = DV / 4;     // value columns per warp in the TMEM epilogues
-  static_assert(64 * DV * sizeof(TIn) <= 32768, "V staging must fit in the TP region");
+  constexpr int kPart = DV / 4;          // value columns per warp in the TMEM epilogues
+  constexpr int kHist = kConv ? 3 : 0;   // tokens of history the conv needs
+  constexpr int kVRows = kChunk + kHist; // rows of the V tile brought by TMA
+  constexpr int kGRows = 4 + kHist;      // q/k rows each thread loads in the gate pass
+  static_assert(kVRows * DV * sizeof(TIn) <= 32768, "V staging must fit in the TP region");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -317,23 +323,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   // channels 4l..4l+3). The next chunk's are loaded while this chunk's MMAs run.
   const int c0 = lane * 4, r0 = warp * 4;
   float4 la4[4];   // raw loads, masked where used (keeps the loads in flight)
-  uint32_t kraw[4][sizeof(TIn)], qraw[4][sizeof(TIn)];  // 4 elements: 2 words (bf16) or 4 (fp32)
+  uint32_t kraw[kGRows][sizeof(TIn)], qraw[kGRows][sizeof(TIn)];  // 4 elements: 2 words (bf16) or 4 (fp32)
   auto load_gate = [&](int64_t tc, int lc) {
+    // q/k row m is chunk row r0 - kHist + m; rows outside [bos, tc + lc) read row tc
+    // (always in bounds) and are replaced by zero where used
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const bool in = r0 + i < lc;  // rows past the sequence end read the chunk's first row
-      const size_t o = static_cast<size_t>(tc + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
-      la4[i] = __ldg(reinterpret_cast<const float4*>(lag + o));
+    for (int m = 0; m < kGRows; ++m) {
+      const int rr = r0 - kHist + m;
+      const bool in = rr < lc && tc + rr >= bos;
+      const size_t o = static_cast<size_t>(in ? tc + rr : tc) * tok_stride + static_cast<size_t>(h) * kD + c0;
       if constexpr (sizeof(TIn) == 2) {
         const uint2 kk2 = __ldg(reinterpret_cast<const uint2*>(kg + o));
         const uint2 qq2 = __ldg(reinterpret_cast<const uint2*>(qg + o));
-        kraw[i][0] = kk2.x; kraw[i][1] = kk2.y; qraw[i][0] = qq2.x; qraw[i][1] = qq2.y;
+        kraw[m][0] = kk2.x; kraw[m][1] = kk2.y; qraw[m][0] = qq2.x; qraw[m][1] = qq2.y;
       } else {
         const uint4 kk4 = __ldg(reinterpret_cast<const uint4*>(kg + o));
         const uint4 qq4 = __ldg(reinterpret_cast<const uint4*>(qg + o));
-        kraw[i][0] = kk4.x; kraw[i][1] = kk4.y; kraw[i][2] = kk4.z; kraw[i][3] = kk4.w;
-        qraw[i][0] = qq4.x; qraw[i][1] = qq4.y; qraw[i][2] = qq4.z; qraw[i][3] = qq4.w;
+        kraw[m][0] = kk4.x; kraw[m][1] = kk4.y; kraw[m][2] = kk4.z; kraw[m][3] = kk4.w;
+        qraw[m][0] = qq4.x; qraw[m][1] = qq4.y; qraw[m][2] = qq4.z; qraw[m][3] = qq4.w;
       }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool in = r0 + i < lc;
+      const size_t o = static_cast<size_t>(tc + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
+      la4[i] = __ldg(reinterpret_cast<const float4*>(lag + o));
     }
   };
   // element e (0..3) of a raw 4-element load
@@ -353,8 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // -- 1. V tile by TMA into the staging area (the TP region, free until step 5) -----
     if (tid == 0) {
-      mbar_arrive_expect_tx(bar_tma, 64u * DV * static_cast<uint32_t>(sizeof(TIn)));
-      tma_load_3d(sm + SM::kStage, &tm_v, col0, h, static_cast<int>(t0), bar_tma);
+      mbar_arrive_expect_tx(bar_tma, static_cast<uint32_t>(kVRows * DV * sizeof(TIn)));
+      tma_load_3d(sm + SM::kStage, &tm_v, col0, h, static_cast<int>(t0) - kHist, bar_tma);
     }
     // warm L2 with the next chunk's q, k, log_alpha rows
     if (t0 + kChunk < eos && lane < 4) {
@@ -380,10 +394,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool in = r0 + i < len;
         la[i][0] = in ? la4[i].x : 0.f; la[i][1] = in ? la4[i].y : 0.f;
         la[i][2] = in ? la4[i].z : 0.f; la[i][3] = in ? la4[i].w : 0.f;
+      }
+      if constexpr (kConv) {
+        // y[t, c] = sum_j w[c, j] x[t - 3 + j, c] (x = 0 before the sequence start), then
+        // x / sqrt(sum_c y^2 + 1e-6) over the head's 128 channels (this warp holds them all)
+        float wq[4][4], wk[4][4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          kv[i][e] = in ? unpack(kraw[i], e) : 0.f;
-          qv[i][e] = in ? unpack(qraw[i], e) : 0.f;
+          const float4 a4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((0 * H + h) * kD + c0 + e) * 4));
+          const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((1 * H + h) * kD + c0 + e) * 4));
+          wq[e][0] = a4.x; wq[e][1] = a4.y; wq[e][2] = a4.z; wq[e][3] = a4.w;
+          wk[e][0] = b4.x; wk[e][1] = b4.y; wk[e][2] = b4.z; wk[e][3] = b4.w;
+        }
+        bool rin[kGRows];
+#pragma unroll
+        for (int m = 0; m < kGRows; ++m) rin[m] = (r0 - kHist + m) < len && t0 + (r0 - kHist + m) >= bos;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float sq = 0.f, sk = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float yq = 0.f, yk = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int m = i + j;
+              yq = fmaf(wq[e][j], rin[m] ? unpack(qraw[m], e) : 0.f, yq);
+              yk = fmaf(wk[e][j], rin[m] ? unpack(kraw[m], e) : 0.f, yk);
+            }
+            qv[i][e] = yq;
+            kv[i][e] = yk;
+            sq = fmaf(yq, yq, sq);
+            sk = fmaf(yk, yk, sk);
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+          }
+          const bool in = r0 + i < len;
+          const float fq = in ? rsqrtf(sq + 1e-6f) : 0.f, fk = in ? rsqrtf(sk + 1e-6f) : 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qv[i][e] *= fq;
+            kv[i][e] *= fk;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const bool in = r0 + i < len;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kv[i][e] = in ? unpack(kraw[i], e) : 0.f;
+            qv[i][e] = in ? unpack(qraw[i], e) : 0.f;
+          }
         }
       }
       // running sums within this warp's 4 tokens, then the totals of the warps before it
@@ -444,12 +508,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!lost && !mbar_wait(bar_tma, tma_phase, a.status)) lost = true;
       tma_phase ^= 1u;
       __syncthreads();  // every thread is done with the decay totals (they share V^T's space)
-      const TIn* st = reinterpret_cast<const TIn*>(sm + SM::kStage);
+      const TIn* st = reinterpret_cast<const TIn*>(sm + SM::kStage);  // row m = token t0 - kHist + m
       for (int i = tid; i < DV * 16; i += kThreads) {
         const int j = i % DV, t4 = (i / DV) * 4;
         float x[4];
+        if constexpr (kConv) {
+          const float4 w4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((2 * H + h) * kD + col0 + j) * 4));
+          const float w[4] = {w4.x, w4.y, w4.z, w4.w};
+          float xs[7];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = (t4 + e < len) ? as_f32(st[(t4 + e) * DV + j]) : 0.f;
+          for (int m = 0; m < 7; ++m) xs[m] = (t0 - kHist + t4 + m >= bos) ? as_f32(st[(t4 + m) * DV + j]) : 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float y = 0.f;
+#pragma unroll
+            for (int tap = 0; tap < 4; ++tap) y = fmaf(w[tap], xs[e + tap], y);
+            x[e] = (t4 + e < len) ? y : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] = (t4 + e < len) ? as_f32(st[(t4 + e) * DV + j]) : 0.f;
+        }
         st4_tf32(sm + SM::kVT, f32_offset(j, t4, DV), x[0], x[1], x[2], x[3]);
       }
     }
@@ -726,16 +805,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [total_T, H, 128] (bf16 or fp32) viewed as (d, head, token); box = (box_d, 1, 64),
+// [total_T, H, 128] (bf16 or fp32) viewed as (d, head, token); box = (box_d, 1, rows),
 // rows land unswizzled (box_d elements each)
-bool encode_value_map(CUtensorMap* m, const void* ptr, int64_t total_T, int H, int box_d, bool f32) {
+bool encode_value_map(CUtensorMap* m, const void* ptr, int64_t total_T, int H, int box_d, int rows, bool f32) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t es = f32 ? 4 : 2;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(total_T)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * es, static_cast<cuuint64_t>(H) * kD * es};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_d), 1u, static_cast<cuuint32_t>(kChunk)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_d), 1u, static_cast<cuuint32_t>(rows)};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                         const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -744,11 +823,12 @@ bool encode_value_map(CUtensorMap* m, const void* ptr, int64_t total_T, int H, i
   return r == CUDA_SUCCESS;
 }
 
-template <int DV, typename TIn, typename TOut>
+template <int DV, typename TIn, typename TOut, bool kConv>
 cudaError_t launch_dv(const PrefillArgs& a, cudaStream_t stream) {
   CUtensorMap tm;
-  if (!encode_value_map(&tm, a.v, a.total_T, a.H, DV, sizeof(TIn) == 4)) return cudaErrorInvalidValue;
-  auto kern = kda_prefill_kernel<DV, TIn, TOut>;
+  if (!encode_value_map(&tm, a.v, a.total_T, a.H, DV, kChunk + (kConv ? 3 : 0), sizeof(TIn) == 4))
+    return cudaErrorInvalidValue;
+  auto kern = kda_prefill_kernel<DV, TIn, TOut, kConv>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -760,14 +840,14 @@ cudaError_t launch_dv(const PrefillArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <typename TIn, typename TOut>
+template <typename TIn, typename TOut, bool kConv>
 cudaError_t launch_types(const PrefillArgs& a, cudaStream_t stream) {
   // value-column slices per chain: split when there are few (sequence, head) chains,
   // as far as a single wave of CTAs over the 148 SMs allows (one CTA per SM)
   const int64_t chains = static_cast<int64_t>(a.N) * a.H;
-  if (4 * chains <= 148) return launch_dv<32, TIn, TOut>(a, stream);
-  if (2 * chains <= 148) return launch_dv<64, TIn, TOut>(a, stream);
-  return launch_dv<128, TIn, TOut>(a, stream);
+  if (4 * chains <= 148) return launch_dv<32, TIn, TOut, kConv>(a, stream);
+  if (2 * chains <= 148) return launch_dv<64, TIn, TOut, kConv>(a, stream);
+  return launch_dv<128, TIn, TOut, kConv>(a, stream);
 }
 
 }  // namespace
@@ -781,8 +861,12 @@ cudaError_t launch_prefill_d128(const PrefillArgs& a, cudaStream_t stream) {
         a.h0, a.ht, n4);
     return cudaGetLastError();
   }
-  if (!a.in_f32) return a.out_f32 ? cudaErrorInvalidValue : launch_types<__nv_bfloat16, __nv_bfloat16>(a, stream);
-  return a.out_f32 ? launch_types<float, float>(a, stream) : launch_types<float, __nv_bfloat16>(a, stream);
+  if (a.conv_w) {  // the fused full mixer: raw bf16 q/k/v, bf16 out
+    if (a.in_f32 || a.out_f32) return cudaErrorInvalidValue;
+    return launch_types<__nv_bfloat16, __nv_bfloat16, true>(a, stream);
+  }
+  if (!a.in_f32) return a.out_f32 ? cudaErrorInvalidValue : launch_types<__nv_bfloat16, __nv_bfloat16, false>(a, stream);
+  return a.out_f32 ? launch_types<float, float, false>(a, stream) : launch_types<float, __nv_bfloat16, false>(a, stream);
 }
 
 }  // namespace kda

@@ -145,7 +145,8 @@ KDA_API kda_status kda_decode_step(const void* q, const void* k, const void* v, 
                            const float* log_alpha, const float* beta, float* state,
                            int N, int H, int dk, int dv, void* out, kda_stream_t stream);
 
-/* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes). */
+/* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes). The
+ * conv/L2 stage runs inside the prefill kernel, so this is the status word only. */
 KDA_API size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv);
 
 /*
@@ -174,8 +175,9 @@ KDA_API kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const voi
  * Full mixer prefill without a workspace, for callers that cannot allocate device
  * memory where they run the mixer (a plugin whose host framework owns every device
  * allocation, a serving loop that may not call cudaMalloc). The paper has no
- * counterpart: this is a packaging of kda_mixer_fwd, same arguments minus the
- * workspace, same results.
+ * counterpart: it takes kda_mixer_fwd's arguments minus the workspace and runs the
+ * mixer in two stages (conv/L2 into fp32 scratch, then the recurrence); results
+ * match kda_mixer_fwd within the parity tolerance.
  *
  * Scratch is a fixed array in the library's device memory (about 24 MiB per GPU
  * that loads the library, held until the process exits). Limit: total_T * H <=

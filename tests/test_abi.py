@@ -50,7 +50,7 @@ def test_workspace_query(lib):
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 0, 16, kda.KDA_DT_F32) == 0
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 129, 16, kda.KDA_DT_BF16) == 0
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 16, 16, 7) == 0
-    assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 128, 128) >= 3 * 1000 * 32 * 128 * 2
+    assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 128, 128) == 256  # status word; conv runs in-kernel
     assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 64, 64) == 0
 
 
