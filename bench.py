@@ -38,6 +38,11 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # ----------------------------------------------------------------------------------
 # algorithmic work (bytes / flops the method must move or do, per call)
 # ----------------------------------------------------------------------------------
+# kernels one kda_chunk_fwd / kda_mixer_fwd call launches: the chunk plan, the
+# intra-chunk pass over all chunks, the recurrence over each chain's chunks
+PREFILL_KERNELS = 3
+
+
 def prefill_bytes(total_T: int, N: int, Hh: int = H, d: int = D, with_h0: bool = True, mixer: bool = False) -> int:
     """q, k, v, out (bf16) + log_alpha (fp32) + beta (fp32) + states in/out (fp32).
     The full mixer adds the gate (bf16) and conv weights; its q, k, v are the raw ones."""
@@ -255,7 +260,7 @@ def run_gpu(args):
 
     with ClockSampler(device.index) as clk:
         per, total_ms = time_region(step, args.steps, args.warmup, stream, device)
-    launches += args.steps
+    launches += PREFILL_KERNELS * args.steps
     kda.workspace_status(ws)
     clocks = clk.summary()
     total_ms_max = max_over_ranks(total_ms, device)
@@ -336,7 +341,7 @@ def run_gpu(args):
 
         msteps = max(3, min(args.steps, 10))
         mper, mtot = time_region(mstep, msteps, 2, stream, device)
-        launches += 2 * msteps
+        launches += PREFILL_KERNELS * msteps
         mtot = max_over_ranks(mtot, device)
         mbytes = prefill_bytes(Bm * Tm, Bm, with_h0=False, mixer=True)
         mms = statistics.mean(mper)
@@ -356,14 +361,16 @@ def run_gpu(args):
         vi = device_prefill_inputs(TT, H, D, 1370004, device, state_N=len(lens))
         vo = torch.empty(TT, H, D, dtype=torch.bfloat16, device=device)
         vf = torch.empty(len(lens), H, D, D, dtype=torch.float32, device=device)
+        vws = torch.empty(kda.chunk_fwd_workspace_bytes(TT, len(lens), H, D, D, kda.KDA_DT_BF16), dtype=torch.uint8,
+                          device=device)
 
         def vstep(i):
             kda.chunk_fwd(vi["q"], vi["k"], vi["v"], vi["log_alpha"], vi["beta"], vi["initial_state"], cu,
-                          N=len(lens), out=vo, final_state=vf, workspace=ws, stream=stream)
+                          N=len(lens), out=vo, final_state=vf, workspace=vws, stream=stream)
 
         vsteps = max(3, min(args.steps, 10))
         vper, vtot = time_region(vstep, vsteps, 2, stream, device)
-        launches += vsteps
+        launches += PREFILL_KERNELS * vsteps
         vtot = max_over_ranks(vtot, device)
         vbytes = prefill_bytes(TT, len(lens))
         vms = statistics.mean(vper)
@@ -372,7 +379,7 @@ def run_gpu(args):
                "roofline": {"bound": "hbm", "achieved": vbytes / (vms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                             "frac": vbytes / (vms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_launch": vbytes},
                "tensor_tflops": prefill_tc_flops(TT) / (vms * 1e-3) / 1e12}
-        del vi, vo, vf
+        del vi, vo, vf, vws
 
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
 
@@ -387,7 +394,8 @@ def run_gpu(args):
                        "l2": f"inputs rotate through {n_sets} device copies ({n_sets * bytes_call / 1e6:.0f} MB > L2)"},
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved_gbs / hbm_peak, "traffic": args.traffic,
-                         "kernel": "kda_prefill_kernel<32>", "algorithmic_bytes_per_launch": bytes_call,
+                         "kernel": "kda_chunk_fwd (plan + intra-chunk + recurrence kernels, one call)",
+                         "algorithmic_bytes_per_launch": bytes_call,
                          "kernel_us": kern_ms * 1e3, "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src}, burst copy)",
                          "tensor": {"achieved_tflops": tc_tflops, "peak_tflops": tc_peak,
                                     "frac": tc_tflops / tc_peak, "flops_per_launch": prefill_tc_flops(T1)}},

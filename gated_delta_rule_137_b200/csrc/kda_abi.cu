@@ -103,8 +103,9 @@ const char* kda_version(void) { return "0.1.0"; }
 size_t kda_chunk_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv, kda_dtype qkv_dtype) {
   if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
   if (qkv_dtype != KDA_DT_F32 && qkv_dtype != KDA_DT_BF16) return 0;
-  if (!needs_staging(dk, dv)) return kda::kStatusBytes;
-  return stage_layout(total_T, N, H, elem_size(qkv_dtype)).total;
+  const size_t base = needs_staging(dk, dv) ? stage_layout(total_T, N, H, elem_size(qkv_dtype)).total
+                                           : kda::kStatusBytes;
+  return base + kda::split_workspace_bytes(total_T, N, H);
 }
 
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype qkv_dtype, const float* log_alpha,
@@ -159,6 +160,8 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype 
   a.N = N;
   a.H = H;
   a.in_f32 = a.out_f32 = (qkv_dtype == KDA_DT_F32);
+  if (kda::split_workspace_bytes(total_T, N, H) > 0)
+    a.split_ws = ws + (needs_staging(dk, dv) ? stage_layout(total_T, N, H, es).total : kda::kStatusBytes);
   if (!needs_staging(dk, dv)) {
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.h0 = initial_state;
     a.out = out; a.ht = final_state;
@@ -212,7 +215,8 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, kda_dtyp
 size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv) {
   if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
   if (dk != kda::kD || dv != kda::kD) return 0;
-  return kda::kStatusBytes;  // the conv/L2 stage runs inside the prefill kernel
+  // status word + the two-pass prefill's scratch (the conv/L2 stage runs inside it)
+  return kda::kStatusBytes + kda::split_workspace_bytes(total_T, N, H);
 }
 
 namespace {
@@ -270,6 +274,7 @@ kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   a.total_T = total_T; a.N = N; a.H = H;
   a.in_f32 = false;  // raw bf16 q, k, v
   a.out_f32 = false;
+  if (kda::split_workspace_bytes(total_T, N, H) > 0) a.split_ws = static_cast<char*>(workspace) + kda::kStatusBytes;
   e = kda::launch_prefill_d128(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return ok();

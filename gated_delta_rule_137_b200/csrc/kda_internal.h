@@ -41,7 +41,31 @@ struct PrefillArgs {
   int N, H;
   bool in_f32;            // q, k, v are fp32 (else bf16)
   bool out_f32;           // out is fp32 (else bf16)
+  void* split_ws;         // split_workspace_bytes() of scratch for the two-pass prefill, or
+                          // null for the single-pass kernel
 };
+
+// ---- two-pass prefill (kda_split.cu) ---------------------------------------------------
+// Pass 1 writes one item of kItemBytes per (chunk, head) — the state-independent part
+// of the chunk; pass 2 runs the recurrence over them. Scratch: the per-sequence chunk
+// offsets, then the items. Above kSplitMaxItemBytes of items the single-pass kernel is
+// used instead (it needs no scratch).
+constexpr size_t kItemBytes = 147968;
+constexpr size_t kSplitMaxItemBytes = size_t{32} << 30;
+// Upper bound on the number of 64-token chunks over all sequences (each sequence adds at
+// most one partial chunk; every chunk holds at least one token).
+inline int64_t split_max_chunks(int64_t total_T, int N) {
+  const int64_t c = total_T / kChunk + N;
+  return c < total_T ? c : total_T;
+}
+inline size_t split_plan_bytes(int N) { return align256((static_cast<size_t>(N) + 1) * sizeof(int32_t)); }
+inline size_t split_workspace_bytes(int64_t total_T, int N, int H) {
+  if (total_T <= 0 || N <= 0) return 0;
+  const size_t items = static_cast<size_t>(split_max_chunks(total_T, N)) * static_cast<size_t>(H) * kItemBytes;
+  if (items > kSplitMaxItemBytes) return 0;
+  return split_plan_bytes(N) + items;
+}
+cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream);
 
 // Sets the message kda_last_error() returns on this host thread.
 void set_last_error(const char* msg);

@@ -1,0 +1,222 @@
+// kda_tile.cuh — device helpers shared by the prefill kernels: operand-tile
+// descriptors, vector loads/stores of inputs and outputs, tf32 rounding stores into
+// 128B-swizzled fp32 tiles, the fp32-accurate 64x64 unit-lower-triangular inverse,
+// and the host-side TMA descriptor encoding. Internal to the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "kda_internal.h"
+
+namespace kda {
+namespace {
+
+constexpr float kMaxChunkDecay = 80.f;
+constexpr int kLd = 68;  // row stride (floats) of the fp32 solve scratch (16-B aligned rows)
+
+// K-major fp32 operand tile with `rows` rows (M or N): descriptor of K step 0, and the
+// constant to add for K step kk (8 columns per step: 32 B within a 128-B row, then
+// the next 32-column block `rows` rows further). The start-address field holds
+// address / 16 in its low 14 bits and shared memory is < 256 KB, so the sum never
+// carries out of the field.
+__device__ __forceinline__ uint64_t kdesc0(uint32_t base) { return sdesc(base, 16u, 1024u, kSwz128); }
+__host__ __device__ constexpr uint64_t kstep(int kk, uint32_t rows) {
+  return static_cast<uint64_t>(((kk >> 2) * rows * 128u + (kk & 3) * 32u) >> 4);
+}
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// read-only loads of an input element as fp32
+__device__ __forceinline__ float ld_in(const __nv_bfloat16* p) { return __bfloat162float(__ldg(p)); }
+__device__ __forceinline__ float ld_in(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float as_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float as_f32(float x) { return x; }
+
+// 4 consecutive input elements (8-byte bf16 or 16-byte fp32 read-only load)
+__device__ __forceinline__ void ld4_in(const __nv_bfloat16* p, float* o) {
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p));
+  const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
+  o[0] = __bfloat162float(b[0]); o[1] = __bfloat162float(b[1]);
+  o[2] = __bfloat162float(b[2]); o[3] = __bfloat162float(b[3]);
+}
+__device__ __forceinline__ void ld4_in(const float* p, float* o) {
+  const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+  o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+}
+
+// 8 consecutive output values of one row (TOut = bf16 or fp32)
+__device__ __forceinline__ void store8(__nv_bfloat16* dst, const float* o) {
+  uint4 p;
+  p.x = pack_bf16x2(o[0], o[1]); p.y = pack_bf16x2(o[2], o[3]);
+  p.z = pack_bf16x2(o[4], o[5]); p.w = pack_bf16x2(o[6], o[7]);
+  *reinterpret_cast<uint4*>(dst) = p;
+}
+__device__ __forceinline__ void store8(float* dst, const float* o) {
+  *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+  *reinterpret_cast<float4*>(dst + 4) = make_float4(o[4], o[5], o[6], o[7]);
+}
+
+// 16 consecutive output values of one row (TOut = bf16 or fp32)
+__device__ __forceinline__ void store16(__nv_bfloat16* dst, const float* o) {
+  uint4 p0, p1;
+  p0.x = pack_bf16x2(o[0], o[1]);   p0.y = pack_bf16x2(o[2], o[3]);
+  p0.z = pack_bf16x2(o[4], o[5]);   p0.w = pack_bf16x2(o[6], o[7]);
+  p1.x = pack_bf16x2(o[8], o[9]);   p1.y = pack_bf16x2(o[10], o[11]);
+  p1.z = pack_bf16x2(o[12], o[13]); p1.w = pack_bf16x2(o[14], o[15]);
+  reinterpret_cast<uint4*>(dst)[0] = p0;
+  reinterpret_cast<uint4*>(dst)[1] = p1;
+}
+__device__ __forceinline__ void store16(float* dst, const float* o) {
+#pragma unroll
+  for (int i = 0; i < 16; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+}
+
+__device__ __forceinline__ void st_tf32(uint8_t* base, uint32_t off, float v) {
+  *reinterpret_cast<float*>(base + off) = to_tf32(v);
+}
+// 4 consecutive fp32 of one row (4-aligned column) as one 16-byte store, tf32-rounded.
+__device__ __forceinline__ void st4_tf32(uint8_t* base, uint32_t off, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(base + off) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
+}
+
+// 4 consecutive fp32 of one row as one 16-byte store, not rounded: operands whose
+// tf32 truncation costs no accuracy (Kt, W, S) skip the rounding.
+__device__ __forceinline__ void st4_f32(uint8_t* base, uint32_t off, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(base + off) = make_float4(a, b, c, d);
+}
+
+// CTA-wide OR of a predicate (every thread gets the same answer).
+__device__ __forceinline__ bool cta_any(bool x) { return __syncthreads_or(x ? 1 : 0) != 0; }
+
+// ---- small fp32-accurate products for the triangular solve (warp-level mma.sync) ----
+// x = hi + lo with hi, lo representable in tf32; the 3-term product hi*hi + hi*lo + lo*hi
+// keeps close to fp32 accuracy on the tensor pipe.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  const float h = to_tf32(x);
+  hi = __float_as_uint(h);
+  lo = __float_as_uint(to_tf32(x - h));
+}
+
+__device__ __forceinline__ void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// One warp: C (16 x 8) = scale * A (16 x K, row stride kLd) * B (K x 8, row stride kLd),
+// fp32 in shared memory, K a multiple of 8; C stored with row stride kLd.
+__device__ __forceinline__ void warp_gemm_16x8(const float* A, const float* B, int K, float* C, float scale) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k = 0; k < K; k += 8) {
+    uint32_t ah[4], al[4], bh[2], bl[2];
+    split_tf32(A[g * kLd + k + t], ah[0], al[0]);
+    split_tf32(A[(g + 8) * kLd + k + t], ah[1], al[1]);
+    split_tf32(A[g * kLd + k + t + 4], ah[2], al[2]);
+    split_tf32(A[(g + 8) * kLd + k + t + 4], ah[3], al[3]);
+    split_tf32(B[(k + t) * kLd + g], bh[0], bl[0]);
+    split_tf32(B[(k + t + 4) * kLd + g], bh[1], bl[1]);
+    mma_m16n8k8_tf32(acc, al, bh);
+    mma_m16n8k8_tf32(acc, ah, bl);
+    mma_m16n8k8_tf32(acc, ah, bh);
+  }
+  *reinterpret_cast<float2*>(C + g * kLd + 2 * t) = make_float2(scale * acc[0], scale * acc[1]);
+  *reinterpret_cast<float2*>(C + (g + 8) * kLd + 2 * t) = make_float2(scale * acc[2], scale * acc[3]);
+}
+
+
+// ---- X = (I + A)^-1 for a strictly lower 64x64 A in fp32 ----------------------------
+// sA: A in [64][kLd] on entry, X in place on return; sY: [32][kLd] scratch. Called by
+// every thread of a CTA of at least 256 threads (warps 0..7 work; all take the barriers).
+// 16x16 diagonal blocks by forward substitution in registers, then two levels of block
+// doubling: [[X1, 0], [A21, X2]]^-1 has lower-left block -X2 (A21 X1).
+__device__ __forceinline__ void invert_unit_lower_64(float* sA, float* sY) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // warp b < 4 owns diagonal block b; lane (r = lane % 16, half hh) holds row r,
+  // columns 8hh..8hh+7
+  if (warp < 4) {
+    const int b = warp, r = lane & 15, hh = lane >> 4;
+    float* Arow = sA + (16 * b + r) * kLd + 16 * b;
+    float av[16], x[8];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) av[i] = Arow[i];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = (8 * hh + j == r) ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 0; i < 15; ++i) {  // row i is final: rows below subtract A[r][i] * row i
+      const float c = (r > i) ? av[i] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = fmaf(-c, __shfl_sync(0xffffffffu, x[j], i + 16 * hh), x[j]);
+    }
+    __syncwarp();
+    *reinterpret_cast<float4*>(Arow + 8 * hh) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4*>(Arow + 8 * hh + 4) = make_float4(x[4], x[5], x[6], x[7]);
+  }
+  __syncthreads();
+  // 16 -> 32 on the two diagonal pairs (warp = pair * 2 + 8-column tile) ...
+  if (warp < 4) {
+    const int p = warp >> 1, nt = warp & 1, o = 32 * p;
+    warp_gemm_16x8(sA + (o + 16) * kLd + o, sA + o * kLd + o + 8 * nt, 16, sY + 16 * p + 8 * nt, 1.f);
+  }
+  __syncthreads();
+  if (warp < 4) {
+    const int p = warp >> 1, nt = warp & 1, o = 32 * p;
+    warp_gemm_16x8(sA + (o + 16) * kLd + o + 16, sY + 16 * p + 8 * nt, 16, sA + (o + 16) * kLd + o + 8 * nt, -1.f);
+  }
+  __syncthreads();
+  // ... then 32 -> 64 (warp = 16-row tile * 4 + 8-column tile)
+  if (warp < 8) {
+    const int mt = warp >> 2, nt = warp & 3;
+    warp_gemm_16x8(sA + (32 + 16 * mt) * kLd, sA + 8 * nt, 32, sY + (16 * mt) * kLd + 8 * nt, 1.f);
+  }
+  __syncthreads();
+  if (warp < 8) {
+    const int mt = warp >> 2, nt = warp & 3;
+    warp_gemm_16x8(sA + (32 + 16 * mt) * kLd + 32, sY + 8 * nt, 32, sA + (32 + 16 * mt) * kLd + 8 * nt, -1.f);
+  }
+  __syncthreads();
+}
+
+// ---- TMA descriptor encoding through the driver entry point ----------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [total_T, H, 128] (bf16 or fp32) viewed as (d, head, token); box = (box_d, 1, rows),
+// rows land unswizzled (box_d elements each)
+bool encode_value_map(CUtensorMap* m, const void* ptr, int64_t total_T, int H, int box_d, int rows, bool f32) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t es = f32 ? 4 : 2;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total_T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * es, static_cast<cuuint64_t>(H) * kD * es};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_d), 1u, static_cast<cuuint32_t>(rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace kda

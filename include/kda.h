@@ -35,9 +35,9 @@
  * - Problems that only the device can see (a cu_seqlens that is not
  *   non-decreasing or overruns total_T; a chunk whose per-channel decay exceeds
  *   the documented range) set bits in a status word held in `workspace`; the
- *   affected (sequence, head) pairs are skipped and their outputs left
- *   unspecified. Read the word with kda_workspace_status() after the stream
- *   has run the call.
+ *   outputs are then unspecified (a bad cu_seqlens may leave every sequence
+ *   unwritten). Read the word with kda_workspace_status() after the stream has
+ *   run the call.
  * - Thread safety: calls may be issued from several host threads; the message
  *   returned by kda_last_error() is thread-local.
  */
@@ -90,6 +90,12 @@ KDA_API const char* kda_version(void);
  * Workspace, in bytes, that kda_chunk_fwd needs for these sizes (a multiple of
  * 256; never 0, the status word always lives there). Returns 0 for sizes the
  * library rejects.
+ *
+ * Beyond the status word (and, for head dims below 128, zero-padded copies of
+ * the inputs), the workspace holds the scratch of the two-pass prefill: about
+ * 145 KB per (64-token chunk, head), e.g. 303 MB for one 4096-token sequence of
+ * 32 heads. When that scratch would exceed 32 GiB the call runs a single-pass
+ * kernel instead (slower, no scratch) and the query leaves it out.
  */
 KDA_API size_t kda_chunk_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv, kda_dtype qkv_dtype);
 
@@ -145,8 +151,9 @@ KDA_API kda_status kda_decode_step(const void* q, const void* k, const void* v, 
                            const float* log_alpha, const float* beta, float* state,
                            int N, int H, int dk, int dv, void* out, kda_stream_t stream);
 
-/* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes). The
- * conv/L2 stage runs inside the prefill kernel, so this is the status word only. */
+/* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes): the
+ * status word plus the two-pass prefill's scratch, sized as for kda_chunk_fwd (the
+ * conv/L2 stage runs inside the prefill's first pass and needs no buffer of its own). */
 KDA_API size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv);
 
 /*

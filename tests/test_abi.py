@@ -43,14 +43,23 @@ def test_status_strings(lib):
 
 
 def test_workspace_query(lib):
+    item = 147968  # two-pass scratch per (64-token chunk, head)
     ws = lib.kda_chunk_fwd_workspace(4096, 1, 32, 128, 128, kda.KDA_DT_BF16)
-    assert ws >= 4 and ws % 256 == 0
+    # status word + chunk offsets + items for at most 4096/64 + 1 chunks per head
+    assert ws == 256 + 256 + (64 + 1) * 32 * item
+    assert ws % 256 == 0
+    full = lib.kda_chunk_fwd_workspace(64, 1, 2, 128, 128, kda.KDA_DT_F32)
     small = lib.kda_chunk_fwd_workspace(64, 1, 2, 16, 16, kda.KDA_DT_F32)
-    assert small > ws  # staging buffers for fp32 / d < 128
+    assert small > full  # zero-padded staging copies for d < 128
+    assert full == 256 + 256 + 2 * 2 * item  # bound min(T/64 + N, T) = 2 chunks, 2 heads
+    assert lib.kda_chunk_fwd_workspace(0, 1, 2, 128, 128, kda.KDA_DT_F32) == 256  # no tokens: status word only
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 0, 16, kda.KDA_DT_F32) == 0
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 129, 16, kda.KDA_DT_BF16) == 0
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 16, 16, 7) == 0
-    assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 128, 128) == 256  # status word; conv runs in-kernel
+    # beyond 32 GiB of scratch the single-pass kernel runs and the query drops the scratch
+    huge_T = (1 << 31) - 1024
+    assert lib.kda_chunk_fwd_workspace(huge_T, 1, 32, 128, 128, kda.KDA_DT_BF16) == 256
+    assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 128, 128) == 256 + 256 + (1000 // 64 + 2) * 32 * item
     assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 64, 64) == 0
 
 

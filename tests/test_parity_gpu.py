@@ -158,6 +158,25 @@ def test_prefill_varlen_sampled(kda):
         assert_prefill_close(fin[n:n + 1, h:h + 1], rf, f"final seq {n} head {h}")
 
 
+def test_prefill_many_short_sequences(kda):
+    """1500 packed sequences (more than one 1024-wide block of the chunk-offset scan),
+    mostly 0..5 tokens with a few longer ones; oracle on a sample of sequences."""
+    rng = np.random.default_rng(I.SEED_BASE + 31)
+    lens = [int(x) for x in rng.integers(0, 6, 1500)]
+    for i, L in ((3, 70), (1024, 130), (1499, 64)):
+        lens[i] = L
+    w = I.make_prefill(lens, 1, 128, 128, seed=I.SEED_BASE + 32)
+    out, fin = _run_prefill(kda, w)
+    picks = sorted(set([3, 1023, 1024, 1025, 1499] + list(range(0, 1500, 97))))
+    for n in picks:
+        s, e = int(w.cu_seqlens[n]), int(w.cu_seqlens[n + 1])
+        ro, rf = O.kda_recurrence(w.q[s:e], w.k[s:e], w.v[s:e], w.log_alpha[s:e], w.beta[s:e],
+                                  w.initial_state[n:n + 1], np.array([0, e - s]))
+        if e > s:
+            assert_prefill_close(out[s:e], ro, f"out seq {n} (len {e - s})", stored_bf16=True)
+        assert_prefill_close(fin[n:n + 1], rf, f"final seq {n} (len {e - s})")
+
+
 def test_prefill_split_and_state_alias(kda):
     """run(T) == run(T1) then run(T - T1) from the carried state, with final_state
     written over initial_state in place; and prefill then one decode step equals
