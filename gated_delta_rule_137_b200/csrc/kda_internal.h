@@ -48,8 +48,12 @@ struct PrefillArgs {
 // ---- two-pass prefill (kda_split.cu) ---------------------------------------------------
 // Pass 1 writes one item of kItemBytes per (chunk, head) — the state-independent part
 // of the chunk; pass 2 runs the recurrence over them. Scratch: the per-sequence chunk
-// offsets, then the items. Above kSplitMaxItemBytes of items the single-pass kernel is
-// used instead (it needs no scratch).
+// offsets, then the items.
+// The split pays when there are few (sequence, head) chains: the single-pass kernel
+// then has to cut each chain into value-column slices that all redo the chunk's
+// state-free work. With more than kSplitMaxChains chains it runs whole chains per CTA
+// with nothing repeated, and stays the faster form; it is used there, and above
+// kSplitMaxItemBytes of items (it needs no scratch).
 constexpr size_t kItemBytes = 147968;
 constexpr size_t kSplitMaxItemBytes = size_t{32} << 30;
 // Upper bound on the number of 64-token chunks over all sequences (each sequence adds at
@@ -59,8 +63,10 @@ inline int64_t split_max_chunks(int64_t total_T, int N) {
   return c < total_T ? c : total_T;
 }
 inline size_t split_plan_bytes(int N) { return align256((static_cast<size_t>(N) + 1) * sizeof(int32_t)); }
+constexpr int64_t kSplitMaxChains = 74;  // half of the 148 SMs: beyond it no slicing is needed
 inline size_t split_workspace_bytes(int64_t total_T, int N, int H) {
   if (total_T <= 0 || N <= 0) return 0;
+  if (static_cast<int64_t>(N) * H > kSplitMaxChains) return 0;
   const size_t items = static_cast<size_t>(split_max_chunks(total_T, N)) * static_cast<size_t>(H) * kItemBytes;
   if (items > kSplitMaxItemBytes) return 0;
   return split_plan_bytes(N) + items;

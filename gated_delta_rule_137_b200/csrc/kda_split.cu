@@ -17,7 +17,7 @@
 //       [-W; Qt]  128 x 128 fp32 tile   (A operand of D1 = [-W; Qt] S)
 //       P         rows 64..127 of a 128 x 64 tile (A operand of D1 += [.; P] U)
 //       Kh^T      128 x 64 tile         (A operand of D2 += Kh^T U)
-//       U~        64 x 128 fp32, row-major
+//       U~        64 x 128 fp32 (same swizzled layout, read back row by row)
 //       e^g_last  128 fp32
 //     The three tiles are written in the exact 128B-swizzled K-major layout the MMAs
 //     read, so pass 2 moves them into shared memory with plain bulk copies;
@@ -48,7 +48,7 @@ namespace {
 constexpr uint32_t kItemQW = 0;          // [-W; Qt] tile, 64 KB
 constexpr uint32_t kItemP = 65536;       // P: rows 64..127 of K blocks 0 and 1, 2 x 8 KB
 constexpr uint32_t kItemKHT = 81920;     // Kh^T tile, 32 KB
-constexpr uint32_t kItemU = 114688;      // U~ [64][128] fp32, 32 KB
+constexpr uint32_t kItemU = 114688;      // U~ 64 x 128 fp32 in the 64-row tile layout, 32 KB
 constexpr uint32_t kItemGamma = 147456;  // e^g_last [128] fp32
 static_assert(kItemGamma + 512 == kItemBytes, "item layout");
 
@@ -108,94 +108,118 @@ __global__ void __launch_bounds__(1024) kda_plan_kernel(const int32_t* __restric
 }
 
 // ================================ pass 1 =============================================
-constexpr int kIntraThreads = 512;  // 16 warps; warp w: tokens 4w..4w+3 in the gate pass
+// Persistent: each CTA walks the items it = blockIdx.x + k * gridDim.x (item = global
+// chunk it / H, head it % H). Two warp groups work on consecutive items at once:
+//   front (warps 0..7):  gate inputs, [Kt; Qt] and Kh, the [A; P] MMA, Kt^T      (item k+1)
+//   back  (warps 8..15): A and P out of TMEM, the triangular inverse, T into TMEM, V^T,
+//                        the W / U~ MMA with A read from TMEM, -W, U~, P into the item (item k)
+// Each buffer the groups share is handed over through an mbarrier (bounded waits).
+constexpr int kIntraThreads = 512;
+constexpr int kGroupThreads = 256;
+constexpr uint32_t kBarFront = 1, kBarBack = 2;  // named barrier ids of the two groups
 
-//  region   size    holds (in order)
-//  KQ       64 KB   [Kt; Qt] (128 x 128)  ->  [-W; Qt]
-//  KH       32 KB   Kh (64 tok x 128 ch)  ->  solve scratch
-//  KTT      32 KB   Kt^T (128 ch x 64 tok)
-//  TP       32 KB   V tile from TMA  ->  [T; P] (128 x 64)
-//  VT       32 KB   decay totals of the gate pass  ->  V^T (128 dv x 64 tok)
+//  region  size     holds
+//  KQ      64 KB    [Kt; Qt] (128 x 128); the gate pass's decay totals first     (front)
+//  KH      32 KB    Kh (64 tok x 128 ch)                                         (front)
+//  KTT     32 KB    Kt^T (128 ch x 64 tok): front writes, back's W MMA reads; then staged -W
+//  VT      32 KB    V^T (128 dv x 64 tok), then staged U~                        (back)
+//  KHT     32 KB    Kh^T staged for the bulk store into the item                 (front)
+//  SCR     25.5 KB  inverse scratch: A/X [64][kLd] + Y [32][kLd]                  (back)
 struct IntraSmem {
   static constexpr int kKQ = 0;
   static constexpr int kKH = 65536;
   static constexpr int kKTT = 98304;
-  static constexpr int kTP = 131072;
-  static constexpr int kVT = 163840;
-  static constexpr int kStage = kTP;
-  static constexpr int kScratch = kKH;
-  static constexpr int kTot = kVT;
-  static constexpr int kBeta = 196608;     // fp32 [64]
-  static constexpr int kBar = kBeta + 256; // 2 mbarriers
-  static constexpr int kTmemSlot = kBar + 16;
+  static constexpr int kVT = 131072;
+  static constexpr int kKHT = 163840;
+  static constexpr int kScr = 196608;
+  static constexpr int kTot = kKQ;                   // [16][128] fp32
+  static constexpr int kBeta = kScr + 96 * kLd * 4;  // fp32 [2][64]
+  static constexpr int kBar = kBeta + 512;
+  static constexpr int kNumBars = 8;
+  static constexpr int kTmemSlot = kBar + 8 * kNumBars;
   static constexpr int kTotal = kTmemSlot + 16;
   static constexpr int kAlloc = kTotal + 1024;
-  static_assert((64 + 32) * kLd * 4 <= 32768, "solve scratch must fit in KH");
+  static_assert(kAlloc <= 232448, "shared memory plan exceeds the per-block limit");
 };
-constexpr uint32_t kIntraD0 = 0;    // [A; P], then [W; -]  (128 columns)
-constexpr uint32_t kIntraD3 = 128;  // [U~; -]              (128 columns)
-constexpr uint32_t kIntraCols = 256;
+enum : int {
+  kBApFull = 0,  // [A; P] MMA done: back may read it, front may rewrite KQ / KH   (commit)
+  kBApFree,      // back has read [A; P] out of TMEM                                (back arrives)
+  kBVtFull,      // front has written Kt^T                                          (front arrives)
+  kBWuDone,      // W / U~ MMA done                                                 (commit)
+  kBWFree,       // back is done with KTT (W MMA read it, staged -W stored from it)  (back arrives)
+  kBDrain        // teardown after a lost wait
+};
+constexpr uint32_t kTmAP = 0;    // D [A; P]             64 columns
+constexpr uint32_t kTmT = 64;    // A operand T (rows 0..63), 64 columns
+constexpr uint32_t kTmW = 128;   // D [W; -]             128 columns
+constexpr uint32_t kTmU = 256;   // D [U~; -]            128 columns
+constexpr uint32_t kTmP = 384;   // P kept for the epilogue (rows 64..127), 64 columns
+constexpr uint32_t kIntraCols = 512;
+
+// position of one item
+struct ItemPos {
+  int64_t t0, bos;
+  int len, h;
+  uint8_t* item;
+};
+__device__ __forceinline__ ItemPos item_pos(int64_t it, const PrefillArgs& a, const SplitPlan& p) {
+  ItemPos o;
+  const int gch = static_cast<int>(it / a.H);
+  o.h = static_cast<int>(it % a.H);
+  int lo = 0, hi = a.N - 1;  // sequence: the last n with chunk_start[n] <= gch
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.chunk_start + mid) <= gch) lo = mid; else hi = mid - 1;
+  }
+  int64_t eos;
+  if (a.cu) {
+    o.bos = __ldg(a.cu + lo);
+    eos = __ldg(a.cu + lo + 1);
+  } else {
+    const int64_t L = a.total_T / a.N;
+    o.bos = static_cast<int64_t>(lo) * L;
+    eos = o.bos + L;
+  }
+  o.t0 = o.bos + static_cast<int64_t>(gch - __ldg(p.chunk_start + lo)) * kChunk;
+  o.len = static_cast<int>(eos - o.t0 < kChunk ? eos - o.t0 : kChunk);
+  o.item = p.items + static_cast<size_t>(it) * kItemBytes;
+  return o;
+}
 
 // kConv: q, k, v are the raw inputs of the full mixer; the causal depthwise conv of
 // width 4 (zero history at each sequence start) is applied to all three and the L2
 // norm x / sqrt(sum x^2 + 1e-6) to q and k, in fp32, before anything else.
 template <typename TIn, bool kConv>
 __global__ void __launch_bounds__(kIntraThreads, 1)
-    kda_intra_kernel(const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a, const SplitPlan p) {
+    kda_intra_kernel(const PrefillArgs a, const SplitPlan p) {
   using SM = IntraSmem;
   constexpr int kHist = kConv ? 3 : 0;    // tokens of history the conv needs
-  constexpr int kVRows = kChunk + kHist;  // rows of the V tile brought by TMA
-  constexpr int kGRows = 4 + kHist;       // q/k rows each thread loads in the gate pass
-  static_assert(kVRows * kD * sizeof(TIn) <= 32768, "V tile must fit in the TP region");
+  constexpr int kGRows = 4 + kHist;       // q/k rows a thread loads per 4-token group
 
-  const int gch = blockIdx.x;
-  const int h = blockIdx.y;
   const int H = a.H;
-  const int32_t* cs = p.chunk_start;
-  const int total_chunks = __ldg(cs + a.N);
-  if (total_chunks < 0 || gch >= total_chunks) return;
-  int lo = 0, hi = a.N - 1;  // sequence: the last n with cs[n] <= gch
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(cs + mid) <= gch) lo = mid; else hi = mid - 1;
-  }
-  const int n = lo;
-  int64_t bos, eos;
-  if (a.cu) {
-    bos = __ldg(a.cu + n);
-    eos = __ldg(a.cu + n + 1);
-  } else {
-    const int64_t L = a.total_T / a.N;
-    bos = static_cast<int64_t>(n) * L;
-    eos = bos + L;
-  }
-  const int64_t t0 = bos + static_cast<int64_t>(gch - __ldg(cs + n)) * kChunk;
-  const int len = static_cast<int>(eos - t0 < kChunk ? eos - t0 : kChunk);
-  uint8_t* item = p.items + (static_cast<size_t>(gch) * H + h) * kItemBytes;
+  const int total_chunks = __ldg(p.chunk_start + a.N);
+  if (total_chunks <= 0) return;  // nothing to do, or bad cu_seqlens (-1, flagged by the plan)
+  const int64_t total_items = static_cast<int64_t>(total_chunks) * H;
+  if (static_cast<int64_t>(blockIdx.x) >= total_items) return;
+  const int n_mine = static_cast<int>((total_items - 1 - blockIdx.x) / gridDim.x + 1);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
-  float* sA = reinterpret_cast<float*>(sm + SM::kScratch);  // [64][kLd]: A, then X in place
-  float* sY = sA + 64 * kLd;                                // [32][kLd]
-  float* sBeta = reinterpret_cast<float*>(sm + SM::kBeta);
+  float* sBeta = reinterpret_cast<float*>(sm + SM::kBeta);  // [2][64]
   float* sTot = reinterpret_cast<float*>(sm + SM::kTot);    // [16][128]
-  uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + SM::kBar);
-  uint64_t* bar_tma = bar_mma + 1;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmemSlot);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int lq = warp & 3;         // TMEM lane quarter this warp may access
-  const int cp = warp >> 2;        // which quarter of a row's columns this warp handles
   const int row = lq * 32 + lane;  // TMEM lane of this thread
 
   if (tid == 0) {
-    mbar_init(bar_mma, 1);
-    mbar_init(bar_tma, 1);
+    for (int i = 0; i < SM::kNumBars; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
-    tma_prefetch_desc(&tm_v);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kIntraCols);
@@ -206,308 +230,489 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = static_cast<uint32_t>(lq * 32) << 16;
-
-  // -- 1. V tile (rows t0 - kHist .. t0 + 63, all 128 columns) by TMA --------------------
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_tma, static_cast<uint32_t>(kVRows * kD * sizeof(TIn)));
-    tma_load_3d(sm + SM::kStage, &tm_v, 0, h, static_cast<int>(t0) - kHist, bar_tma);
-  }
-
-  const TIn* __restrict__ qg = static_cast<const TIn*>(a.q);
-  const TIn* __restrict__ kg = static_cast<const TIn*>(a.k);
   const int64_t tok_stride = static_cast<int64_t>(H) * kD;
 
   bool lost = false;
-  uint32_t mma_phase = 0;
-  auto wait_mma = [&]() {
-    if (!lost && !mbar_wait(bar_mma, mma_phase, a.status)) lost = true;
-    mma_phase ^= 1u;
-    tc_fence_after_sync();
-  };
 
-  // -- 2. gates. Warp w takes tokens 4w..4w+3, lane l key channels 4l..4l+3 -------------
-  {
-    const int c0 = lane * 4, r0 = warp * 4;
-    // q/k row m is chunk row r0 - kHist + m; rows outside [bos, t0 + len) read row t0
-    // (always in bounds) and are replaced by zero where used
-    uint32_t kraw[kGRows][sizeof(TIn)], qraw[kGRows][sizeof(TIn)];
-    bool rin[kGRows];
-#pragma unroll
-    for (int m = 0; m < kGRows; ++m) {
-      const int rr = r0 - kHist + m;
-      rin[m] = rr < len && t0 + rr >= bos;
-      const size_t o = static_cast<size_t>(rin[m] ? t0 + rr : t0) * tok_stride + static_cast<size_t>(h) * kD + c0;
-      if constexpr (sizeof(TIn) == 2) {
-        const uint2 kk2 = __ldg(reinterpret_cast<const uint2*>(kg + o));
-        const uint2 qq2 = __ldg(reinterpret_cast<const uint2*>(qg + o));
-        kraw[m][0] = kk2.x; kraw[m][1] = kk2.y; qraw[m][0] = qq2.x; qraw[m][1] = qq2.y;
-      } else {
-        const uint4 kk4 = __ldg(reinterpret_cast<const uint4*>(kg + o));
-        const uint4 qq4 = __ldg(reinterpret_cast<const uint4*>(qg + o));
-        kraw[m][0] = kk4.x; kraw[m][1] = kk4.y; kraw[m][2] = kk4.z; kraw[m][3] = kk4.w;
-        qraw[m][0] = qq4.x; qraw[m][1] = qq4.y; qraw[m][2] = qq4.z; qraw[m][3] = qq4.w;
+  if (warp < 8) {
+    // ================================= front group =================================
+    const int fw = warp;  // tokens 8fw .. 8fw+7: two groups of 4 (grp = 2fw + s)
+    const int ftid = tid;
+    const int c0 = lane * 4;  // key channels c0 .. c0+3
+    const TIn* __restrict__ qg = static_cast<const TIn*>(a.q);
+    const TIn* __restrict__ kg = static_cast<const TIn*>(a.k);
+    const TIn* __restrict__ vg = static_cast<const TIn*>(a.v);
+    uint32_t ph_apfull = 0, ph_apfree = 0, ph_wfree = 0;
+    auto fsync = [] { group_sync(kBarFront, kGroupThreads); };
+
+    for (int k = 0; k < n_mine; ++k) {
+      const int64_t it = blockIdx.x + static_cast<int64_t>(k) * gridDim.x;
+      const ItemPos ip = item_pos(it, a, p);
+      const int64_t t0 = ip.t0, bos = ip.bos;
+      const int len = ip.len, h = ip.h;
+      uint8_t* item = ip.item;
+      float* sB = sBeta + (k & 1) * 64;
+
+      // warm L2 with the next item's inputs (64 rows: 4 lines of log_alpha, 2 each of k, q, v)
+      if (k + 1 < n_mine) {
+        const ItemPos nx = item_pos(it + gridDim.x, a, p);
+        const int r = ftid >> 2, part = ftid & 3;
+        if (r < nx.len) {
+          const size_t o = static_cast<size_t>(nx.t0 + r) * tok_stride + static_cast<size_t>(nx.h) * kD;
+          constexpr int kLine = 128 / sizeof(TIn);  // elements per 128-B line
+          prefetch_l2(a.log_alpha + o + part * 32);
+          prefetch_l2((part < 2 ? kg : qg) + o + (part & 1) * kLine);
+          prefetch_l2(vg + o + (part & 1) * kLine + (part >> 1) * (sizeof(TIn) == 4 ? 2 * kLine : 0));
+        }
       }
-    }
-    float la[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const bool in = r0 + i < len;
-      const size_t o = static_cast<size_t>(t0 + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
-      const float4 l4 = __ldg(reinterpret_cast<const float4*>(a.log_alpha + o));
-      la[i][0] = in ? l4.x : 0.f; la[i][1] = in ? l4.y : 0.f; la[i][2] = in ? l4.z : 0.f; la[i][3] = in ? l4.w : 0.f;
-    }
-    if (tid < 64) sBeta[tid] = tid < len ? __ldg(a.beta + (t0 + tid) * H + h) : 0.f;
-    auto unpack = [&](const uint32_t* w, int e) -> float {
-      if constexpr (sizeof(TIn) == 2) {
-        const uint32_t x = w[e >> 1];
-        return __uint_as_float((e & 1) ? (x & 0xFFFF0000u) : (x << 16));
-      } else {
-        return __uint_as_float(w[e]);
+      // KQ (the totals' space) and KH are free once the previous [A; P] MMA is done. One
+      // thread waits on each mbarrier; the group follows it through a named barrier.
+      if (k > 0) {
+        if (ftid == 0 && !lost && !mbar_wait(bars + kBApFull, ph_apfull, a.status)) lost = true;
+        ph_apfull ^= 1u;
+        fsync();
       }
-    };
-    float kv[4][4], qv[4][4];
-    if constexpr (kConv) {
-      // y[t, c] = sum_j w[c, j] x[t - 3 + j, c] (x = 0 before the sequence start), then
-      // x / sqrt(sum_c y^2 + 1e-6) over the head's 128 channels (this warp holds them all)
-      float wq[4][4], wk[4][4];
+      if (ftid < 64) sB[ftid] = ftid < len ? __ldg(a.beta + (t0 + ftid) * H + h) : 0.f;
+
+      // raw q/k rows of both 4-token groups, in flight together with log_alpha (no conv:
+      // the conv's extra history rows are loaded per group below)
+      uint32_t kpre[2][4][sizeof(TIn)], qpre[2][4][sizeof(TIn)];
+      if constexpr (!kConv) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 a4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((0 * H + h) * kD + c0 + e) * 4));
-        const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((1 * H + h) * kD + c0 + e) * 4));
-        wq[e][0] = a4.x; wq[e][1] = a4.y; wq[e][2] = a4.z; wq[e][3] = a4.w;
-        wk[e][0] = b4.x; wk[e][1] = b4.y; wk[e][2] = b4.z; wk[e][3] = b4.w;
-      }
+        for (int s = 0; s < 2; ++s)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float sq = 0.f, sk = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float yq = 0.f, yk = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int m = i + j;
-            yq = fmaf(wq[e][j], rin[m] ? unpack(qraw[m], e) : 0.f, yq);
-            yk = fmaf(wk[e][j], rin[m] ? unpack(kraw[m], e) : 0.f, yk);
+          for (int i = 0; i < 4; ++i) {
+            const int rr = 4 * (2 * fw + s) + i;
+            const size_t o = static_cast<size_t>(rr < len ? t0 + rr : t0) * tok_stride + static_cast<size_t>(h) * kD + c0;
+            if constexpr (sizeof(TIn) == 2) {
+              const uint2 kk2 = __ldg(reinterpret_cast<const uint2*>(kg + o));
+              const uint2 qq2 = __ldg(reinterpret_cast<const uint2*>(qg + o));
+              kpre[s][i][0] = kk2.x; kpre[s][i][1] = kk2.y; qpre[s][i][0] = qq2.x; qpre[s][i][1] = qq2.y;
+            } else {
+              const uint4 kk4 = __ldg(reinterpret_cast<const uint4*>(kg + o));
+              const uint4 qq4 = __ldg(reinterpret_cast<const uint4*>(qg + o));
+              kpre[s][i][0] = kk4.x; kpre[s][i][1] = kk4.y; kpre[s][i][2] = kk4.z; kpre[s][i][3] = kk4.w;
+              qpre[s][i][0] = qq4.x; qpre[s][i][1] = qq4.y; qpre[s][i][2] = qq4.z; qpre[s][i][3] = qq4.w;
+            }
           }
-          qv[i][e] = yq;
-          kv[i][e] = yk;
-          sq = fmaf(yq, yq, sq);
-          sk = fmaf(yk, yk, sk);
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          sq += __shfl_xor_sync(0xffffffffu, sq, off);
-          sk += __shfl_xor_sync(0xffffffffu, sk, off);
-        }
-        const bool in = r0 + i < len;
-        const float fq = in ? rsqrtf(sq + 1e-6f) : 0.f, fk = in ? rsqrtf(sk + 1e-6f) : 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          qv[i][e] *= fq;
-          kv[i][e] *= fk;
-        }
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          kv[i][e] = rin[i] ? unpack(kraw[i], e) : 0.f;
-          qv[i][e] = rin[i] ? unpack(qraw[i], e) : 0.f;
-        }
-      }
-    }
-    // running sums within this warp's 4 tokens, then the totals of the warps before it
-    float tot[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) { tot[e] += la[i][e]; la[i][e] = tot[e]; }
-    *reinterpret_cast<float4*>(sTot + warp * kD + c0) = make_float4(tot[0], tot[1], tot[2], tot[3]);
-    __syncthreads();
-    float pre[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int w = 0; w < warp; ++w) {
-      const float4 t4 = *reinterpret_cast<const float4*>(sTot + w * kD + c0);
-      pre[0] += t4.x; pre[1] += t4.y; pre[2] += t4.z; pre[3] += t4.w;
-    }
-    if (tid < 128) {
-      float gl = 0.f;
-#pragma unroll
-      for (int w = 0; w < 16; ++w) gl += sTot[w * kD + tid];
-      if (-gl > kMaxChunkDecay) atomicOr(a.status, kFlagDecayRange);
-      reinterpret_cast<float*>(item + kItemGamma)[tid] = __expf(gl);
-    }
-    float kt[4][4], kh[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float qt[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float g = pre[e] + la[i][e];
-        const float eg = __expf(g), eng = __expf(-g);
-        kt[i][e] = kv[i][e] * eg;
-        kh[i][e] = to_tf32(kv[i][e] * eng);
-        qt[e] = qv[i][e] * eg;
-      }
-      const int r = r0 + i;
-      st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[i][0], kt[i][1], kt[i][2], kt[i][3]);  // Kt [tok][ch]
-      st4_tf32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);        // Qt [tok][ch]
-      st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);   // Kh [tok][ch]
-    }
-    // channel-major copies: Kt^T into shared memory, Kh^T straight into the item; lanes
-    // rotate e so that one store instruction touches different swizzle rows
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = (j + lane) & 3;
-      float x[4], y[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        x[i] = e == 0 ? kt[i][0] : e == 1 ? kt[i][1] : e == 2 ? kt[i][2] : kt[i][3];
-        y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
-      }
-      st4_f32(sm + SM::kKTT, f32_offset(c0 + e, r0, 128), x[0], x[1], x[2], x[3]);             // Kt^T [ch][tok]
-      *reinterpret_cast<float4*>(item + kItemKHT + f32_offset(c0 + e, r0, 128)) = make_float4(y[0], y[1], y[2], y[3]);
-    }
-  }
 
-  // -- 3. V landed: widen/transpose to V^T fp32 (rows past the sequence end -> 0) --------
-  {
-    if (!lost && !mbar_wait(bar_tma, 0, a.status)) lost = true;
-    __syncthreads();  // every thread is done with the decay totals (they share V^T's space)
-    const TIn* st = reinterpret_cast<const TIn*>(sm + SM::kStage);  // row m = token t0 - kHist + m
-    for (int i = tid; i < kD * 16; i += kIntraThreads) {
-      const int j = i % kD, t4 = (i / kD) * 4;
-      float x[4];
-      if constexpr (kConv) {
-        const float4 w4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((2 * H + h) * kD + j) * 4));
-        const float w[4] = {w4.x, w4.y, w4.z, w4.w};
-        float xs[7];
+      // -- gate pass A: running sums of log_alpha inside each 4-token group -------------
+      float la[2][4][4], tot[2][4];
 #pragma unroll
-        for (int m = 0; m < 7; ++m) xs[m] = (t0 - kHist + t4 + m >= bos) ? as_f32(st[(t4 + m) * kD + j]) : 0.f;
+      for (int s = 0; s < 2; ++s) {
+        const int r0 = 4 * (2 * fw + s);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const bool in = r0 + i < len;
+          const size_t o = static_cast<size_t>(t0 + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
+          const float4 l4 = __ldg(reinterpret_cast<const float4*>(a.log_alpha + o));
+          la[s][i][0] = in ? l4.x : 0.f; la[s][i][1] = in ? l4.y : 0.f;
+          la[s][i][2] = in ? l4.z : 0.f; la[s][i][3] = in ? l4.w : 0.f;
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          float y = 0.f;
+          tot[s][e] = 0.f;
 #pragma unroll
-          for (int tap = 0; tap < 4; ++tap) y = fmaf(w[tap], xs[e + tap], y);
-          x[e] = (t4 + e < len) ? y : 0.f;
+          for (int i = 0; i < 4; ++i) { tot[s][e] += la[s][i][e]; la[s][i][e] = tot[s][e]; }
+        }
+        *reinterpret_cast<float4*>(sTot + (2 * fw + s) * kD + c0) = make_float4(tot[s][0], tot[s][1], tot[s][2], tot[s][3]);
+      }
+      fsync();
+      float pre[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int g = 0; g < 2 * fw; ++g) {
+        const float4 t4 = *reinterpret_cast<const float4*>(sTot + g * kD + c0);
+        pre[0][0] += t4.x; pre[0][1] += t4.y; pre[0][2] += t4.z; pre[0][3] += t4.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pre[1][e] = pre[0][e] + tot[0][e];
+      if (ftid < 128) {
+        float gl = 0.f;
+#pragma unroll
+        for (int g = 0; g < 16; ++g) gl += sTot[g * kD + ftid];
+        if (-gl > kMaxChunkDecay) atomicOr(a.status, kFlagDecayRange);
+        reinterpret_cast<float*>(item + kItemGamma)[ftid] = __expf(gl);
+      }
+      if (ftid == 0) bulk_wait_read();  // the previous item's Qt and Kh^T have left KQ and KHT
+      fsync();  // the totals are read: KQ may be written
+
+      // -- gate pass B: q, k (conv, L2 norm), Kt, Qt, Kh -----------------------------------
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int r0 = 4 * (2 * fw + s);
+        // q/k row m is chunk row r0 - kHist + m; rows outside [bos, t0 + len) read row t0
+        // (always in bounds) and are replaced by zero where used
+        uint32_t kraw[kGRows][sizeof(TIn)], qraw[kGRows][sizeof(TIn)];
+        bool rin[kGRows];
+#pragma unroll
+        for (int m = 0; m < kGRows; ++m) {
+          const int rr = r0 - kHist + m;
+          rin[m] = rr < len && t0 + rr >= bos;
+          if constexpr (!kConv) {
+#pragma unroll
+            for (int w = 0; w < static_cast<int>(sizeof(TIn)); ++w) {
+              kraw[m][w] = kpre[s][m][w];
+              qraw[m][w] = qpre[s][m][w];
+            }
+            continue;
+          }
+          const size_t o = static_cast<size_t>(rin[m] ? t0 + rr : t0) * tok_stride + static_cast<size_t>(h) * kD + c0;
+          if constexpr (sizeof(TIn) == 2) {
+            const uint2 kk2 = __ldg(reinterpret_cast<const uint2*>(kg + o));
+            const uint2 qq2 = __ldg(reinterpret_cast<const uint2*>(qg + o));
+            kraw[m][0] = kk2.x; kraw[m][1] = kk2.y; qraw[m][0] = qq2.x; qraw[m][1] = qq2.y;
+          } else {
+            const uint4 kk4 = __ldg(reinterpret_cast<const uint4*>(kg + o));
+            const uint4 qq4 = __ldg(reinterpret_cast<const uint4*>(qg + o));
+            kraw[m][0] = kk4.x; kraw[m][1] = kk4.y; kraw[m][2] = kk4.z; kraw[m][3] = kk4.w;
+            qraw[m][0] = qq4.x; qraw[m][1] = qq4.y; qraw[m][2] = qq4.z; qraw[m][3] = qq4.w;
+          }
+        }
+        auto unpack = [&](const uint32_t* w, int e) -> float {
+          if constexpr (sizeof(TIn) == 2) {
+            const uint32_t x = w[e >> 1];
+            return __uint_as_float((e & 1) ? (x & 0xFFFF0000u) : (x << 16));
+          } else {
+            return __uint_as_float(w[e]);
+          }
+        };
+        float kv[4][4], qv[4][4];
+        if constexpr (kConv) {
+          // y[t, c] = sum_j w[c, j] x[t - 3 + j, c] (x = 0 before the sequence start), then
+          // x / sqrt(sum_c y^2 + 1e-6) over the head's 128 channels (this warp holds them all)
+          float wq[4][4], wk[4][4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float4 a4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((0 * H + h) * kD + c0 + e) * 4));
+            const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((1 * H + h) * kD + c0 + e) * 4));
+            wq[e][0] = a4.x; wq[e][1] = a4.y; wq[e][2] = a4.z; wq[e][3] = a4.w;
+            wk[e][0] = b4.x; wk[e][1] = b4.y; wk[e][2] = b4.z; wk[e][3] = b4.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float sq = 0.f, sk = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float yq = 0.f, yk = 0.f;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int m = i + j;
+                yq = fmaf(wq[e][j], rin[m] ? unpack(qraw[m], e) : 0.f, yq);
+                yk = fmaf(wk[e][j], rin[m] ? unpack(kraw[m], e) : 0.f, yk);
+              }
+              qv[i][e] = yq;
+              kv[i][e] = yk;
+              sq = fmaf(yq, yq, sq);
+              sk = fmaf(yk, yk, sk);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+              sq += __shfl_xor_sync(0xffffffffu, sq, off);
+              sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            }
+            const bool in = r0 + i < len;
+            const float fq = in ? rsqrtf(sq + 1e-6f) : 0.f, fk = in ? rsqrtf(sk + 1e-6f) : 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              qv[i][e] *= fq;
+              kv[i][e] *= fk;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              kv[i][e] = rin[i] ? unpack(kraw[i], e) : 0.f;
+              qv[i][e] = rin[i] ? unpack(qraw[i], e) : 0.f;
+            }
+        }
+        float kh[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float kt[4], qt[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float g = pre[s][e] + la[s][i][e];
+            const float eg = __expf(g), eng = __expf(-g);
+            kt[e] = kv[i][e] * eg;
+            kh[i][e] = to_tf32(kv[i][e] * eng);
+            qt[e] = to_tf32(qv[i][e] * eg);
+          }
+          const int r = r0 + i;
+          st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[0], kt[1], kt[2], kt[3]);          // Kt [tok][ch]
+          st4_f32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);     // Qt [tok][ch]
+          st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);  // Kh [tok][ch]
+        }
+        // Kh^T (staged for the item): channel c0+e, tokens r0..r0+3
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = (j + lane) & 3;
+          float y[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
+          st4_f32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      fsync();
+      if (ftid == 0) {  // Qt: rows 64..127 of each 32-column block of the tile; Kh^T whole
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb)
+          bulk_store(item + kItemQW + kb * 16384 + 8192, sm + SM::kKQ + kb * 16384 + 8192, 8192);
+        bulk_store(item + kItemKHT, sm + SM::kKHT, 32768);
+        bulk_commit_group();
+      }
+
+      // -- D[A; P] = [Kt; Qt] Kh^T, once the back group has read the previous one out ------
+      if (ftid == 0) {
+        if (k > 0) {
+          if (!lost && !mbar_wait(bars + kBApFree, ph_apfree, a.status)) lost = true;
+          ph_apfree ^= 1u;
+        }
+        tc_fence_after_sync();
+        constexpr uint32_t kIdAP = idesc_tf32(128, 64, false, false);
+        const uint64_t a0 = kdesc0(sb + SM::kKQ), b0 = kdesc0(sb + SM::kKH);
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk)
+          umma_tf32(tmem + kTmAP, a0 + kstep(kk, 128), b0 + kstep(kk, 64), kIdAP, kk > 0);
+        umma_commit(bars + kBApFull);
+      }
+
+      // -- Kt^T, once the back group's previous W / U~ MMA and its staging have let go of KTT --
+      if (k > 0) {
+        if (ftid == 0 && !lost && !mbar_wait(bars + kBWFree, ph_wfree, a.status)) lost = true;
+        ph_wfree ^= 1u;
+        fsync();
+      }
+      for (int i = ftid; i < kD * 16; i += kGroupThreads) {  // Kt (rows 0..63 of KQ) -> Kt^T
+        const int c = i % kD, r4 = (i / kD) * 4;
+        const float* kq = reinterpret_cast<const float*>(sm + SM::kKQ);
+        st4_f32(sm + SM::kKTT, f32_offset(c, r4, 128), kq[f32_offset(r4, c, 128) >> 2],
+                kq[f32_offset(r4 + 1, c, 128) >> 2], kq[f32_offset(r4 + 2, c, 128) >> 2],
+                kq[f32_offset(r4 + 3, c, 128) >> 2]);
+      }
+      fence_proxy_async_smem();
+      fsync();
+      if (ftid == 0) mbar_arrive(bars + kBVtFull);
+      if (group_any(kBarFront, kGroupThreads, lost)) {
+        lost = true;
+        break;
+      }
+    }
+  } else {
+    // ================================= back group ==================================
+    const int bw = warp - 8;
+    const int btid = tid - kGroupThreads;
+    const int half = bw >> 2;  // which half of a row's columns this warp handles
+    float* sA = reinterpret_cast<float*>(sm + SM::kScr);  // [64][kLd]: A, then X in place
+    float* sY = sA + 64 * kLd;                            // [32][kLd]
+    uint32_t ph_apfull = 0, ph_vtfull = 0, ph_wu = 0;
+    auto bsync = [] { group_sync(kBarBack, kGroupThreads); };
+    constexpr uint32_t kIdN128 = idesc_tf32(128, 128, false, false);
+
+    const TIn* __restrict__ vg = static_cast<const TIn*>(a.v);
+    for (int k = 0; k < n_mine; ++k) {
+      const int64_t it = blockIdx.x + static_cast<int64_t>(k) * gridDim.x;
+      const ItemPos ip = item_pos(it, a, p);
+      uint8_t* item = ip.item;
+      const float* sB = sBeta + (k & 1) * 64;
+
+      // -- A (rows 0..63: beta-scaled, strictly lower) -> scratch; P (rows 64..127: lower) -> item
+      if (btid == 0 && !lost && !mbar_wait(bars + kBApFull, ph_apfull, a.status)) lost = true;
+      ph_apfull ^= 1u;
+      bsync();
+      tc_fence_after_sync();
+      {
+        const int cb = half * 32;
+        float d[32];
+        tmem_ld16(tmem + lane_off + kTmAP + cb, *reinterpret_cast<float(*)[16]>(d));
+        tmem_ld16(tmem + lane_off + kTmAP + cb + 16, *reinterpret_cast<float(*)[16]>(d + 16));
+        tmem_ld_wait();
+        if (lq < 2) {
+          const int r = row;
+          const float br = sB[r];
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const int c = cb + i;
+            *reinterpret_cast<float4*>(sA + r * kLd + c) =
+                make_float4(c < r ? br * d[i] : 0.f, c + 1 < r ? br * d[i + 1] : 0.f,
+                            c + 2 < r ? br * d[i + 2] : 0.f, c + 3 < r ? br * d[i + 3] : 0.f);
+          }
+        } else {  // P row r (lower, tf32) kept in TMEM until the epilogue stages it
+          const int r = row - 64;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = (cb + i + e <= r) ? to_tf32(d[i + e]) : 0.f;
+            tmem_st8(tmem + lane_off + kTmP + cb + i, x);
+          }
+          tmem_st_wait();
+        }
+      }
+      tc_fence_before_sync();
+      bsync();
+      if (btid == 0) mbar_arrive(bars + kBApFree);
+
+      // -- X = (I + A)^-1; T = X Diag(beta) into TMEM rows 0..63 (the W / U~ MMA's A) ---------
+      invert_unit_lower_64(sA, sY, bw, bsync);
+      if (lq < 2) {
+        const int r = row;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          const int c = half * 32 + j;
+          float x[8];
+          const float4 x0 = *reinterpret_cast<const float4*>(sA + r * kLd + c);
+          const float4 x1 = *reinterpret_cast<const float4*>(sA + r * kLd + c + 4);
+          const float xr[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = (c + e <= r) ? to_tf32(xr[e] * sB[c + e]) : 0.f;
+          tmem_st8(tmem + lane_off + kTmT + c, x);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before_sync();
+      bsync();
+
+      // -- V^T (tf32; conv for the mixer): each thread takes 4-token x 4-column blocks, all
+      //    of whose rows are loaded before any is used (the rows were warmed into L2) ----------
+      {
+        constexpr int kW = sizeof(TIn);  // 32-bit words per 4 elements
+        const TIn* vh = vg + static_cast<size_t>(ip.h) * kD;
+        uint32_t vraw[2][kGRows][kW];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+#pragma unroll
+          for (int m = 0; m < kGRows; ++m) {
+            const int rr = t4 - kHist + m;
+            const bool in = rr < ip.len && ip.t0 + rr >= ip.bos;
+            const TIn* src = vh + static_cast<size_t>(in ? ip.t0 + rr : ip.t0) * tok_stride + j4;
+            if constexpr (kW == 2) {
+              const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
+              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
+            } else {
+              const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
+              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
+              vraw[bb][m][2] = in ? x.z : 0u; vraw[bb][m][3] = in ? x.w : 0u;
+            }
+          }
+        }
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const int jr = (jj + lane) & 3;  // lanes rotate the column so a store spreads over swizzle rows
+            auto elem = [&](int m) -> float {  // selects, not indexing: the array stays in registers
+              if constexpr (kW == 2) {
+                const uint32_t x = (jr >> 1) ? vraw[bb][m][1] : vraw[bb][m][0];
+                return __uint_as_float((jr & 1) ? (x & 0xFFFF0000u) : (x << 16));
+              } else {
+                const uint32_t lo = (jr & 1) ? vraw[bb][m][1] : vraw[bb][m][0];
+                const uint32_t hi = (jr & 1) ? vraw[bb][m][3] : vraw[bb][m][2];
+                return __uint_as_float((jr >> 1) ? hi : lo);
+              }
+            };
+            float x[4];
+            if constexpr (kConv) {
+              const float4 w4 =
+                  __ldg(reinterpret_cast<const float4*>(a.conv_w + ((2 * H + ip.h) * kD + j4 + jr) * 4));
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float y = fmaf(w4.x, elem(e), fmaf(w4.y, elem(e + 1), fmaf(w4.z, elem(e + 2), w4.w * elem(e + 3))));
+                x[e] = (t4 + e < ip.len) ? y : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) x[e] = elem(e);
+            }
+            st4_tf32(sm + SM::kVT, f32_offset(j4 + jr, t4, 128), x[0], x[1], x[2], x[3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      bsync();
+
+      // -- D[W; -] = T Kt, D[U~; -] = T V, once the front group has written Kt^T ------------
+      if (btid == 0) {
+        if (!lost && !mbar_wait(bars + kBVtFull, ph_vtfull, a.status)) lost = true;
+        ph_vtfull ^= 1u;
+        tc_fence_after_sync();
+        const uint64_t kt0 = kdesc0(sb + SM::kKTT), v0 = kdesc0(sb + SM::kVT);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_tf32_ta(tmem + kTmW, tmem + kTmT + kk * 8, kt0 + kstep(kk, 128), kIdN128, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_tf32_ta(tmem + kTmU, tmem + kTmT + kk * 8, v0 + kstep(kk, 128), kIdN128, kk > 0);
+        umma_commit(bars + kBWuDone);
+      }
+      if (btid == 0 && !lost && !mbar_wait(bars + kBWuDone, ph_wu, a.status)) lost = true;
+      ph_wu ^= 1u;
+      bsync();
+      tc_fence_after_sync();
+
+      // -- -W, U~ (over Kt^T and V^T, which the MMA has read) and P (over the scratch) staged
+      //    as 64-row tiles, then bulk-stored into the item --------------------------------------
+      if (lq < 2) {
+        const int r = row;
+#pragma unroll
+        for (int j = 0; j < 64; j += 16) {
+          const int c = half * 64 + j;
+          float w[16], u[16];
+          tmem_ld16(tmem + lane_off + kTmW + c, w);
+          tmem_ld16(tmem + lane_off + kTmU + c, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            st4_f32(sm + SM::kKTT, f32_offset(r, c + e, 64), -w[e], -w[e + 1], -w[e + 2], -w[e + 3]);
+            st4_f32(sm + SM::kVT, f32_offset(r, c + e, 64), u[e], u[e + 1], u[e + 2], u[e + 3]);
+          }
         }
       } else {
+        const int r = row - 64;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = (t4 + e < len) ? as_f32(st[(t4 + e) * kD + j]) : 0.f;
+        for (int j = 0; j < 32; j += 16) {
+          const int c = half * 32 + j;
+          float x[16];
+          tmem_ld16(tmem + lane_off + kTmP + c, x);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            st4_f32(sm + SM::kScr, f32_offset(r, c + e, 64), x[e], x[e + 1], x[e + 2], x[e + 3]);
+        }
       }
-      st4_tf32(sm + SM::kVT, f32_offset(j, t4, 128), x[0], x[1], x[2], x[3]);
-    }
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-
-  constexpr uint32_t kIdAP = idesc_tf32(128, 64, false, false);
-  constexpr uint32_t kIdN128 = idesc_tf32(128, 128, false, false);
-
-  // -- 4. D0 = [A_raw; P_raw] = [Kt; Qt] Kh^T ------------------------------------------------
-  if (tid == 0) {
-    tc_fence_after_sync();
-    const uint64_t a0 = kdesc0(sb + SM::kKQ), b0 = kdesc0(sb + SM::kKH);
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      bsync();
+      if (btid == 0) {
 #pragma unroll
-    for (int kk = 0; kk < 16; ++kk)
-      umma_tf32(tmem + kIntraD0, a0 + kstep(kk, 128), b0 + kstep(kk, 64), kIdAP, kk > 0);
-    umma_commit(bar_mma);
-  }
-  wait_mma();
-
-  // -- 5. A (rows 0..63: beta-scaled, strictly lower) -> solve scratch, P (rows 64..127:
-  //       lower) -> rows 64..127 of the TP tile -----------------------------------------------
-  {
-    const int cb = cp * 16;
-    float d[16];
-    tmem_ld16(tmem + lane_off + kIntraD0 + cb, d);
-    tmem_ld_wait();
-    if (lq < 2) {
-      const int r = row;
-      const float br = sBeta[r];
-#pragma unroll
-      for (int i = 0; i < 16; i += 4) {
-        const int c = cb + i;
-        *reinterpret_cast<float4*>(sA + r * kLd + c) =
-            make_float4(c < r ? br * d[i] : 0.f, c + 1 < r ? br * d[i + 1] : 0.f, c + 2 < r ? br * d[i + 2] : 0.f,
-                        c + 3 < r ? br * d[i + 3] : 0.f);
+        for (int kb = 0; kb < 4; ++kb)  // -W: rows 0..63 of each 32-column block of the tile
+          bulk_store(item + kItemQW + kb * 16384, sm + SM::kKTT + kb * 8192, 8192);
+        bulk_store(item + kItemU, sm + SM::kVT, 32768);
+        bulk_store(item + kItemP, sm + SM::kScr, 16384);
+        bulk_commit_group();
+        bulk_wait_read();  // Kt^T, V^T and the scratch are free again
+        mbar_arrive(bars + kBWFree);
       }
-    } else {
-      const int r = row - 64;
-#pragma unroll
-      for (int i = 0; i < 16; i += 4) {
-        const int c = cb + i;
-        st4_tf32(sm + SM::kTP, f32_offset(64 + r, c, 128), c <= r ? d[i] : 0.f, c + 1 <= r ? d[i + 1] : 0.f,
-                 c + 2 <= r ? d[i + 2] : 0.f, c + 3 <= r ? d[i + 3] : 0.f);
+      if (group_any(kBarBack, kGroupThreads, lost)) {
+        lost = true;
+        break;
       }
     }
+  }
+
+  // ---- teardown: bulk stores complete; after a lost wait, let the tensor pipe drain
+  //      (bounded) before the TMEM goes back ----------------------------------------------
+  if (tid == 0 || tid == kGroupThreads) bulk_wait_all();  // the items' bulk stores are done
+  const bool any_lost = __syncthreads_or(lost ? 1 : 0) != 0;
+  if (any_lost && tid == 0) {
+    umma_commit(bars + kBDrain);
+    mbar_wait(bars + kBDrain, 0, a.status);
   }
   tc_fence_before_sync();
-  __syncthreads();
-
-  // -- 6. X = (I + A)^-1 in fp32 (in place over A), T = X Diag(beta) -> rows 0..63 of TP ---
-  invert_unit_lower_64(sA, sY);
-  {
-    const int r = tid & 63, c = (tid >> 6) * 8;
-#pragma unroll
-    for (int i = c; i < c + 8; i += 4) {
-      const float4 xr = *reinterpret_cast<const float4*>(sA + r * kLd + i);
-      st4_tf32(sm + SM::kTP, f32_offset(r, i, 128), i <= r ? xr.x * sBeta[i] : 0.f,
-               i + 1 <= r ? xr.y * sBeta[i + 1] : 0.f, i + 2 <= r ? xr.z * sBeta[i + 2] : 0.f,
-               i + 3 <= r ? xr.w * sBeta[i + 3] : 0.f);
-    }
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-
-  // -- 7. D0 = [W; -] = [T; P] Kt,  D3 = [U~; -] = [T; P] V;  P rows -> item --------------------
-  if (tid == 0) {
-    tc_fence_after_sync();
-    const uint64_t a0 = kdesc0(sb + SM::kTP), b0 = kdesc0(sb + SM::kKTT), v0 = kdesc0(sb + SM::kVT);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      umma_tf32(tmem + kIntraD0, a0 + kstep(kk, 128), b0 + kstep(kk, 128), kIdN128, kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      umma_tf32(tmem + kIntraD3, a0 + kstep(kk, 128), v0 + kstep(kk, 128), kIdN128, kk > 0);
-    umma_commit(bar_mma);
-    bulk_store(item + kItemP, sm + SM::kTP + 8192, 8192);
-    bulk_store(item + kItemP + 8192, sm + SM::kTP + 16384 + 8192, 8192);
-    bulk_commit_group();
-  }
-  wait_mma();
-
-  // -- 8. -W -> rows 0..63 of KQ (over Kt), U~ -> item ----------------------------------------
-  if (lq < 2) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int cb = cp * 32 + 16 * j;
-      float w[16], u[16];
-      tmem_ld16(tmem + lane_off + kIntraD0 + cb, w);
-      tmem_ld16(tmem + lane_off + kIntraD3 + cb, u);
-      tmem_ld_wait();
-#pragma unroll
-      for (int e = 0; e < 16; e += 4)
-        st4_f32(sm + SM::kKQ, f32_offset(row, cb + e, 128), -w[e], -w[e + 1], -w[e + 2], -w[e + 3]);
-      float4* ug = reinterpret_cast<float4*>(item + kItemU + static_cast<size_t>(row) * (kD * 4) + cb * 4);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ug[e] = make_float4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before_sync();
-  __syncthreads();
-
-  // -- 9. [-W; Qt] -> item; every bulk store done before the shared memory goes away -----------
-  if (tid == 0) {
-    bulk_store(item + kItemQW, sm + SM::kKQ, 65536);
-    bulk_commit_group();
-    bulk_wait_all();
-    if (lost) {  // let the tensor pipe drain (bounded) before the TMEM goes back
-      umma_commit(bar_mma);
-      mbar_wait(bar_mma, mma_phase, a.status);
-    }
-  }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after_sync();
@@ -647,11 +852,10 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
   // U~ of the next chunk for this thread (rows 0..63: row, columns col0 + cp*kPart ..)
   float ut[kPart];
   auto load_ut = [&](int c) {
-    const float4* src = reinterpret_cast<const float4*>(item_of(c) + kItemU + static_cast<size_t>(row) * (kD * 4) +
-                                                        (col0 + cp * kPart) * 4);
+    const uint8_t* src = item_of(c) + kItemU;
 #pragma unroll
     for (int e = 0; e < kPart / 4; ++e) {
-      const float4 x = __ldg(src + e);
+      const float4 x = __ldg(reinterpret_cast<const float4*>(src + f32_offset(row, col0 + cp * kPart + 4 * e, 64)));
       ut[4 * e] = x.x; ut[4 * e + 1] = x.y; ut[4 * e + 2] = x.z; ut[4 * e + 3] = x.w;
     }
   };
@@ -818,9 +1022,6 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
 // ================================ host =================================================
 template <typename TIn, bool kConv>
 cudaError_t launch_intra(const PrefillArgs& a, const SplitPlan& p, int64_t max_chunks, cudaStream_t stream) {
-  CUtensorMap tm;
-  if (!encode_value_map(&tm, a.v, a.total_T, a.H, kD, kChunk + (kConv ? 3 : 0), sizeof(TIn) == 4))
-    return cudaErrorInvalidValue;
   auto kern = kda_intra_kernel<TIn, kConv>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -828,8 +1029,14 @@ cudaError_t launch_intra(const PrefillArgs& a, const SplitPlan& p, int64_t max_c
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, IntraSmem::kAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  const dim3 grid(static_cast<unsigned>(max_chunks), static_cast<unsigned>(a.H));
-  kern<<<grid, kIntraThreads, IntraSmem::kAlloc, stream>>>(tm, a, p);
+  // persistent: one CTA per SM (the shared memory plan allows no more), each walking items
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int64_t items = max_chunks * a.H;
+  const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
+  kern<<<grid, kIntraThreads, IntraSmem::kAlloc, stream>>>(a, p);
   return cudaGetLastError();
 }
 

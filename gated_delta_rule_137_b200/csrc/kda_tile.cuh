@@ -132,15 +132,17 @@ __device__ __forceinline__ void warp_gemm_16x8(const float* A, const float* B, i
 
 // ---- X = (I + A)^-1 for a strictly lower 64x64 A in fp32 ----------------------------
 // sA: A in [64][kLd] on entry, X in place on return; sY: [32][kLd] scratch. Called by
-// every thread of a CTA of at least 256 threads (warps 0..7 work; all take the barriers).
+// every thread of a group of at least 8 warps; `gw` is the caller's warp index within
+// the group and `sync()` a barrier over the group (warps 0..7 work; all take it).
 // 16x16 diagonal blocks by forward substitution in registers, then two levels of block
 // doubling: [[X1, 0], [A21, X2]]^-1 has lower-left block -X2 (A21 X1).
-__device__ __forceinline__ void invert_unit_lower_64(float* sA, float* sY) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+template <typename Sync>
+__device__ __forceinline__ void invert_unit_lower_64(float* sA, float* sY, int gw, Sync sync) {
+  const int lane = threadIdx.x & 31;
   // warp b < 4 owns diagonal block b; lane (r = lane % 16, half hh) holds row r,
   // columns 8hh..8hh+7
-  if (warp < 4) {
-    const int b = warp, r = lane & 15, hh = lane >> 4;
+  if (gw < 4) {
+    const int b = gw, r = lane & 15, hh = lane >> 4;
     float* Arow = sA + (16 * b + r) * kLd + 16 * b;
     float av[16], x[8];
 #pragma unroll
@@ -157,29 +159,33 @@ __device__ __forceinline__ void invert_unit_lower_64(float* sA, float* sY) {
     *reinterpret_cast<float4*>(Arow + 8 * hh) = make_float4(x[0], x[1], x[2], x[3]);
     *reinterpret_cast<float4*>(Arow + 8 * hh + 4) = make_float4(x[4], x[5], x[6], x[7]);
   }
-  __syncthreads();
+  sync();
   // 16 -> 32 on the two diagonal pairs (warp = pair * 2 + 8-column tile) ...
-  if (warp < 4) {
-    const int p = warp >> 1, nt = warp & 1, o = 32 * p;
+  if (gw < 4) {
+    const int p = gw >> 1, nt = gw & 1, o = 32 * p;
     warp_gemm_16x8(sA + (o + 16) * kLd + o, sA + o * kLd + o + 8 * nt, 16, sY + 16 * p + 8 * nt, 1.f);
   }
-  __syncthreads();
-  if (warp < 4) {
-    const int p = warp >> 1, nt = warp & 1, o = 32 * p;
+  sync();
+  if (gw < 4) {
+    const int p = gw >> 1, nt = gw & 1, o = 32 * p;
     warp_gemm_16x8(sA + (o + 16) * kLd + o + 16, sY + 16 * p + 8 * nt, 16, sA + (o + 16) * kLd + o + 8 * nt, -1.f);
   }
-  __syncthreads();
+  sync();
   // ... then 32 -> 64 (warp = 16-row tile * 4 + 8-column tile)
-  if (warp < 8) {
-    const int mt = warp >> 2, nt = warp & 3;
+  if (gw < 8) {
+    const int mt = gw >> 2, nt = gw & 3;
     warp_gemm_16x8(sA + (32 + 16 * mt) * kLd, sA + 8 * nt, 32, sY + (16 * mt) * kLd + 8 * nt, 1.f);
   }
-  __syncthreads();
-  if (warp < 8) {
-    const int mt = warp >> 2, nt = warp & 3;
+  sync();
+  if (gw < 8) {
+    const int mt = gw >> 2, nt = gw & 3;
     warp_gemm_16x8(sA + (32 + 16 * mt) * kLd + 32, sY + 8 * nt, 32, sA + (32 + 16 * mt) * kLd + 8 * nt, -1.f);
   }
-  __syncthreads();
+  sync();
+}
+// Whole-CTA form (threadIdx.x / 32 is the warp index, __syncthreads the barrier).
+__device__ __forceinline__ void invert_unit_lower_64(float* sA, float* sY) {
+  invert_unit_lower_64(sA, sY, static_cast<int>(threadIdx.x >> 5), [] { __syncthreads(); });
 }
 
 // ---- TMA descriptor encoding through the driver entry point ----------------------------

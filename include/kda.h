@@ -94,8 +94,9 @@ KDA_API const char* kda_version(void);
  * Beyond the status word (and, for head dims below 128, zero-padded copies of
  * the inputs), the workspace holds the scratch of the two-pass prefill: about
  * 145 KB per (64-token chunk, head), e.g. 303 MB for one 4096-token sequence of
- * 32 heads. When that scratch would exceed 32 GiB the call runs a single-pass
- * kernel instead (slower, no scratch) and the query leaves it out.
+ * 32 heads. The two-pass form is used for at most 74 (sequence, head) pairs
+ * (N * H <= 74) and at most 32 GiB of scratch; otherwise the call runs a
+ * single-pass kernel that needs no scratch and the query leaves it out.
  */
 KDA_API size_t kda_chunk_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv, kda_dtype qkv_dtype);
 

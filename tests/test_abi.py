@@ -56,9 +56,12 @@ def test_workspace_query(lib):
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 0, 16, kda.KDA_DT_F32) == 0
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 129, 16, kda.KDA_DT_BF16) == 0
     assert lib.kda_chunk_fwd_workspace(64, 1, 2, 16, 16, 7) == 0
-    # beyond 32 GiB of scratch the single-pass kernel runs and the query drops the scratch
+    # beyond 32 GiB of scratch, or beyond 74 (sequence, head) chains, the single-pass kernel
+    # runs and the query drops the scratch
     huge_T = (1 << 31) - 1024
     assert lib.kda_chunk_fwd_workspace(huge_T, 1, 32, 128, 128, kda.KDA_DT_BF16) == 256
+    assert lib.kda_chunk_fwd_workspace(4096, 3, 25, 128, 128, kda.KDA_DT_BF16) == 256  # 75 chains
+    assert lib.kda_chunk_fwd_workspace(4096, 2, 37, 128, 128, kda.KDA_DT_BF16) > 256   # 74 chains
     assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 128, 128) == 256 + 256 + (1000 // 64 + 2) * 32 * item
     assert lib.kda_mixer_fwd_workspace(1000, 2, 32, 64, 64) == 0
 
