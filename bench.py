@@ -38,9 +38,11 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # ----------------------------------------------------------------------------------
 # algorithmic work (bytes / flops the method must move or do, per call)
 # ----------------------------------------------------------------------------------
-# kernels one kda_chunk_fwd / kda_mixer_fwd call launches: the chunk plan, the
-# intra-chunk pass over all chunks, the recurrence over each chain's chunks
-PREFILL_KERNELS = 3
+def kernels_per_call(workspace_bytes: int) -> int:
+    """Kernels one kda_chunk_fwd / kda_mixer_fwd call launches (d = 128): the chunk plan,
+    the intra-chunk pass and the recurrence when the workspace query asked for the
+    two-pass scratch (more than the 256-byte status word), else the single-pass kernel."""
+    return 3 if workspace_bytes > 256 else 1
 
 
 def prefill_bytes(total_T: int, N: int, Hh: int = H, d: int = D, with_h0: bool = True, mixer: bool = False) -> int:
@@ -71,6 +73,32 @@ def load_peaks():
         j = json.load(open(p))
         return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_sources_sha256() -> str:
+    """Hash of the CUDA sources (csrc/*.cu, *.cuh, *.h, sorted by name): identifies the
+    kernels an ncu traffic figure was captured from."""
+    import hashlib
+    csrc = os.path.join(ROOT, "gated_delta_rule_137_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()
+
+
+def load_traffic(override=None):
+    """DRAM bytes per headline call (read + write of the plan, intra-chunk and recurrence
+    kernels) from profiles/traffic.json, if it was captured from these kernel sources;
+    None once the sources have changed since."""
+    if override is not None:
+        return override
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p))
+    return float(j["bytes_per_call"]) if j.get("source_sha256") == kernel_sources_sha256() else None
 
 
 # ----------------------------------------------------------------------------------
@@ -251,6 +279,7 @@ def run_gpu(args):
     outs = [torch.empty(T1, H, D, dtype=torch.bfloat16, device=device) for _ in range(n_sets)]
     fins = [torch.empty(1, H, D, D, dtype=torch.float32, device=device) for _ in range(n_sets)]
     ws_bytes = kda.chunk_fwd_workspace_bytes(T1, 1, H, D, D, kda.KDA_DT_BF16)
+    head_kernels = kernels_per_call(ws_bytes)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
 
     def step(i):
@@ -260,7 +289,7 @@ def run_gpu(args):
 
     with ClockSampler(device.index) as clk:
         per, total_ms = time_region(step, args.steps, args.warmup, stream, device)
-    launches += PREFILL_KERNELS * args.steps
+    launches += head_kernels * args.steps
     kda.workspace_status(ws)
     clocks = clk.summary()
     total_ms_max = max_over_ranks(total_ms, device)
@@ -341,7 +370,7 @@ def run_gpu(args):
 
         msteps = max(3, min(args.steps, 10))
         mper, mtot = time_region(mstep, msteps, 2, stream, device)
-        launches += PREFILL_KERNELS * msteps
+        launches += kernels_per_call(mws.numel()) * msteps
         mtot = max_over_ranks(mtot, device)
         mbytes = prefill_bytes(Bm * Tm, Bm, with_h0=False, mixer=True)
         mms = statistics.mean(mper)
@@ -370,7 +399,7 @@ def run_gpu(args):
 
         vsteps = max(3, min(args.steps, 10))
         vper, vtot = time_region(vstep, vsteps, 2, stream, device)
-        launches += PREFILL_KERNELS * vsteps
+        launches += kernels_per_call(vws.numel()) * vsteps
         vtot = max_over_ranks(vtot, device)
         vbytes = prefill_bytes(TT, len(lens))
         vms = statistics.mean(vper)
@@ -393,7 +422,7 @@ def run_gpu(args):
                        "parallelism": f"replicas x{world} (independent (sequence, head) chains, no collective)",
                        "l2": f"inputs rotate through {n_sets} device copies ({n_sets * bytes_call / 1e6:.0f} MB > L2)"},
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved_gbs / hbm_peak, "traffic": args.traffic,
+                         "frac": achieved_gbs / hbm_peak, "traffic": load_traffic(args.traffic),
                          "kernel": "kda_chunk_fwd (plan + intra-chunk + recurrence kernels, one call)",
                          "algorithmic_bytes_per_launch": bytes_call,
                          "kernel_us": kern_ms * 1e3, "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src}, burst copy)",
@@ -469,7 +498,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=32)
     ap.add_argument("--traffic", type=float, default=None,
-                    help="DRAM bytes per launch of the prefill kernel from an ncu capture (reported as given)")
+                    help="DRAM bytes per headline call to report instead of profiles/traffic.json")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

@@ -725,7 +725,8 @@ constexpr int kRecThreads = 512;  // 16 warps; warp w reads TMEM lanes 32*(w%4).
 
 //  region   size        holds
 //  QW       64 KB       [-W; Qt] of the current chunk
-//  PT       32 KB       P in rows 64..127 (K blocks at +8K, +24K); e^g_last slots [2][128] at +0
+//  PT       2 x 32 KB   P of chunks i, i+1 (alternating) in rows 64..127 (K blocks at +8K,
+//                       +24K); the chunk's e^g_last in the unused rows at +0
 //  KHT      32 KB       Kh^T
 //  ST       DV*512 B    S^T (DV x 128), the B operand of group 1
 //  UT       DV*256 B    U^T (DV x 64), the B operand of group 2
@@ -733,10 +734,10 @@ template <int DV>
 struct RecSmem {
   static constexpr int kQW = 0;
   static constexpr int kPT = 65536;
-  static constexpr int kKHT = 98304;
-  static constexpr int kST = 131072;
+  static constexpr int kKHT = 131072;
+  static constexpr int kST = 163840;
   static constexpr int kUT = kST + DV * 512;
-  static constexpr int kBar = kUT + DV * 256;  // 3 mbarriers
+  static constexpr int kBar = kUT + DV * 256;  // 4 mbarriers
   static constexpr int kTmemSlot = kBar + 32;
   static constexpr int kTotal = kTmemSlot + 16;
   static constexpr int kAlloc = kTotal + 1024;
@@ -781,16 +782,17 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
-  const float* sGamma = reinterpret_cast<const float*>(sm + SM::kPT);  // [2][128]
   uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + SM::kBar);
   uint64_t* bar_qw = bar_mma + 1;
   uint64_t* bar_pk = bar_mma + 2;
+  uint64_t* bar_o = bar_mma + 3;  // the chunk's P U is done: its output rows may be read
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmemSlot);
 
   if (tid == 0) {
     mbar_init(bar_mma, 1);
     mbar_init(bar_qw, 1);
     mbar_init(bar_pk, 1);
+    mbar_init(bar_o, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -812,13 +814,14 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
     bulk_load(sm + SM::kQW, item_of(c) + kItemQW, 65536u, bar_qw);
     ++qw_issued;
   };
-  auto load_pk = [&](int c, int slot) {
+  auto load_pk = [&](int c, int slot) {  // P and e^g_last into PT[slot], Kh^T
     const uint8_t* it = item_of(c);
+    uint8_t* pt = sm + SM::kPT + slot * 32768;
     mbar_arrive_expect_tx(bar_pk, 16384u + 32768u + 512u);
-    bulk_load(sm + SM::kPT + 8192, it + kItemP, 8192u, bar_pk);
-    bulk_load(sm + SM::kPT + 24576, it + kItemP + 8192, 8192u, bar_pk);
+    bulk_load(pt + 8192, it + kItemP, 8192u, bar_pk);
+    bulk_load(pt + 24576, it + kItemP + 8192, 8192u, bar_pk);
     bulk_load(sm + SM::kKHT, it + kItemKHT, 32768u, bar_pk);
-    bulk_load(sm + SM::kPT + slot * 512, it + kItemGamma, 512u, bar_pk);
+    bulk_load(pt, it + kItemGamma, 512u, bar_pk);
     ++pk_issued;
   };
   if (tid == 0 && c_begin < c_end) {
@@ -902,6 +905,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
     tc_fence_after_sync();
   };
   int qw_waited = 0, pk_waited = 0;  // (thread 0: QW; every thread: PK)
+  uint32_t o_phase = 0;               // output-row warps: completions of bar_o seen
 
   int64_t prev_t0 = -1;
   int prev_len = 0;
@@ -922,7 +926,12 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
       for (int kk = 0; kk < 16; ++kk) umma_tf32(d1, a0 + kstep(kk, 128), b0 + kstep(kk, DV), kIdV, kk > 0);
       umma_commit(bar_mma);
     }
-    if (prev_t0 >= 0) out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);  // while the MMAs run
+    if (prev_t0 >= 0 && lq >= 2) {  // the previous chunk's output rows, while the MMAs run
+      if (!lost && !mbar_wait(bar_o, o_phase, a.status)) lost = true;
+      o_phase ^= 1u;
+      tc_fence_after_sync();
+      out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);
+    }
     wait_mma();
 
     // -- U = U~ + D1[0:64] -> U^T operand; next chunk's [-W; Qt] on its way ------------------
@@ -948,22 +957,26 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
     tc_fence_before_sync();
     __syncthreads();
 
-    // -- group 2: D2 += Kh^T U,  D1 += [.; P] U  ->  O = Qt S + P U in rows 64..127 ---------
+    // -- group 2: D2 += Kh^T U (the state chain waits for this commit only), then
+    //    D1 += [.; P] U -> O = Qt S + P U in rows 64..127 (read a chunk later) ----------------
     if (tid == 0) {
       tc_fence_after_sync();
-      const uint64_t ka = kdesc0(sb + SM::kKHT), ub = kdesc0(sb + SM::kUT), pa = kdesc0(sb + SM::kPT);
+      const uint64_t ka = kdesc0(sb + SM::kKHT), ub = kdesc0(sb + SM::kUT);
+      const uint64_t pa = kdesc0(sb + SM::kPT + (i & 1) * 32768);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) umma_tf32(tmem + kD2, ka + kstep(kk, 128), ub + kstep(kk, DV), kIdV, 1u);
+      umma_commit(bar_mma);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) umma_tf32(d1, pa + kstep(kk, 128), ub + kstep(kk, DV), kIdV, 1u);
-      umma_commit(bar_mma);
+      umma_commit(bar_o);
     }
     wait_mma();
 
-    // -- S <- e^g_last D2 (TMEM and S^T); next chunk's P, Kh^T, e^g_last on their way -------
+    // -- S <- e^g_last D2 (TMEM and S^T); next chunk's P, Kh^T, e^g_last on their way (the
+    //    other PT buffer: its last reader, the P U of chunk i-1, finished before group 1) --
     if (tid == 0 && c + 1 < c_end) load_pk(c + 1, (i + 1) & 1);
     {
-      const float gm = sGamma[(i & 1) * 128 + row];
+      const float gm = reinterpret_cast<const float*>(sm + SM::kPT + (i & 1) * 32768)[row];
 #pragma unroll
       for (int j = 0; j < kPart; j += 8) {
         const int cc = cp * kPart + j;
@@ -987,7 +1000,12 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
     prev_len = len;
     b ^= 1;
   }
-  if (!failed && prev_t0 >= 0) out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);
+  if (!failed && prev_t0 >= 0 && lq >= 2) {
+    if (!lost && !mbar_wait(bar_o, o_phase, a.status)) lost = true;
+    o_phase ^= 1u;
+    tc_fence_after_sync();
+    out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);
+  }
 
   // ---- final state ---------------------------------------------------------------------------
   if (!failed && a.ht) {
@@ -1056,12 +1074,12 @@ cudaError_t launch_recur_dv(const PrefillArgs& a, const SplitPlan& p, cudaStream
 
 template <typename TOut>
 cudaError_t launch_recur(const PrefillArgs& a, const SplitPlan& p, cudaStream_t stream) {
-  // value-column slices per chain: split when there are few (sequence, head) chains, as
-  // far as a single wave of CTAs over the 148 SMs allows (one CTA per SM)
+  // value-column slices per chain: as many as a single wave of CTAs over the 148 SMs
+  // allows (one CTA per SM); the two-pass form is only chosen for <= 74 chains
   const int64_t chains = static_cast<int64_t>(a.N) * a.H;
   if (4 * chains <= 148) return launch_recur_dv<32, TOut>(a, p, stream);
-  if (2 * chains <= 148) return launch_recur_dv<64, TOut>(a, p, stream);
-  return launch_recur_dv<128, TOut>(a, p, stream);
+  if (chains <= kSplitMaxChains) return launch_recur_dv<64, TOut>(a, p, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace

@@ -62,3 +62,26 @@ def test_algorithmic_work_figures():
     assert bench.prefill_tc_flops(4096) == 4096 * 32 * (6 * 128 * 128 + 10 * 64 * 128)
     # decode: two passes over a 64 KiB fp32 state per (sequence, head) plus the token
     assert bench.decode_bytes(256) == 256 * 32 * (2 * 128 * 128 * 4 + 4 * 128 * 2 + 128 * 4 + 4)
+
+
+def test_traffic_figure_is_tied_to_the_kernel_sources(tmp_path, monkeypatch):
+    import json
+    import bench
+    # the committed figure is reported only while the kernel sources hash the same
+    j = json.load(open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    expected = float(j["bytes_per_call"]) if j["source_sha256"] == bench.kernel_sources_sha256() else None
+    assert bench.load_traffic() == expected
+    assert bench.load_traffic(123.0) == 123.0  # an explicit figure wins
+    # a figure captured from other sources reads null
+    fake_root = tmp_path / "root"
+    (fake_root / "profiles").mkdir(parents=True)
+    (fake_root / "profiles" / "traffic.json").write_text(json.dumps({"source_sha256": "0" * 64, "bytes_per_call": 1.0}))
+    monkeypatch.setattr(bench, "ROOT", str(fake_root))
+    monkeypatch.setattr(bench, "kernel_sources_sha256", lambda: "f" * 64)
+    assert bench.load_traffic() is None
+
+
+def test_launch_count_follows_the_dispatch():
+    import bench
+    assert bench.kernels_per_call(256) == 1          # status word only: single-pass kernel
+    assert bench.kernels_per_call(303_000_000) == 3  # two-pass scratch: plan, intra, recurrence
