@@ -177,6 +177,35 @@ def test_prefill_many_short_sequences(kda):
         assert_prefill_close(fin[n:n + 1], rf, f"final seq {n} (len {e - s})")
 
 
+def test_prefill_two_pass_limit_and_many_short_sequences(kda):
+    """74 (sequence, head) chains run the two-pass kernels, 75 the single-pass kernel (the
+    workspace query tells which). 74 packed sequences of 0..130 tokens (empty, single-token
+    and chunk-boundary lengths) through the two-pass path against the oracle; then one more
+    sequence through the single-pass path, which must agree on the shared sequences."""
+    import torch
+    rng = np.random.default_rng(I.SEED_BASE + 33)
+    lens = [int(x) for x in rng.integers(0, 131, 74)]
+    lens[:6] = [0, 1, 63, 64, 65, 128]
+    w = I.make_prefill(lens + [40], 1, 128, 128, seed=I.SEED_BASE + 34)
+    assert kda.chunk_fwd_workspace_bytes(int(w.cu_seqlens[74]), 74, 1, 128, 128, kda.KDA_DT_BF16) > 256
+    assert kda.chunk_fwd_workspace_bytes(int(w.cu_seqlens[75]), 75, 1, 128, 128, kda.KDA_DT_BF16) == 256
+    d = _upload(w)
+    T74 = int(w.cu_seqlens[74])
+    cut = lambda x: x[:T74].contiguous()
+    out2, fin2 = kda.chunk_fwd(cut(d["q"]), cut(d["k"]), cut(d["v"]), cut(d["log_alpha"]), cut(d["beta"]),
+                               d["initial_state"][:74].contiguous(), d["cu_seqlens"][:75].contiguous(), N=74,
+                               check_status=True)
+    out1, fin1 = kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                               d["cu_seqlens"], N=75, check_status=True)
+    torch.cuda.synchronize()
+    out2, fin2, out1, fin1 = to_host(out2), to_host(fin2), to_host(out1), to_host(fin1)
+    ro, rf = O.kda_recurrence(w.q, w.k, w.v, w.log_alpha, w.beta, w.initial_state, w.cu_seqlens)
+    assert_prefill_close(out2, ro[:T74], "two-pass out (74 sequences)", stored_bf16=True)
+    assert_prefill_close(fin2, rf[:74], "two-pass final states")
+    assert_prefill_close(out1, ro, "single-pass out (75 sequences)", stored_bf16=True)
+    assert_prefill_close(fin1, rf, "single-pass final states")
+
+
 def test_prefill_split_and_state_alias(kda):
     """run(T) == run(T1) then run(T - T1) from the carried state, with final_state
     written over initial_state in place; and prefill then one decode step equals
