@@ -31,6 +31,10 @@ What it computes (all in float64, from the exact input values upcast):
 * ``kda_decode_step`` — one token of the recurrence for a batch of sequences,
   updating the state in place (the constant-size state is what makes decode
   cost independent of context length, same article section).
+* ``kda_mixer_decode_step`` — one serving decode token of the full mixer: the
+  same conv4 / L2 norm / recurrence / gate steps as ``kda_mixer`` applied to one
+  new token, with the convolution's last three raw inputs kept per sequence (a
+  conv history) instead of the whole sequence.
 
 Readings where the pages are silent (the full list is kept with the design
 notes): no 1/sqrt(d_k) query scale; log_alpha is given directly (natural log,
@@ -236,3 +240,32 @@ def kda_decode_steps(q, k, v, log_alpha, beta, state, seq_subset: Optional[np.nd
                                np.asarray(log_alpha[s])[idx], np.asarray(beta[s])[idx], S)
         outs.append(o)
     return np.stack(outs), S
+
+
+def kda_mixer_decode_step(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state, conv_hist):
+    """One serving decode token of the full mixer for N sequences (d_k = d_v = d).
+
+    q_raw, k_raw, v_raw [N, H, d]: this token's raw projections; conv_w [3, H*d, 4];
+    log_alpha [N, H, d]; beta [N, H]; gate [N, H, d] or None; state [N, H, d, d];
+    conv_hist [N, H, 3, 3, d]: for q, k, v (axis 2) the three previous raw rows of
+    each sequence, oldest first (zeros before the sequence's first token).
+
+    Steps, as ``kda_mixer`` takes them for one token: y[c] = sum_j w[c, j] x[t-3+j, c]
+    over (history, current token); q, k <- l2norm(y); v <- y; the KDA token step
+    (``kda_decode_step``); out * sigmoid(gate). The history then drops its oldest row
+    and appends the current raw token.
+    Returns (out [N, H, d], new state [N, H, d, d], new conv_hist).
+    """
+    hist = _f64(conv_hist)
+    N, H, _, _, d = hist.shape
+    w = _f64(conv_w).reshape(3, H, d, CONV_WIDTH)
+    ys, new_hist = [], hist.copy()
+    for i, x in enumerate((q_raw, k_raw, v_raw)):
+        x = _f64(x)
+        window = np.concatenate([hist[:, :, i], x[:, :, None, :]], axis=2)  # [N, H, 4, d], oldest first
+        ys.append(np.einsum("nhjc,hcj->nhc", window, w[i]))
+        new_hist[:, :, i] = window[:, :, 1:]
+    out, new_state = kda_decode_step(l2norm(ys[0]), l2norm(ys[1]), ys[2], log_alpha, beta, state)
+    if gate is not None:
+        out = output_gate(out, gate)
+    return out, new_state, new_hist

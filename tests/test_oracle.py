@@ -312,3 +312,51 @@ def test_cost_model_figures_pin_state_shape():
     for wrong in (state // 2, state * 2):
         t2 = mla_bytes_per_token * g["context_tokens"] + f["kda_layers"] * (wrong + conv)
         assert round(t2 / 2**30, 2) != g["kv_cache_plus_state_at_256k_bf16_gib"]
+
+
+def test_mixer_decode_steps_reproduce_the_mixer_prefill():
+    """Decoding a sequence token by token from an empty conv history and a zero state,
+    with the serving decode step, gives the prefill mixer's outputs and final state
+    (the two take their convolution windows from different code: packed sequences
+    with zero history at each start, against a rolling three-row history)."""
+    rng = np.random.default_rng(137101)
+    N, T, H, d = 3, 9, 2, 8
+    q = rng.standard_normal((N, T, H, d))
+    k = rng.standard_normal((N, T, H, d))
+    v = rng.standard_normal((N, T, H, d))
+    la = -np.log1p(np.exp(rng.standard_normal((N, T, H, d)))) / 4
+    b = 1 / (1 + np.exp(-rng.standard_normal((N, T, H))))
+    g = rng.standard_normal((N, T, H, d))
+    w = rng.standard_normal((3, H * d, 4)) * 0.5
+    s0 = rng.standard_normal((N, H, d, d)) * 0.1
+    packed = lambda x: x.reshape(N * T, *x.shape[2:])
+    cu = np.arange(N + 1) * T
+    ref_o, ref_s = O.kda_mixer(packed(q), packed(k), packed(v), w, packed(la), packed(b), packed(g), cu, s0)
+    S, hist = s0.copy(), np.zeros((N, H, 3, 3, d))
+    outs = []
+    for t in range(T):
+        o, S, hist = O.kda_mixer_decode_step(q[:, t], k[:, t], v[:, t], w, la[:, t], b[:, t], g[:, t], S, hist)
+        outs.append(o)
+    np.testing.assert_allclose(np.stack(outs, axis=1).reshape(N * T, H, d), ref_o, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S, ref_s, rtol=1e-11, atol=1e-12)
+    # the history holds the last three raw rows, oldest first
+    np.testing.assert_array_equal(hist[:, :, 0], q[:, T - 3:].transpose(0, 2, 1, 3))
+    np.testing.assert_array_equal(hist[:, :, 2], v[:, T - 3:].transpose(0, 2, 1, 3))
+
+
+def test_mixer_decode_step_with_history_matches_a_longer_prefill():
+    """After a prefill of T tokens, one decode step fed the prefill's last three raw rows
+    as its history equals the prefill of T + 1 tokens at the last token."""
+    rng = np.random.default_rng(137102)
+    T, H, d = 6, 2, 8
+    mk = lambda *s: rng.standard_normal(s)
+    q, k, v, g = mk(T + 1, H, d), mk(T + 1, H, d), mk(T + 1, H, d), mk(T + 1, H, d)
+    la = -np.log1p(np.exp(mk(T + 1, H, d))) / 4
+    b = 1 / (1 + np.exp(-mk(T + 1, H)))
+    w = mk(3, H * d, 4) * 0.5
+    o_long, s_long = O.kda_mixer(q, k, v, w, la, b, g, np.array([0, T + 1]))
+    _, s_T = O.kda_mixer(q[:T], k[:T], v[:T], w, la[:T], b[:T], g[:T], np.array([0, T]))
+    hist = np.stack([x[T - 3:T].transpose(1, 0, 2) for x in (q, k, v)], axis=1)[None]  # [1, H, 3, 3, d]
+    o, S, _ = O.kda_mixer_decode_step(q[T:], k[T:], v[T:], w, la[T:], b[T:], g[T:], s_T, hist)
+    np.testing.assert_allclose(o[0], o_long[T], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S[0], s_long[0], rtol=1e-11, atol=1e-12)
