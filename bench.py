@@ -67,6 +67,13 @@ def decode_bytes(N: int, Hh: int = H, d: int = D) -> int:
     return N * Hh * (2 * d * d * 4 + 4 * d * 2 + d * 4 + 4)
 
 
+def mixer_decode_bytes(N: int, Hh: int = H, d: int = D) -> int:
+    """Serving mixer decode step: the fp32 state and the bf16 three-row conv history of q, k,
+    v read and written per (sequence, head), plus the token's raw q, k, v, gate, out (bf16),
+    log_alpha (fp32), beta and the slot index."""
+    return N * Hh * (2 * d * d * 4 + 2 * 9 * d * 2 + 5 * d * 2 + d * 4 + 4) + N * 4
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -397,6 +404,45 @@ def run_gpu(args):
                            "algorithmic_bytes_per_launch": dbytes}}
     del state, toks
 
+    # ---------------- serving mixer decode: conv history + L2 + KDA + gate, pooled ---------
+    mdec = None
+    if not args.quick:
+        pool = Nd
+        gm = torch.Generator(device=device).manual_seed(1370005)
+        sp = 0.02 * torch.randn(pool, H, D, D, generator=gm, device=device)
+        cp = torch.randn(pool, H, 3, 3, D, generator=gm, device=device).bfloat16()
+        idx = torch.randperm(pool, generator=gm, device=device).to(torch.int32)
+        cw = (0.5 * torch.randn(3, H * D, 4, generator=gm, device=device)).contiguous()
+        mtoks = []
+        for _ in range(n_tok_sets):
+            mtoks.append(dict(q=torch.randn(Nd, H, D, generator=gm, device=device).bfloat16(),
+                              k=torch.randn(Nd, H, D, generator=gm, device=device).bfloat16(),
+                              v=torch.randn(Nd, H, D, generator=gm, device=device).bfloat16(),
+                              g=torch.randn(Nd, H, D, generator=gm, device=device).bfloat16(),
+                              la=(-torch.nn.functional.softplus(torch.randn(Nd, H, D, generator=gm, device=device))
+                                  / 16).contiguous(),
+                              b=torch.sigmoid(torch.randn(Nd, H, generator=gm, device=device)).contiguous()))
+        md_out = torch.empty(Nd, H, D, dtype=torch.bfloat16, device=device)
+
+        def mdstep(i):
+            t = mtoks[i % n_tok_sets]
+            kda.mixer_decode_step(t["q"], t["k"], t["v"], cw, t["la"], t["b"], t["g"], sp, cp, idx, out=md_out,
+                                  stream=stream)
+
+        mper, mtot = time_region(mdstep, dsteps, 3, stream, device)
+        launches += dsteps
+        mtot = max_over_ranks(mtot, device)
+        mbytes_d = mixer_decode_bytes(Nd)
+        m_us = mtot / dsteps * 1e3
+        mdec = {"workload": f"serving mixer decode N={Nd} H={H} d={D}: conv4 over a 3-row history, L2, KDA, gate; "
+                            f"states and histories at permuted slots of a {pool}-slot pool, {dsteps} steps",
+                "us_per_step": m_us, "tokens_per_s": job_throughput(Nd * dsteps, world, mtot / 1e3),
+                "roofline": {"bound": "hbm", "achieved": mbytes_d / (statistics.mean(mper) * 1e-3) / 1e9,
+                             "peak": hbm_peak, "unit": "GB/s",
+                             "frac": mbytes_d / (statistics.mean(mper) * 1e-3) / 1e9 / hbm_peak,
+                             "algorithmic_bytes_per_launch": mbytes_d}}
+        del sp, cp, mtoks
+
     # ---------------- full mixer (conv4 + L2 + KDA + gate), B=2 x T=32768 ----------------
     mix = None
     if not args.quick:
@@ -473,7 +519,7 @@ def run_gpu(args):
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "pipelining": "2 device buffer sets; upload, kernels and download of consecutive steps overlap "
                                   "on three streams; every step's copies are inside the timed region"},
-            "decode": decode, "mixer": mix, "varlen": var,
+            "decode": decode, "mixer_decode": mdec, "mixer": mix, "varlen": var,
             "clocks": clocks, "gpu_launches": launches, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

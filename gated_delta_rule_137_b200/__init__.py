@@ -9,6 +9,8 @@ calls raise.
     out, final = chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens)
     out        = decode_step(q, k, v, log_alpha, beta, state)      # state in place
     out, final = mixer_fwd(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, ...)
+    out        = mixer_decode_step(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate,
+                                   state_pool, conv_pool, state_indices)  # pools in place
 
 Shapes (token-major, packed): q, k, log_alpha [total_T, H, dk]; v [total_T, H, dv];
 beta [total_T, H]; states [N, H, dk, dv]; cu_seqlens int32 [N+1] (device).
@@ -28,6 +30,7 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUD
 KDA_DT_F32, KDA_DT_BF16 = 0, 1
 DEVFLAG_BAD_SEQLENS = 0x1
 DEVFLAG_DECAY_RANGE = 0x2
+DEVFLAG_BAD_INDEX = 0x4
 
 _lib = None
 
@@ -57,6 +60,8 @@ _SIGNATURES = {
     "kda_workspace_status": (_i32, [_vp, _vp, _u32p]),
     "kda_mixer_fwd_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
                                      _vp, _vp, _vp]),
+    "kda_mixer_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                                     _i32, _vp, _vp, _vp]),
 }
 
 
@@ -198,6 +203,24 @@ def mixer_fwd(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate=None, initial_s
     if check_status:
         workspace_status(workspace, stream)
     return out, final_state
+
+
+def mixer_decode_step(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool, conv_pool,
+                      state_indices=None, *, out=None, status=None, stream=None):
+    """Serving decode step of the full mixer (kda_mixer_decode_step): one token per
+    sequence, q_raw/k_raw/v_raw/gate bf16 [N, H, 128]; state_pool fp32 [P, H, 128, 128]
+    and conv_pool bf16 [P, H, 3, 3, 128] updated in place; state_indices int32 [N] or
+    None (slot n). `status`: a device uint32 tensor (>= 4 bytes) for device flags."""
+    torch = _torch()
+    lib = load_library()
+    N, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=torch.bfloat16, device=q_raw.device)
+    _check(lib.kda_mixer_decode_step(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w), _ptr(log_alpha),
+                                     _ptr(beta), _ptr(gate), _ptr(state_pool), _ptr(conv_pool), _ptr(state_indices),
+                                     state_pool.shape[0], N, H, dk, dv, _ptr(out), _ptr(status), _stream(stream)))
+    return out
 
 
 def workspace_status(workspace, stream=None) -> int:

@@ -80,6 +80,12 @@ cudaError_t launch_decode_step(const void* q, const void* k, const void* v, bool
                                const float* beta, float* state, int N, int H, int dk, int dv, void* out,
                                cudaStream_t stream);
 
+// Serving decode step of the full mixer (d = 128, bf16 raw inputs and out).
+cudaError_t launch_mixer_decode_step(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                                     const float* log_alpha, const float* beta, const void* gate, float* state_pool,
+                                     void* conv_pool, const int32_t* state_indices, int pool_size, int N, int H,
+                                     void* out, uint32_t* status, cudaStream_t stream);
+
 // Tensor-core chunked prefill on d = 128 operands (bf16 or fp32 q/k/v/out).
 cudaError_t launch_prefill_d128(const PrefillArgs& a, cudaStream_t stream);
 

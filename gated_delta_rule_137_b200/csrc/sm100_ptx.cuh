@@ -35,6 +35,7 @@ constexpr uint64_t kWaitBudgetNs = 2000000000ull;
 // KDA_DEVFLAG_* for the user-visible ones).
 constexpr uint32_t kFlagBadSeqlens = 0x1u;
 constexpr uint32_t kFlagDecayRange = 0x2u;
+constexpr uint32_t kFlagBadIndex = 0x4u;
 constexpr uint32_t kFlagWaitTimeout = 0x80000000u;
 
 // ---------------------------------------------------------------------------------

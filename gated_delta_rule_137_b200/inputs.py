@@ -194,6 +194,49 @@ def make_decode(N, H, dk, dv, steps, *, seed, state_std=0.02, name="decode") -> 
                           q=q, k=k, v=v, log_alpha=la, beta=beta, state=st)
 
 
+@dataclasses.dataclass
+class MixerDecodeWorkload:
+    """Serving decode of the full mixer: `steps` tokens for N sequences whose states and
+    conv histories live in pools of `pool` slots (slot of sequence n: indices[n])."""
+    name: str
+    N: int
+    H: int
+    d: int
+    steps: int
+    pool: int
+    q: np.ndarray          # raw [steps, N, H, d], bf16 values
+    k: np.ndarray
+    v: np.ndarray
+    log_alpha: np.ndarray  # [steps, N, H, d]
+    beta: np.ndarray       # [steps, N, H]
+    gate: np.ndarray       # [steps, N, H, d], bf16 values
+    conv_w: np.ndarray     # [3, H*d, 4]
+    state_pool: np.ndarray  # [pool, H, d, d]
+    conv_pool: np.ndarray   # [pool, H, 3, 3, d], bf16 values (raw rows, oldest first)
+    indices: np.ndarray     # int32 [N], distinct slots
+
+
+def make_mixer_decode(N, H, d, steps, pool, *, seed, state_std=0.02, name="mixer_decode") -> MixerDecodeWorkload:
+    rng = np.random.default_rng(seed)
+    q = _normal(rng, (steps, N, H, d))
+    k = _normal(rng, (steps, N, H, d))
+    v = _normal(rng, (steps, N, H, d))
+    gate = _normal(rng, (steps, N, H, d))
+    for x in (q, k, v, gate):
+        _bf16_round_inplace(x)
+    la = _normal(rng, (steps, N, H, d))
+    _neg_softplus_over_16_inplace(la)
+    beta = _normal(rng, (steps, N, H))
+    _sigmoid_inplace(beta)
+    conv_w = _normal(rng, (3, H * d, 4), 0.5)
+    st = _normal(rng, (pool, H, d, d), state_std)
+    hist = _normal(rng, (pool, H, 3, 3, d))
+    _bf16_round_inplace(hist)
+    idx = rng.permutation(pool)[:N].astype(np.int32)
+    return MixerDecodeWorkload(name=name, N=N, H=H, d=d, steps=steps, pool=pool, q=q, k=k, v=v, log_alpha=la,
+                               beta=beta, gate=gate, conv_w=conv_w, state_pool=st, conv_pool=hist, indices=idx)
+
+
 # --- the five named workloads ------------------------------------------------
 
 def tiny_recurrence() -> Workload:

@@ -73,6 +73,7 @@ typedef enum { KDA_DT_F32 = 0, KDA_DT_BF16 = 1 } kda_dtype;
 /* Bits of the device status word (kda_workspace_status). */
 #define KDA_DEVFLAG_BAD_SEQLENS 0x1u  /* cu_seqlens not monotone / out of range */
 #define KDA_DEVFLAG_DECAY_RANGE 0x2u  /* chunk decay beyond the supported range  */
+#define KDA_DEVFLAG_BAD_INDEX 0x4u    /* a state index outside [0, pool_size)    */
 
 /* Largest head dimensions this build accepts (d_k, d_v <= 128; the model uses 128). */
 #define KDA_MAX_HEAD_DIM 128
@@ -151,6 +152,40 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, kd
 KDA_API kda_status kda_decode_step(const void* q, const void* k, const void* v, kda_dtype qkv_dtype,
                            const float* log_alpha, const float* beta, float* state,
                            int N, int H, int dk, int dv, void* out, kda_stream_t stream);
+
+/*
+ * Serving decode step of the full mixer: one new token for each of N sequences,
+ * through the same steps as kda_mixer_fwd — conv4 on q, k, v (over the sequence's
+ * last three raw inputs and this token), L2 norm of q and k, the KDA decode step,
+ * the sigmoid output gate — with the states and the conv histories kept in pools
+ * indexed per sequence (the KDA panel of the article cited above, one token at a
+ * time; the pool indexing is the library's own serving layout).
+ *
+ *   q_raw, k_raw, v_raw  device bf16 [N, H, d]: this token's raw projections
+ *   conv_w       device fp32 [3, H*d, 4] (q, k, v), as for kda_mixer_fwd
+ *   log_alpha    device fp32 [N, H, d];  beta device fp32 [N, H]
+ *   gate         device bf16 [N, H, d] or NULL (no gate)
+ *   state_pool   device fp32 [pool_size, H, d, d], read and updated in place
+ *   conv_pool    device bf16 [pool_size, H, 3, 3, d]: per slot and head, for q, k, v
+ *                the last three raw rows, oldest first; updated in place (the
+ *                oldest row drops, this token's row is appended). A new sequence
+ *                starts from zeros; after a prefill it holds the prompt's last three
+ *                raw q, k, v rows (zeros where the prompt is shorter).
+ *   state_indices device int32 [N]: the slot of each sequence, or NULL for slot n.
+ *                Slots must be distinct within a call (two sequences on one slot
+ *                race); an index outside [0, pool_size) leaves that sequence untouched
+ *                and sets KDA_DEVFLAG_BAD_INDEX in `status`.
+ *   out          device bf16 [N, H, d]
+ *   status       device uint32 word (e.g. a workspace's first word) or NULL; read it
+ *                with kda_workspace_status.
+ * Requires dk = dv = d = 128. Alignment: 16 bytes for every pointer but
+ * state_indices (4). Returns KDA_OK once the work is enqueued.
+ */
+KDA_API kda_status kda_mixer_decode_step(const void* q_raw, const void* k_raw, const void* v_raw,
+                                 const float* conv_w, const float* log_alpha, const float* beta,
+                                 const void* gate, float* state_pool, void* conv_pool,
+                                 const int32_t* state_indices, int pool_size, int N, int H, int dk, int dv,
+                                 void* out, void* status, kda_stream_t stream);
 
 /* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes): the
  * status word plus the two-pass prefill's scratch, sized as for kda_chunk_fwd (the

@@ -140,3 +140,22 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
             mod.load_library(str(tmp_path / "nope.so"))
     finally:
         mod._lib = saved
+
+
+def test_mixer_decode_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, w=FAKE, la=FAKE, b=FAKE, g=None, sp=FAKE * 4, cp=FAKE * 64, idx=None,
+                 pool=8, N=4, H=2, dk=128, dv=128, out=FAKE * 128, status=None)
+        a.update(kw)
+        return lib.kda_mixer_decode_step(a["q"], a["k"], a["v"], a["w"], a["la"], a["b"], a["g"], a["sp"], a["cp"],
+                                         a["idx"], a["pool"], a["N"], a["H"], a["dk"], a["dv"], a["out"], a["status"],
+                                         None)
+    assert call(dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
+    assert call(pool=0) == kda.KDA_ERR_INVALID_ARG
+    assert call(N=9) == kda.KDA_ERR_INVALID_ARG             # no indices: slot n needs n < pool_size
+    assert call(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(sp=FAKE * 4 + 8) == kda.KDA_ERR_INVALID_ARG  # misaligned state pool
+    assert call(idx=FAKE + 2) == kda.KDA_ERR_INVALID_ARG     # misaligned indices
+    assert call(out=FAKE * 4) == kda.KDA_ERR_INVALID_ARG     # out overlaps the state pool
+    assert call(N=0) == kda.KDA_OK                           # nothing to do
+    assert b"pool_size" in lib.kda_last_error() or lib.kda_last_error() == b""

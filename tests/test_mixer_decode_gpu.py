@@ -1,0 +1,88 @@
+"""kda_mixer_decode_step (the serving decode step of the full mixer) through the C ABI
+against the oracle's kda_mixer_decode_step: several consecutive steps on sequences
+whose states and conv histories sit at permuted slots of larger pools. The out rows and
+states are held to the decode tolerance; the rolled conv histories must be bit-exact
+(they are copies of bf16 inputs), and the slots no sequence uses must not change."""
+import numpy as np
+import pytest
+
+from gated_delta_rule_137_b200 import inputs as I
+from oracle import kda_oracle as O
+from tests.helpers import assert_decode_out_close, assert_decode_state_close, to_device, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kda():
+    import torch
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    from gated_delta_rule_137_b200 import build
+    build.build()
+    import gated_delta_rule_137_b200 as m
+    m.load_library()
+    return m
+
+
+def _run(kda, w, use_gate=True):
+    import torch
+    sp = to_device(w.state_pool, "f32")
+    cp = to_device(w.conv_pool, "bf16")
+    idx = to_device(w.indices, "i32")
+    cw = to_device(w.conv_w, "f32")
+    status = torch.zeros(64, dtype=torch.int32, device="cuda")
+    outs = []
+    for s in range(w.steps):
+        o = kda.mixer_decode_step(to_device(w.q[s], "bf16"), to_device(w.k[s], "bf16"), to_device(w.v[s], "bf16"),
+                                  cw, to_device(w.log_alpha[s], "f32"), to_device(w.beta[s], "f32"),
+                                  to_device(w.gate[s], "bf16") if use_gate else None, sp, cp, idx, status=status)
+        outs.append(to_host(o))
+    torch.cuda.synchronize()
+    return np.stack(outs), to_host(sp), cp, int(to_host(status)[0])
+
+
+def _oracle(w, use_gate=True):
+    idx = w.indices
+    S, hist = w.state_pool[idx], w.conv_pool[idx]
+    outs = []
+    for s in range(w.steps):
+        o, S, hist = O.kda_mixer_decode_step(w.q[s], w.k[s], w.v[s], w.conv_w, w.log_alpha[s], w.beta[s],
+                                             w.gate[s] if use_gate else None, S, hist)
+        outs.append(o)
+    return np.stack(outs), S, hist
+
+
+@pytest.mark.parametrize("use_gate", [True, False])
+def test_mixer_decode_matches_oracle_on_permuted_pool_slots(kda, use_gate):
+    import torch
+    w = I.make_mixer_decode(12, 4, 128, 3, 20, seed=I.SEED_BASE + 41)
+    out, sp, cp, status = _run(kda, w, use_gate)
+    ro, rs, rh = _oracle(w, use_gate)
+    assert status == 0
+    assert_decode_out_close(out, ro, "mixer decode out")
+    assert_decode_state_close(sp[w.indices], rs, "mixer decode state")
+    # the history holds copies of bf16 inputs: bit-exact
+    got_h = cp.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref_h = I.bf16_bits(rh)
+    np.testing.assert_array_equal(got_h[w.indices], ref_h)
+    unused = np.setdiff1d(np.arange(w.pool), w.indices)
+    np.testing.assert_array_equal(sp[unused], w.state_pool[unused].astype(np.float32))
+    np.testing.assert_array_equal(got_h[unused], I.bf16_bits(w.conv_pool[unused]))
+
+
+def test_mixer_decode_flags_an_index_outside_the_pool(kda):
+    import torch
+    w = I.make_mixer_decode(4, 2, 128, 1, 6, seed=I.SEED_BASE + 42)
+    w.indices = np.array([0, 9, 2, -1], dtype=np.int32)  # 9 and -1 are outside [0, 6)
+    out, sp, cp, status = _run(kda, w)
+    assert status & kda.DEVFLAG_BAD_INDEX
+    # the valid sequences still match the oracle, the slots of the others are untouched
+    ok = np.array([0, 2])
+    w2 = I.make_mixer_decode(4, 2, 128, 1, 6, seed=I.SEED_BASE + 42)
+    S, hist = w2.state_pool[[0, 2]], w2.conv_pool[[0, 2]]
+    ro, rs, _ = O.kda_mixer_decode_step(w2.q[0][ok], w2.k[0][ok], w2.v[0][ok], w2.conv_w, w2.log_alpha[0][ok],
+                                        w2.beta[0][ok], w2.gate[0][ok], S, hist)
+    assert_decode_out_close(out[0][ok], ro, "valid rows")
+    assert_decode_state_close(sp[[0, 2]], rs, "valid states")
+    for slot in (1, 3, 4, 5):
+        np.testing.assert_array_equal(sp[slot], w2.state_pool[slot].astype(np.float32))

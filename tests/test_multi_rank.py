@@ -85,3 +85,10 @@ def test_launch_count_follows_the_dispatch():
     import bench
     assert bench.kernels_per_call(256) == 1          # status word only: single-pass kernel
     assert bench.kernels_per_call(303_000_000) == 3  # two-pass scratch: plan, intra, recurrence
+
+
+def test_mixer_decode_work_figure():
+    import bench
+    # state r+w, conv history r+w (3 tensors x 3 rows, bf16), q/k/v/gate/out bf16, log_alpha, beta, index
+    per_seq_head = 2 * 128 * 128 * 4 + 2 * 9 * 128 * 2 + 5 * 128 * 2 + 128 * 4 + 4
+    assert bench.mixer_decode_bytes(256) == 256 * 32 * per_seq_head + 256 * 4
