@@ -74,6 +74,12 @@ def mixer_decode_bytes(N: int, Hh: int = H, d: int = D) -> int:
     return N * Hh * (2 * d * d * 4 + 2 * 9 * d * 2 + 5 * d * 2 + d * 4 + 4) + N * 4
 
 
+def mixer_decode_tokens_bytes(N: int, K: int, Hh: int = H, d: int = D) -> int:
+    """K tokens per call without checkpoints: the state and conv history read and written
+    once, each token's raw q, k, v, gate, out (bf16), log_alpha and beta, the slot index."""
+    return N * Hh * (2 * d * d * 4 + 2 * 9 * d * 2 + K * (5 * d * 2 + d * 4 + 4)) + N * 4
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -441,7 +447,29 @@ def run_gpu(args):
                              "peak": hbm_peak, "unit": "GB/s",
                              "frac": mbytes_d / (statistics.mean(mper) * 1e-3) / 1e9 / hbm_peak,
                              "algorithmic_bytes_per_launch": mbytes_d}}
-        del sp, cp, mtoks
+        # K = 4 draft tokens per call (no checkpoints: the pools get the state after the 4)
+        Kt = 4
+        ktok = [{k: torch.stack([mtoks[(s + j) % n_tok_sets][k] for j in range(Kt)], dim=1).contiguous()
+                 for k in mtoks[0]} for s in range(2)]
+        mk_out = torch.empty(Nd, Kt, H, D, dtype=torch.bfloat16, device=device)
+
+        def mkstep(i):
+            t = ktok[i % 2]
+            kda.mixer_decode_tokens(t["q"], t["k"], t["v"], cw, t["la"], t["b"], t["g"], sp, cp, idx, out=mk_out,
+                                    stream=stream)
+
+        ksteps = 16
+        kper, ktot = time_region(mkstep, ksteps, 3, stream, device)
+        launches += ksteps
+        ktot = max_over_ranks(ktot, device)
+        kbytes = mixer_decode_tokens_bytes(Nd, Kt)
+        mdec["k_tokens"] = {
+            "workload": f"{Kt} tokens per sequence per call (N={Nd} H={H}), state kept on chip across them",
+            "us_per_call": ktot / ksteps * 1e3, "tokens_per_s": job_throughput(Nd * Kt * ksteps, world, ktot / 1e3),
+            "roofline": {"bound": "hbm", "achieved": kbytes / (statistics.mean(kper) * 1e-3) / 1e9, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": kbytes / (statistics.mean(kper) * 1e-3) / 1e9 / hbm_peak,
+                         "algorithmic_bytes_per_launch": kbytes}}
+        del sp, cp, mtoks, ktok
 
     # ---------------- full mixer (conv4 + L2 + KDA + gate), B=2 x T=32768 ----------------
     mix = None

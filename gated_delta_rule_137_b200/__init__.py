@@ -62,6 +62,9 @@ _SIGNATURES = {
                                      _vp, _vp, _vp]),
     "kda_mixer_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
                                      _i32, _vp, _vp, _vp]),
+    "kda_mixer_decode_tokens": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                                       _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "kda_mixer_decode_commit": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
 }
 
 
@@ -221,6 +224,34 @@ def mixer_decode_step(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_
                                      _ptr(beta), _ptr(gate), _ptr(state_pool), _ptr(conv_pool), _ptr(state_indices),
                                      state_pool.shape[0], N, H, dk, dv, _ptr(out), _ptr(status), _stream(stream)))
     return out
+
+
+def mixer_decode_tokens(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool, conv_pool,
+                        state_indices=None, *, out=None, state_ckpt=None, conv_ckpt=None, status=None, stream=None):
+    """K tokens per sequence (kda_mixer_decode_tokens): q_raw/k_raw/v_raw/gate bf16
+    [N, K, H, 128]; with state_ckpt fp32 [N, K, H, 128, 128] and conv_ckpt bf16
+    [N, K, H, 3, 3, 128] the pools stay unchanged (see mixer_decode_commit)."""
+    torch = _torch()
+    lib = load_library()
+    N, K, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    if out is None:
+        out = torch.empty((N, K, H, dv), dtype=torch.bfloat16, device=q_raw.device)
+    _check(lib.kda_mixer_decode_tokens(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w), _ptr(log_alpha),
+                                       _ptr(beta), _ptr(gate), _ptr(state_pool), _ptr(conv_pool),
+                                       _ptr(state_indices), state_pool.shape[0], N, K, H, dk, dv, _ptr(out),
+                                       _ptr(state_ckpt), _ptr(conv_ckpt), _ptr(status), _stream(stream)))
+    return out
+
+
+def mixer_decode_commit(state_ckpt, conv_ckpt, accepted, state_pool, conv_pool, state_indices=None, *,
+                        status=None, stream=None):
+    """Install checkpoint accepted[n] - 1 into each sequence's slot (kda_mixer_decode_commit)."""
+    lib = load_library()
+    N, K, H, d = state_ckpt.shape[:4]
+    _check(lib.kda_mixer_decode_commit(_ptr(state_ckpt), _ptr(conv_ckpt), _ptr(accepted), _ptr(state_pool),
+                                       _ptr(conv_pool), _ptr(state_indices), state_pool.shape[0], N, K, H, d,
+                                       _ptr(status), _stream(stream)))
 
 
 def workspace_status(workspace, stream=None) -> int:

@@ -212,19 +212,21 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, kda_dtyp
   return ok();
 }
 
-kda_status kda_mixer_decode_step(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
-                                 const float* log_alpha, const float* beta, const void* gate, float* state_pool,
-                                 void* conv_pool, const int32_t* state_indices, int pool_size, int N, int H, int dk,
-                                 int dv, void* out, void* status, kda_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+}  // extern "C"
+namespace {
+// Checks shared by the serving mixer decode entry points (K tokens per sequence).
+kda_status check_mixer_decode(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                              const float* log_alpha, const float* beta, const void* gate, const float* state_pool,
+                              const void* conv_pool, const int32_t* state_indices, int pool_size, int N, int K, int H,
+                              int dk, int dv, const void* out, const void* status) {
   kda_status st = check_common(0, N, H, dk, dv);
   if (st != KDA_OK) return st;
   if (dk != kda::kD || dv != kda::kD)
-    return fail(KDA_ERR_UNSUPPORTED, "the mixer decode step is built for dk = dv = 128 (got %d, %d)", dk, dv);
+    return fail(KDA_ERR_UNSUPPORTED, "the mixer decode is built for dk = dv = 128 (got %d, %d)", dk, dv);
+  if (K < 0) return fail(KDA_ERR_INVALID_ARG, "K=%d must be >= 0", K);
   if (pool_size < 1) return fail(KDA_ERR_INVALID_ARG, "pool_size=%d must be >= 1", pool_size);
   if (!state_indices && N > pool_size)
     return fail(KDA_ERR_INVALID_ARG, "state_indices is NULL but N=%d exceeds pool_size=%d", N, pool_size);
-  if (N == 0) return ok();
   const void* ptrs[] = {q_raw, k_raw, v_raw, conv_w, log_alpha, beta, state_pool, conv_pool, out};
   const char* names[] = {"q_raw", "k_raw", "v_raw", "conv_w", "log_alpha", "beta", "state_pool", "conv_pool", "out"};
   for (int i = 0; i < 9; ++i) {
@@ -235,16 +237,70 @@ kda_status kda_mixer_decode_step(const void* q_raw, const void* k_raw, const voi
   if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return fail(KDA_ERR_INVALID_ARG, "status is not 4-byte aligned");
   if (state_indices && (reinterpret_cast<uintptr_t>(state_indices) & 3u))
     return fail(KDA_ERR_INVALID_ARG, "state_indices is not 4-byte aligned");
-  const size_t n_out = static_cast<size_t>(N) * H * dv * 2;
+  const size_t n_out = static_cast<size_t>(N) * K * H * dv * 2;
   const size_t n_state = static_cast<size_t>(pool_size) * H * dk * dv * sizeof(float);
   const size_t n_conv = static_cast<size_t>(pool_size) * H * 9 * dk * 2;
   if (ranges_overlap(out, n_out, state_pool, n_state) || ranges_overlap(out, n_out, conv_pool, n_conv) ||
       ranges_overlap(state_pool, n_state, conv_pool, n_conv))
     return fail(KDA_ERR_INVALID_ARG, "out, state_pool and conv_pool must not overlap");
-  cudaError_t e = kda::launch_mixer_decode_step(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool,
-                                                conv_pool, state_indices, pool_size, N, H, out,
-                                                static_cast<uint32_t*>(status), stream);
+  return KDA_OK;
+}
+}  // namespace
+extern "C" {
+kda_status kda_mixer_decode_step(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                                 const float* log_alpha, const float* beta, const void* gate, float* state_pool,
+                                 void* conv_pool, const int32_t* state_indices, int pool_size, int N, int H, int dk,
+                                 int dv, void* out, void* status, kda_stream_t stream_) {
+  kda_status st = check_mixer_decode(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool, conv_pool,
+                                     state_indices, pool_size, N, 1, H, dk, dv, out, status);
+  if (st != KDA_OK || N == 0) return st == KDA_OK ? ok() : st;
+  cudaError_t e = kda::launch_mixer_decode(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool, conv_pool,
+                                           state_indices, pool_size, N, 1, H, out, nullptr, nullptr,
+                                           static_cast<uint32_t*>(status), reinterpret_cast<cudaStream_t>(stream_));
   if (e != cudaSuccess) return cuda_fail(e, "mixer decode kernel launch");
+  return ok();
+}
+kda_status kda_mixer_decode_tokens(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                                   const float* log_alpha, const float* beta, const void* gate, float* state_pool,
+                                   void* conv_pool, const int32_t* state_indices, int pool_size, int N, int K, int H,
+                                   int dk, int dv, void* out, float* state_ckpt, void* conv_ckpt, void* status,
+                                   kda_stream_t stream_) {
+  kda_status st = check_mixer_decode(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool, conv_pool,
+                                     state_indices, pool_size, N, K, H, dk, dv, out, status);
+  if (st != KDA_OK) return st;
+  if ((state_ckpt == nullptr) != (conv_ckpt == nullptr))
+    return fail(KDA_ERR_INVALID_ARG, "state_ckpt and conv_ckpt must both be given or both be NULL");
+  if (state_ckpt && (!aligned16(state_ckpt) || !aligned16(conv_ckpt)))
+    return fail(KDA_ERR_INVALID_ARG, "state_ckpt and conv_ckpt must be 16-byte aligned");
+  if (N == 0 || K == 0) return ok();
+  cudaError_t e = kda::launch_mixer_decode(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool, conv_pool,
+                                           state_indices, pool_size, N, K, H, out, state_ckpt, conv_ckpt,
+                                           static_cast<uint32_t*>(status), reinterpret_cast<cudaStream_t>(stream_));
+  if (e != cudaSuccess) return cuda_fail(e, "mixer decode kernel launch");
+  return ok();
+}
+kda_status kda_mixer_decode_commit(const float* state_ckpt, const void* conv_ckpt, const int32_t* accepted,
+                                   float* state_pool, void* conv_pool, const int32_t* state_indices, int pool_size,
+                                   int N, int K, int H, int d, void* status, kda_stream_t stream_) {
+  kda_status st = check_common(0, N, H, d, d);
+  if (st != KDA_OK) return st;
+  if (d != kda::kD) return fail(KDA_ERR_UNSUPPORTED, "the mixer decode is built for d = 128 (got %d)", d);
+  if (K < 1 || pool_size < 1) return fail(KDA_ERR_INVALID_ARG, "K=%d and pool_size=%d must be >= 1", K, pool_size);
+  if (!state_indices && N > pool_size)
+    return fail(KDA_ERR_INVALID_ARG, "state_indices is NULL but N=%d exceeds pool_size=%d", N, pool_size);
+  const void* ptrs[] = {state_ckpt, conv_ckpt, accepted, state_pool, conv_pool};
+  const char* names[] = {"state_ckpt", "conv_ckpt", "accepted", "state_pool", "conv_pool"};
+  for (int i = 0; i < 5; ++i)
+    if (!ptrs[i]) return fail(KDA_ERR_INVALID_ARG, "%s must be non-NULL", names[i]);
+  if (!aligned16(state_ckpt) || !aligned16(conv_ckpt) || !aligned16(state_pool) || !aligned16(conv_pool))
+    return fail(KDA_ERR_INVALID_ARG, "checkpoints and pools must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(accepted) & 3u) || (state_indices && (reinterpret_cast<uintptr_t>(state_indices) & 3u)))
+    return fail(KDA_ERR_INVALID_ARG, "accepted and state_indices must be 4-byte aligned");
+  if (N == 0) return ok();
+  cudaError_t e = kda::launch_mixer_decode_commit(state_ckpt, conv_ckpt, accepted, state_pool, conv_pool,
+                                                  state_indices, pool_size, N, K, H, static_cast<uint32_t*>(status),
+                                                  reinterpret_cast<cudaStream_t>(stream_));
+  if (e != cudaSuccess) return cuda_fail(e, "mixer decode commit kernel launch");
   return ok();
 }
 size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv) {

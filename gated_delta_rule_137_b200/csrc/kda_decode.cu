@@ -148,14 +148,16 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
   }
 }
 
-// ---- serving decode step of the full mixer ------------------------------------------
+// ---- serving decode of the full mixer ---------------------------------------------------
 // Per (n, h) with slot p = state_indices[n] (n when the indices are NULL): the conv
-// history of slot p holds the last three raw q, k, v rows (bf16, oldest first). Thread
-// c < 128 convolves channel c of q and k over (history, this token), thread 128 + c
-// channel c of v; q and k are L2-normalised over the head's 128 channels; then the
-// decode step of decode_step_kernel on the slot's state, the sigmoid gate on the
-// output, and the history rolls by one row. (Ling-3.0-flash article, KDA panel: conv4,
-// L2 norm, the recurrence, the output gate; one token at a time.)
+// history of slot p holds the last three raw q, k, v rows (bf16, oldest first). For each
+// of the K tokens in order: thread c < 128 convolves channel c of q and k over (history,
+// token) and thread 128 + c channel c of v, rolling the history in registers; q and k are
+// L2-normalised over the head's 128 channels; the KDA decode step updates the state
+// (held in registers across the K tokens); the output gets the sigmoid gate. The state
+// and history after token j go to the checkpoints if given (the pools are then left
+// as they were), else the final ones go back into the pools. (Ling-3.0-flash article,
+// KDA panel: conv4, L2 norm, the recurrence, the output gate; one token at a time.)
 constexpr int kMixD = 128;
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -164,140 +166,231 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-__global__ void __launch_bounds__(kDecodeWarps * 32, 2)
-    mixer_decode_kernel(const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __restrict__ k_raw,
-                        const __nv_bfloat16* __restrict__ v_raw, const float* __restrict__ conv_w,
-                        const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                        const __nv_bfloat16* __restrict__ gate, float* __restrict__ state_pool,
-                        __nv_bfloat16* __restrict__ conv_pool, const int32_t* __restrict__ state_indices,
-                        int pool_size, int H, __nv_bfloat16* __restrict__ out, uint32_t* status) {
+struct MixerDecodeArgs {
+  const __nv_bfloat16* q_raw;  // [N, K, H, d]
+  const __nv_bfloat16* k_raw;
+  const __nv_bfloat16* v_raw;
+  const float* conv_w;         // [3, H*d, 4]
+  const float* log_alpha;      // [N, K, H, d]
+  const float* beta;           // [N, K, H]
+  const __nv_bfloat16* gate;   // [N, K, H, d] or null
+  float* state_pool;           // [P, H, d, d]
+  __nv_bfloat16* conv_pool;    // [P, H, 3, 3, d]
+  const int32_t* state_indices;
+  float* state_ckpt;           // [N, K, H, d, d] or null
+  __nv_bfloat16* conv_ckpt;    // [N, K, H, 3, 3, d] or null
+  __nv_bfloat16* out;          // [N, K, H, d]
+  uint32_t* status;
+  int pool_size, K, H;
+};
+
+// kSingle: one token and no checkpoints (the serving step), compiled without the token
+// loop's bookkeeping.
+template <bool kSingle>
+__global__ void __launch_bounds__(kDecodeWarps * 32, 2) mixer_decode_kernel(const MixerDecodeArgs a) {
   const int nh = blockIdx.x;  // n * H + h
+  const int H = a.H, K = kSingle ? 1 : a.K;
+  float* const state_ckpt = kSingle ? nullptr : a.state_ckpt;
   const int n = nh / H, h = nh % H;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int col = lane * 4;
-  const int slot = state_indices ? state_indices[n] : n;
-  if (slot < 0 || slot >= pool_size) {  // the whole CTA takes this branch
-    if (threadIdx.x == 0 && status) atomicOr(status, kFlagBadIndex);
+  const int slot = a.state_indices ? a.state_indices[n] : n;
+  if (slot < 0 || slot >= a.pool_size) {  // the whole CTA takes this branch
+    if (threadIdx.x == 0 && a.status) atomicOr(a.status, kFlagBadIndex);
     return;
   }
-  float* S = state_pool + (static_cast<size_t>(slot) * H + h) * kMixD * kMixD;
-  __nv_bfloat16* hist = conv_pool + (static_cast<size_t>(slot) * H + h) * (3 * 3 * kMixD);  // [q,k,v][row][c]
+  float* S = a.state_pool + (static_cast<size_t>(slot) * H + h) * kMixD * kMixD;
+  __nv_bfloat16* hist = a.conv_pool + (static_cast<size_t>(slot) * H + h) * (3 * 3 * kMixD);  // [q,k,v][row][c]
 
   __shared__ float s_k[kMixD], s_q[kMixD], s_alpha[kMixD], s_v[kMixD];
   __shared__ float s_ss[2][4];
   __shared__ float4 s_red[2][kDecodeWarps][32];
 
-  // 1) the state slice of this warp in flight
+  // the state slice of this warp, in flight first; it stays in registers for all K tokens
   float4 s[kRowsPerWarp];
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r)
     s[r] = __ldcs(reinterpret_cast<const float4*>(S + static_cast<size_t>(warp * kRowsPerWarp + r) * kMixD + col));
 
-  // 2) conv4 over (history, token); roll the history; L2 norm of q and k
+  // this thread's channel: history rows (oldest first) and conv weights of q, k (i < 128) or v
   const int i = threadIdx.x, c = i & (kMixD - 1);
-  const size_t tok = static_cast<size_t>(nh) * kMixD + c;
-  auto conv = [&](int t, const __nv_bfloat16* raw) -> float {
-    __nv_bfloat16* hr = hist + t * 3 * kMixD + c;
-    const __nv_bfloat16 x0 = hr[0], x1 = hr[kMixD], x2 = hr[2 * kMixD], x3 = raw[tok];
-    const float4 w = __ldg(reinterpret_cast<const float4*>(conv_w + ((static_cast<size_t>(t) * H + h) * kMixD + c) * 4));
-    hr[0] = x1;
-    hr[kMixD] = x2;
-    hr[2 * kMixD] = x3;
-    return fmaf(w.x, __bfloat162float(x0),
-                fmaf(w.y, __bfloat162float(x1), fmaf(w.z, __bfloat162float(x2), w.w * __bfloat162float(x3))));
-  };
-  float yq = 0.f, yk = 0.f;
-  if (i < kMixD) {
-    yq = conv(0, q_raw);
-    yk = conv(1, k_raw);
-    s_alpha[c] = expf(log_alpha[tok]);
-    const float sq = warp_sum(yq * yq), sk = warp_sum(yk * yk);
-    if (lane == 0) {
-      s_ss[0][warp] = sq;
-      s_ss[1][warp] = sk;
+  const int t0 = i < kMixD ? 0 : 2;    // first tensor of this thread: q (then k) or v
+  const int nt = i < kMixD ? 2 : 1;
+  float hx[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    if (u >= nt) break;
+    const __nv_bfloat16* hr = hist + (t0 + u) * 3 * kMixD + c;
+    hx[u][0] = __bfloat162float(hr[0]);
+    hx[u][1] = __bfloat162float(hr[kMixD]);
+    hx[u][2] = __bfloat162float(hr[2 * kMixD]);
+  }
+  const float* cwp = a.conv_w + (static_cast<size_t>(t0) * H + h) * kMixD * 4 + c * 4;  // + u * H * d * 4
+  const __nv_bfloat16* raw0 = i < kMixD ? a.q_raw : a.v_raw;  // this thread's tensors: q, k or v
+
+  for (int j = 0; j < K; ++j) {
+    const size_t tok = ((static_cast<size_t>(n) * K + j) * H + h) * kMixD + c;  // [n][j][h][c]
+    // conv4 over (history, token); roll the history; L2 norm of q and k
+    float y[2] = {0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u >= nt) break;
+      const float x3 = __bfloat162float((u == 0 ? raw0 : a.k_raw)[tok]);
+      const float4 cw = __ldg(reinterpret_cast<const float4*>(cwp + static_cast<size_t>(u) * H * kMixD * 4));
+      y[u] = fmaf(cw.x, hx[u][0], fmaf(cw.y, hx[u][1], fmaf(cw.z, hx[u][2], cw.w * x3)));
+      hx[u][0] = hx[u][1];
+      hx[u][1] = hx[u][2];
+      hx[u][2] = x3;
     }
-  } else {
-    s_v[c] = conv(2, v_raw);
-  }
-  __syncthreads();
-  if (i < kMixD) {
-    const float fq = rsqrtf(s_ss[0][0] + s_ss[0][1] + s_ss[0][2] + s_ss[0][3] + 1e-6f);
-    const float fk = rsqrtf(s_ss[1][0] + s_ss[1][1] + s_ss[1][2] + s_ss[1][3] + 1e-6f);
-    s_q[c] = yq * fq;
-    s_k[c] = yk * fk;
-  }
-  __syncthreads();
-
-  // 3) decay the rows and accumulate a = S'^T k, b = S'^T q (as decode_step_kernel)
-  float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
-#pragma unroll
-  for (int r = 0; r < kRowsPerWarp; ++r) {
-    const int row = warp * kRowsPerWarp + r;
-    const float al = s_alpha[row], kr = s_k[row], qr = s_q[row];
-    s[r].x *= al; s[r].y *= al; s[r].z *= al; s[r].w *= al;
-    pa.x = fmaf(kr, s[r].x, pa.x); pa.y = fmaf(kr, s[r].y, pa.y);
-    pa.z = fmaf(kr, s[r].z, pa.z); pa.w = fmaf(kr, s[r].w, pa.w);
-    pb.x = fmaf(qr, s[r].x, pb.x); pb.y = fmaf(qr, s[r].y, pb.y);
-    pb.z = fmaf(qr, s[r].z, pb.z); pb.w = fmaf(qr, s[r].w, pb.w);
-  }
-  s_red[0][warp][lane] = pa;
-  s_red[1][warp][lane] = pb;
-  float kq = 0.f;
-#pragma unroll
-  for (int j = lane; j < kMixD; j += 32) kq = fmaf(s_k[j], s_q[j], kq);
-  kq = warp_sum(kq);
-  __syncthreads();
-
-  float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-#pragma unroll
-  for (int w = 0; w < kDecodeWarps; ++w) {
-    const float4 x = s_red[0][w][lane], y = s_red[1][w][lane];
-    a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
-    b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
-  }
-  const float bt = beta[nh];
-  float4 u;
-  u.x = bt * (s_v[col + 0] - a.x);
-  u.y = bt * (s_v[col + 1] - a.y);
-  u.z = bt * (s_v[col + 2] - a.z);
-  u.w = bt * (s_v[col + 3] - a.w);
-
-  if (warp == 0) {
-    float o[4] = {fmaf(u.x, kq, b.x), fmaf(u.y, kq, b.y), fmaf(u.z, kq, b.z), fmaf(u.w, kq, b.w)};
-    const size_t oo = static_cast<size_t>(nh) * kMixD + col;
-    if (gate) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] *= 1.f / (1.f + expf(-__bfloat162float(gate[oo + e])));
+    if (i < kMixD) {
+      s_alpha[c] = expf(a.log_alpha[tok]);
+      const float sq = warp_sum(y[0] * y[0]), sk = warp_sum(y[1] * y[1]);
+      if (lane == 0) {
+        s_ss[0][warp] = sq;
+        s_ss[1][warp] = sk;
+      }
+    } else {
+      s_v[c] = y[0];
     }
-    store4<__nv_bfloat16>(out + oo, make_float4(o[0], o[1], o[2], o[3]));
+    __syncthreads();
+    if (i < kMixD) {
+      s_q[c] = y[0] * rsqrtf(s_ss[0][0] + s_ss[0][1] + s_ss[0][2] + s_ss[0][3] + 1e-6f);
+      s_k[c] = y[1] * rsqrtf(s_ss[1][0] + s_ss[1][1] + s_ss[1][2] + s_ss[1][3] + 1e-6f);
+    }
+    __syncthreads();
+
+    // decay the rows and accumulate a = S'^T k, b = S'^T q (as decode_step_kernel)
+    float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+      const int row = warp * kRowsPerWarp + r;
+      const float al = s_alpha[row], kr = s_k[row], qr = s_q[row];
+      s[r].x *= al; s[r].y *= al; s[r].z *= al; s[r].w *= al;
+      pa.x = fmaf(kr, s[r].x, pa.x); pa.y = fmaf(kr, s[r].y, pa.y);
+      pa.z = fmaf(kr, s[r].z, pa.z); pa.w = fmaf(kr, s[r].w, pa.w);
+      pb.x = fmaf(qr, s[r].x, pb.x); pb.y = fmaf(qr, s[r].y, pb.y);
+      pb.z = fmaf(qr, s[r].z, pb.z); pb.w = fmaf(qr, s[r].w, pb.w);
+    }
+    s_red[0][warp][lane] = pa;
+    s_red[1][warp][lane] = pb;
+    float kq = 0.f;
+#pragma unroll
+    for (int e = lane; e < kMixD; e += 32) kq = fmaf(s_k[e], s_q[e], kq);
+    kq = warp_sum(kq);
+    __syncthreads();
+
+    float4 ra = make_float4(0.f, 0.f, 0.f, 0.f), rb = ra;
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) {
+      const float4 x = s_red[0][w][lane], z = s_red[1][w][lane];
+      ra.x += x.x; ra.y += x.y; ra.z += x.z; ra.w += x.w;
+      rb.x += z.x; rb.y += z.y; rb.z += z.z; rb.w += z.w;
+    }
+    const float bt = a.beta[(static_cast<size_t>(n) * K + j) * H + h];
+    float4 uu;
+    uu.x = bt * (s_v[col + 0] - ra.x);
+    uu.y = bt * (s_v[col + 1] - ra.y);
+    uu.z = bt * (s_v[col + 2] - ra.z);
+    uu.w = bt * (s_v[col + 3] - ra.w);
+    if (warp == 0) {
+      float o[4] = {fmaf(uu.x, kq, rb.x), fmaf(uu.y, kq, rb.y), fmaf(uu.z, kq, rb.z), fmaf(uu.w, kq, rb.w)};
+      const size_t oo = ((static_cast<size_t>(n) * K + j) * H + h) * kMixD + col;
+      if (a.gate) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] *= 1.f / (1.f + expf(-__bfloat162float(a.gate[oo + e])));
+      }
+      store4<__nv_bfloat16>(a.out + oo, make_float4(o[0], o[1], o[2], o[3]));
+    }
+    // S' + k u^T
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+      const float kr = s_k[warp * kRowsPerWarp + r];
+      s[r].x = fmaf(kr, uu.x, s[r].x); s[r].y = fmaf(kr, uu.y, s[r].y);
+      s[r].z = fmaf(kr, uu.z, s[r].z); s[r].w = fmaf(kr, uu.w, s[r].w);
+    }
+    if (state_ckpt) {  // the state and history after token j
+      float* C = state_ckpt + ((static_cast<size_t>(n) * K + j) * H + h) * kMixD * kMixD;
+#pragma unroll
+      for (int r = 0; r < kRowsPerWarp; ++r)
+        __stcs(reinterpret_cast<float4*>(C + static_cast<size_t>(warp * kRowsPerWarp + r) * kMixD + col), s[r]);
+      __nv_bfloat16* hc = a.conv_ckpt + ((static_cast<size_t>(n) * K + j) * H + h) * (3 * 3 * kMixD) + c;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (u >= nt) break;
+#pragma unroll
+        for (int m = 0; m < 3; ++m) hc[((t0 + u) * 3 + m) * kMixD] = __float2bfloat16_rn(hx[u][m]);
+      }
+    }
+    if (!kSingle) __syncthreads();  // s_k, s_q, s_v, s_alpha are rewritten by the next token
   }
 
-  // 4) S' + k u^T back into the slot
+  if (!state_ckpt) {  // no checkpoints: the state and history after the K tokens go back
 #pragma unroll
-  for (int r = 0; r < kRowsPerWarp; ++r) {
-    const int row = warp * kRowsPerWarp + r;
-    const float kr = s_k[row];
-    float4 x = s[r];
-    x.x = fmaf(kr, u.x, x.x); x.y = fmaf(kr, u.y, x.y);
-    x.z = fmaf(kr, u.z, x.z); x.w = fmaf(kr, u.w, x.w);
-    __stcs(reinterpret_cast<float4*>(S + static_cast<size_t>(row) * kMixD + col), x);
+    for (int r = 0; r < kRowsPerWarp; ++r)
+      __stcs(reinterpret_cast<float4*>(S + static_cast<size_t>(warp * kRowsPerWarp + r) * kMixD + col), s[r]);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u >= nt) break;
+#pragma unroll
+      for (int m = 0; m < 3; ++m) hist[((t0 + u) * 3 + m) * kMixD + c] = __float2bfloat16_rn(hx[u][m]);
+    }
   }
+}
+
+// Commit after speculative decoding: slot <- the checkpoint after token accepted[n] - 1
+// (accepted[n] = 0 keeps the slot as it is). One CTA per (n, h) copies 64 KiB of state
+// and the 2.25 KiB history.
+__global__ void __launch_bounds__(256) mixer_decode_commit_kernel(
+    const float* __restrict__ state_ckpt, const __nv_bfloat16* __restrict__ conv_ckpt,
+    const int32_t* __restrict__ accepted, float* __restrict__ state_pool, __nv_bfloat16* __restrict__ conv_pool,
+    const int32_t* __restrict__ state_indices, int pool_size, int K, int H, uint32_t* status) {
+  const int nh = blockIdx.x, n = nh / H, h = nh % H;
+  const int slot = state_indices ? state_indices[n] : n;
+  const int acc = accepted[n];
+  if (slot < 0 || slot >= pool_size || acc < 0 || acc > K) {
+    if (threadIdx.x == 0 && status) atomicOr(status, kFlagBadIndex);
+    return;
+  }
+  if (acc == 0) return;
+  const size_t src = (static_cast<size_t>(n) * K + (acc - 1)) * H + h;
+  const size_t dst = static_cast<size_t>(slot) * H + h;
+  const float4* cs = reinterpret_cast<const float4*>(state_ckpt + src * kMixD * kMixD);
+  float4* ps = reinterpret_cast<float4*>(state_pool + dst * kMixD * kMixD);
+  for (int e = threadIdx.x; e < kMixD * kMixD / 4; e += blockDim.x) __stcs(ps + e, __ldcs(cs + e));
+  const uint4* ch = reinterpret_cast<const uint4*>(conv_ckpt + src * 9 * kMixD);
+  uint4* ph = reinterpret_cast<uint4*>(conv_pool + dst * 9 * kMixD);
+  for (int e = threadIdx.x; e < 9 * kMixD / 8; e += blockDim.x) ph[e] = ch[e];
 }
 
 }  // namespace
 
-cudaError_t launch_mixer_decode_step(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
-                                     const float* log_alpha, const float* beta, const void* gate, float* state_pool,
-                                     void* conv_pool, const int32_t* state_indices, int pool_size, int N, int H,
-                                     void* out, uint32_t* status, cudaStream_t stream) {
+cudaError_t launch_mixer_decode(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                                const float* log_alpha, const float* beta, const void* gate, float* state_pool,
+                                void* conv_pool, const int32_t* state_indices, int pool_size, int N, int K, int H,
+                                void* out, float* state_ckpt, void* conv_ckpt, uint32_t* status, cudaStream_t stream) {
+  const unsigned grid = static_cast<unsigned>(N) * static_cast<unsigned>(H);
+  if (grid == 0 || K == 0) return cudaSuccess;
+  MixerDecodeArgs a{static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(k_raw),
+                    static_cast<const __nv_bfloat16*>(v_raw), conv_w, log_alpha, beta,
+                    static_cast<const __nv_bfloat16*>(gate), state_pool, static_cast<__nv_bfloat16*>(conv_pool),
+                    state_indices, state_ckpt, static_cast<__nv_bfloat16*>(conv_ckpt),
+                    static_cast<__nv_bfloat16*>(out), status, pool_size, K, H};
+  if (K == 1 && !state_ckpt)
+    mixer_decode_kernel<true><<<grid, kDecodeWarps * 32, 0, stream>>>(a);
+  else
+    mixer_decode_kernel<false><<<grid, kDecodeWarps * 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mixer_decode_commit(const float* state_ckpt, const void* conv_ckpt, const int32_t* accepted,
+                                       float* state_pool, void* conv_pool, const int32_t* state_indices,
+                                       int pool_size, int N, int K, int H, uint32_t* status, cudaStream_t stream) {
   const unsigned grid = static_cast<unsigned>(N) * static_cast<unsigned>(H);
   if (grid == 0) return cudaSuccess;
-  mixer_decode_kernel<<<grid, kDecodeWarps * 32, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(k_raw),
-      static_cast<const __nv_bfloat16*>(v_raw), conv_w, log_alpha, beta, static_cast<const __nv_bfloat16*>(gate),
-      state_pool, static_cast<__nv_bfloat16*>(conv_pool), state_indices, pool_size, H,
-      static_cast<__nv_bfloat16*>(out), status);
+  mixer_decode_commit_kernel<<<grid, 256, 0, stream>>>(state_ckpt, static_cast<const __nv_bfloat16*>(conv_ckpt),
+                                                       accepted, state_pool, static_cast<__nv_bfloat16*>(conv_pool),
+                                                       state_indices, pool_size, K, H, status);
   return cudaGetLastError();
 }
 

@@ -80,11 +80,15 @@ cudaError_t launch_decode_step(const void* q, const void* k, const void* v, bool
                                const float* beta, float* state, int N, int H, int dk, int dv, void* out,
                                cudaStream_t stream);
 
-// Serving decode step of the full mixer (d = 128, bf16 raw inputs and out).
-cudaError_t launch_mixer_decode_step(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
-                                     const float* log_alpha, const float* beta, const void* gate, float* state_pool,
-                                     void* conv_pool, const int32_t* state_indices, int pool_size, int N, int H,
-                                     void* out, uint32_t* status, cudaStream_t stream);
+// Serving decode of the full mixer, K tokens per sequence (d = 128, bf16 raw inputs and
+// out); with checkpoints the pools are left unchanged.
+cudaError_t launch_mixer_decode(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                                const float* log_alpha, const float* beta, const void* gate, float* state_pool,
+                                void* conv_pool, const int32_t* state_indices, int pool_size, int N, int K, int H,
+                                void* out, float* state_ckpt, void* conv_ckpt, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_mixer_decode_commit(const float* state_ckpt, const void* conv_ckpt, const int32_t* accepted,
+                                       float* state_pool, void* conv_pool, const int32_t* state_indices,
+                                       int pool_size, int N, int K, int H, uint32_t* status, cudaStream_t stream);
 
 // Tensor-core chunked prefill on d = 128 operands (bf16 or fp32 q/k/v/out).
 cudaError_t launch_prefill_d128(const PrefillArgs& a, cudaStream_t stream);

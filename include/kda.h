@@ -187,6 +187,38 @@ KDA_API kda_status kda_mixer_decode_step(const void* q_raw, const void* k_raw, c
                                  const int32_t* state_indices, int pool_size, int N, int H, int dk, int dv,
                                  void* out, void* status, kda_stream_t stream);
 
+/*
+ * K consecutive tokens per sequence through the serving decode step (speculative
+ * decoding: K draft tokens in one call). Same arguments as kda_mixer_decode_step with
+ * a token axis: q_raw, k_raw, v_raw, log_alpha, gate, out [N, K, H, d]; beta [N, K, H].
+ * The state of a (sequence, head) stays on chip across the K tokens, so a call moves
+ * it once instead of K times.
+ *   state_ckpt  device fp32 [N, K, H, d, d] or NULL
+ *   conv_ckpt   device bf16 [N, K, H, 3, 3, d] or NULL (both or neither)
+ * Without checkpoints the pools receive the state and history after the K tokens.
+ * With checkpoints the pools are left unchanged and entry j holds the state and
+ * history after token j; kda_mixer_decode_commit then installs the entry of the last
+ * accepted token. K = 1 without checkpoints is kda_mixer_decode_step.
+ */
+KDA_API kda_status kda_mixer_decode_tokens(const void* q_raw, const void* k_raw, const void* v_raw,
+                                   const float* conv_w, const float* log_alpha, const float* beta,
+                                   const void* gate, float* state_pool, void* conv_pool,
+                                   const int32_t* state_indices, int pool_size, int N, int K, int H, int dk,
+                                   int dv, void* out, float* state_ckpt, void* conv_ckpt, void* status,
+                                   kda_stream_t stream);
+
+/*
+ * After kda_mixer_decode_tokens with checkpoints: for each sequence n with
+ * accepted[n] = a (device int32 [N], 0 <= a <= K) copy checkpoint a - 1 into the
+ * sequence's pool slot (a = 0 keeps the slot as it was before the K tokens). An
+ * out-of-range slot or count sets KDA_DEVFLAG_BAD_INDEX in `status` and leaves that
+ * sequence untouched. d = 128; pointers 16-byte aligned (accepted, state_indices: 4).
+ */
+KDA_API kda_status kda_mixer_decode_commit(const float* state_ckpt, const void* conv_ckpt,
+                                   const int32_t* accepted, float* state_pool, void* conv_pool,
+                                   const int32_t* state_indices, int pool_size, int N, int K, int H, int d,
+                                   void* status, kda_stream_t stream);
+
 /* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes): the
  * status word plus the two-pass prefill's scratch, sized as for kda_chunk_fwd (the
  * conv/L2 stage runs inside the prefill's first pass and needs no buffer of its own). */

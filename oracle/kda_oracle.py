@@ -35,6 +35,9 @@ What it computes (all in float64, from the exact input values upcast):
   same conv4 / L2 norm / recurrence / gate steps as ``kda_mixer`` applied to one
   new token, with the convolution's last three raw inputs kept per sequence (a
   conv history) instead of the whole sequence.
+* ``kda_mixer_decode_tokens`` — K consecutive tokens per sequence through
+  ``kda_mixer_decode_step``, keeping the state and history after every token (the
+  checkpoints a speculative decoder rolls back to when it accepts fewer tokens).
 
 Readings where the pages are silent (the full list is kept with the design
 notes): no 1/sqrt(d_k) query scale; log_alpha is given directly (natural log,
@@ -269,3 +272,21 @@ def kda_mixer_decode_step(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, st
     if gate is not None:
         out = output_gate(out, gate)
     return out, new_state, new_hist
+
+
+def kda_mixer_decode_tokens(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state, conv_hist):
+    """K consecutive decode tokens per sequence: q_raw, k_raw, v_raw, log_alpha, gate
+    [N, K, H, d]; beta [N, K, H]; state [N, H, d, d]; conv_hist [N, H, 3, 3, d].
+    Returns (out [N, K, H, d], states after each token [N, K, H, d, d], histories after
+    each token [N, K, H, 3, 3, d]); the last entries are the final state and history."""
+    K = np.shape(q_raw)[1]
+    S, hist = _f64(state), _f64(conv_hist)
+    outs, states, hists = [], [], []
+    for j in range(K):
+        o, S, hist = kda_mixer_decode_step(np.asarray(q_raw)[:, j], np.asarray(k_raw)[:, j], np.asarray(v_raw)[:, j],
+                                           conv_w, np.asarray(log_alpha)[:, j], np.asarray(beta)[:, j],
+                                           None if gate is None else np.asarray(gate)[:, j], S, hist)
+        outs.append(o)
+        states.append(S)
+        hists.append(hist)
+    return np.stack(outs, axis=1), np.stack(states, axis=1), np.stack(hists, axis=1)

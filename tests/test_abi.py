@@ -159,3 +159,21 @@ def test_mixer_decode_rejects_bad_arguments(lib):
     assert call(out=FAKE * 4) == kda.KDA_ERR_INVALID_ARG     # out overlaps the state pool
     assert call(N=0) == kda.KDA_OK                           # nothing to do
     assert b"pool_size" in lib.kda_last_error() or lib.kda_last_error() == b""
+
+
+def test_mixer_decode_tokens_and_commit_reject_bad_arguments(lib):
+    base = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE * 4, FAKE * 64, None, 8, 4, 3, 2, 128, 128, FAKE * 128,
+            None, None, None, None]
+    bad = list(base); bad[12] = -1                 # K < 0
+    assert lib.kda_mixer_decode_tokens(*bad) == kda.KDA_ERR_INVALID_ARG
+    bad = list(base); bad[17] = FAKE * 256         # state checkpoint without the history checkpoint
+    assert lib.kda_mixer_decode_tokens(*bad) == kda.KDA_ERR_INVALID_ARG
+    bad = list(base); bad[12] = 0                  # K = 0: nothing to do
+    assert lib.kda_mixer_decode_tokens(*bad) == kda.KDA_OK
+    cbase = [FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5, None, 8, 4, 3, 2, 128, None, None]
+    bad = list(cbase); bad[2] = None                # accepted missing
+    assert lib.kda_mixer_decode_commit(*bad) == kda.KDA_ERR_INVALID_ARG
+    bad = list(cbase); bad[8] = 0                   # K = 0
+    assert lib.kda_mixer_decode_commit(*bad) == kda.KDA_ERR_INVALID_ARG
+    bad = list(cbase); bad[10] = 64                 # d != 128
+    assert lib.kda_mixer_decode_commit(*bad) == kda.KDA_ERR_UNSUPPORTED

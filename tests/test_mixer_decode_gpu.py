@@ -86,3 +86,89 @@ def test_mixer_decode_flags_an_index_outside_the_pool(kda):
     assert_decode_state_close(sp[[0, 2]], rs, "valid states")
     for slot in (1, 3, 4, 5):
         np.testing.assert_array_equal(sp[slot], w2.state_pool[slot].astype(np.float32))
+
+
+def _tok(x):
+    """[K, N, ...] as drawn by the generator -> [N, K, ...] as the multi-token call takes it."""
+    return np.ascontiguousarray(np.swapaxes(x, 0, 1))
+
+
+def test_mixer_decode_tokens_without_checkpoints_matches_k_steps(kda):
+    import torch
+    w = I.make_mixer_decode(10, 4, 128, 4, 16, seed=I.SEED_BASE + 43)
+    sp, cp = to_device(w.state_pool, "f32"), to_device(w.conv_pool, "bf16")
+    out = kda.mixer_decode_tokens(to_device(_tok(w.q), "bf16"), to_device(_tok(w.k), "bf16"),
+                                  to_device(_tok(w.v), "bf16"), to_device(w.conv_w, "f32"),
+                                  to_device(_tok(w.log_alpha), "f32"), to_device(_tok(w.beta), "f32"),
+                                  to_device(_tok(w.gate), "bf16"), sp, cp, to_device(w.indices, "i32"))
+    torch.cuda.synchronize()
+    idx = w.indices
+    ro, rs, rh = O.kda_mixer_decode_tokens(_tok(w.q), _tok(w.k), _tok(w.v), w.conv_w, _tok(w.log_alpha),
+                                           _tok(w.beta), _tok(w.gate), w.state_pool[idx], w.conv_pool[idx])
+    assert_decode_out_close(to_host(out), ro, "K-token out")
+    assert_decode_state_close(to_host(sp)[idx], rs[:, -1], "state after K tokens")
+    np.testing.assert_array_equal(cp.view(torch.int16).cpu().numpy().view(np.uint16)[idx], I.bf16_bits(rh[:, -1]))
+
+
+def test_mixer_decode_tokens_checkpoints_and_commit(kda):
+    import torch
+    w = I.make_mixer_decode(6, 2, 128, 4, 9, seed=I.SEED_BASE + 44)
+    N, K, H = 6, 4, 2
+    sp, cp = to_device(w.state_pool, "f32"), to_device(w.conv_pool, "bf16")
+    idx = to_device(w.indices, "i32")
+    sck = torch.full((N, K, H, 128, 128), float("nan"), device="cuda")
+    cck = torch.zeros((N, K, H, 3, 3, 128), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(64, dtype=torch.int32, device="cuda")
+    out = kda.mixer_decode_tokens(to_device(_tok(w.q), "bf16"), to_device(_tok(w.k), "bf16"),
+                                  to_device(_tok(w.v), "bf16"), to_device(w.conv_w, "f32"),
+                                  to_device(_tok(w.log_alpha), "f32"), to_device(_tok(w.beta), "f32"),
+                                  to_device(_tok(w.gate), "bf16"), sp, cp, idx, state_ckpt=sck, conv_ckpt=cck,
+                                  status=status)
+    torch.cuda.synchronize()
+    # with checkpoints the pools stay as they were
+    np.testing.assert_array_equal(to_host(sp), w.state_pool.astype(np.float32))
+    ro, rs, rh = O.kda_mixer_decode_tokens(_tok(w.q), _tok(w.k), _tok(w.v), w.conv_w, _tok(w.log_alpha),
+                                           _tok(w.beta), _tok(w.gate), w.state_pool[w.indices],
+                                           w.conv_pool[w.indices])
+    assert_decode_out_close(to_host(out), ro, "K-token out")
+    assert_decode_state_close(to_host(sck), rs, "checkpoint states")
+    ck_bits = cck.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(ck_bits, I.bf16_bits(rh))
+    # commit: sequence n keeps accepted[n] tokens
+    accepted = np.array([0, 1, 4, 2, 3, 1], dtype=np.int32)
+    kda.mixer_decode_commit(sck, cck, to_device(accepted, "i32"), sp, cp, idx, status=status)
+    torch.cuda.synchronize()
+    assert int(to_host(status)[0]) == 0
+    got_s, got_h = to_host(sp), cp.view(torch.int16).cpu().numpy().view(np.uint16)
+    sck_h = to_host(sck)
+    for n, a in enumerate(accepted):
+        slot = w.indices[n]
+        if a == 0:
+            np.testing.assert_array_equal(got_s[slot], w.state_pool[slot].astype(np.float32))
+            np.testing.assert_array_equal(got_h[slot], I.bf16_bits(w.conv_pool[slot]))
+        else:
+            np.testing.assert_array_equal(got_s[slot], sck_h[n, a - 1])
+            np.testing.assert_array_equal(got_h[slot], ck_bits[n, a - 1])
+    unused = np.setdiff1d(np.arange(w.pool), w.indices)
+    np.testing.assert_array_equal(got_s[unused], w.state_pool[unused].astype(np.float32))
+
+
+def test_mixer_decode_one_token_call_is_the_decode_step(kda):
+    import torch
+    w = I.make_mixer_decode(5, 2, 128, 1, 5, seed=I.SEED_BASE + 45)
+    outs = []
+    for multi in (False, True):
+        sp, cp = to_device(w.state_pool, "f32"), to_device(w.conv_pool, "bf16")
+        args = [to_device(x, dt) for x, dt in ((w.q, "bf16"), (w.k, "bf16"), (w.v, "bf16"))]
+        if multi:
+            o = kda.mixer_decode_tokens(*[a.transpose(0, 1).contiguous() for a in args], to_device(w.conv_w, "f32"),
+                                        to_device(_tok(w.log_alpha), "f32"), to_device(_tok(w.beta), "f32"),
+                                        to_device(_tok(w.gate), "bf16"), sp, cp)[:, 0]
+        else:
+            o = kda.mixer_decode_step(*[a[0] for a in args], to_device(w.conv_w, "f32"),
+                                      to_device(w.log_alpha[0], "f32"), to_device(w.beta[0], "f32"),
+                                      to_device(w.gate[0], "bf16"), sp, cp)
+        torch.cuda.synchronize()
+        outs.append((to_host(o), to_host(sp)))
+    np.testing.assert_array_equal(outs[0][0], outs[1][0])
+    np.testing.assert_array_equal(outs[0][1], outs[1][1])

@@ -92,3 +92,10 @@ def test_mixer_decode_work_figure():
     # state r+w, conv history r+w (3 tensors x 3 rows, bf16), q/k/v/gate/out bf16, log_alpha, beta, index
     per_seq_head = 2 * 128 * 128 * 4 + 2 * 9 * 128 * 2 + 5 * 128 * 2 + 128 * 4 + 4
     assert bench.mixer_decode_bytes(256) == 256 * 32 * per_seq_head + 256 * 4
+
+
+def test_mixer_decode_tokens_work_figure():
+    import bench
+    assert bench.mixer_decode_tokens_bytes(256, 1) == bench.mixer_decode_bytes(256)
+    per_token = 5 * 128 * 2 + 128 * 4 + 4
+    assert bench.mixer_decode_tokens_bytes(256, 4) - bench.mixer_decode_tokens_bytes(256, 1) == 256 * 32 * 3 * per_token

@@ -360,3 +360,25 @@ def test_mixer_decode_step_with_history_matches_a_longer_prefill():
     o, S, _ = O.kda_mixer_decode_step(q[T:], k[T:], v[T:], w, la[T:], b[T:], g[T:], s_T, hist)
     np.testing.assert_allclose(o[0], o_long[T], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(S[0], s_long[0], rtol=1e-11, atol=1e-12)
+
+
+def test_mixer_decode_tokens_checkpoints_equal_shorter_runs():
+    """K tokens at once: the outputs are the single-step outputs, and checkpoint a-1 is
+    the state and history after decoding only the first a tokens (what a speculative
+    decoder rolls back to); the last checkpoint is the state after all K."""
+    rng = np.random.default_rng(137103)
+    N, K, H, d = 2, 4, 2, 8
+    mk = lambda *s: rng.standard_normal(s)
+    q, k, v, g = mk(N, K, H, d), mk(N, K, H, d), mk(N, K, H, d), mk(N, K, H, d)
+    la = -np.log1p(np.exp(mk(N, K, H, d))) / 4
+    b = 1 / (1 + np.exp(-mk(N, K, H)))
+    w = mk(3, H * d, 4) * 0.5
+    s0, h0 = mk(N, H, d, d) * 0.1, mk(N, H, 3, 3, d)
+    out, states, hists = O.kda_mixer_decode_tokens(q, k, v, w, la, b, g, s0, h0)
+    for a in range(1, K + 1):
+        S, hist = s0, h0
+        for j in range(a):
+            o, S, hist = O.kda_mixer_decode_step(q[:, j], k[:, j], v[:, j], w, la[:, j], b[:, j], g[:, j], S, hist)
+            np.testing.assert_allclose(out[:, j], o, rtol=0, atol=0)
+        np.testing.assert_allclose(states[:, a - 1], S, rtol=0, atol=0)
+        np.testing.assert_allclose(hists[:, a - 1], hist, rtol=0, atol=0)
