@@ -65,6 +65,7 @@ _SIGNATURES = {
     "kda_mixer_decode_tokens": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
                                        _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "kda_mixer_decode_commit": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "kda_state_affine": (_i32, [_vp, _vp, _vp, _vp, _i64, _i32, _vp]),
 }
 
 
@@ -252,6 +253,18 @@ def mixer_decode_commit(state_ckpt, conv_ckpt, accepted, state_pool, conv_pool, 
     _check(lib.kda_mixer_decode_commit(_ptr(state_ckpt), _ptr(conv_ckpt), _ptr(accepted), _ptr(state_pool),
                                        _ptr(conv_pool), _ptr(state_indices), state_pool.shape[0], N, K, H, d,
                                        _ptr(status), _stream(stream)))
+
+
+def state_affine(M, S=None, B=None, *, out=None, stream=None):
+    """out = M S + B over [..., 128, 128] fp32 matrices (kda_state_affine); S or B None = 0."""
+    torch = _torch()
+    lib = load_library()
+    d = M.shape[-1]
+    count = M.numel() // (d * d)
+    if out is None:
+        out = torch.empty_like(M)
+    _check(lib.kda_state_affine(_ptr(M), _ptr(S), _ptr(B), _ptr(out), count, d, _stream(stream)))
+    return out
 
 
 def workspace_status(workspace, stream=None) -> int:

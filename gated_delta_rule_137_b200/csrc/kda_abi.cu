@@ -303,6 +303,24 @@ kda_status kda_mixer_decode_commit(const float* state_ckpt, const void* conv_ckp
   if (e != cudaSuccess) return cuda_fail(e, "mixer decode commit kernel launch");
   return ok();
 }
+kda_status kda_state_affine(const float* M, const float* S, const float* B, float* out, int64_t count, int d,
+                            kda_stream_t stream_) {
+  if (count < 0) return fail(KDA_ERR_INVALID_ARG, "count=%lld must be >= 0", static_cast<long long>(count));
+  if (d != kda::kD) return fail(KDA_ERR_UNSUPPORTED, "kda_state_affine is built for d = 128 (got %d)", d);
+  if (count > (int64_t{1} << 31) - 1) return fail(KDA_ERR_INVALID_ARG, "count too large");
+  if (count == 0) return ok();
+  if (!M || !out) return fail(KDA_ERR_INVALID_ARG, "M and out must be non-NULL");
+  const void* ptrs[] = {M, S, B, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "M, S, B and out must be 16-byte aligned");
+  const size_t n = static_cast<size_t>(count) * d * d * sizeof(float);
+  if (ranges_overlap(out, n, M, n) || ranges_overlap(out, n, S, n))
+    return fail(KDA_ERR_INVALID_ARG, "out must not overlap M or S");
+  if (B && B != out && ranges_overlap(out, n, B, n)) return fail(KDA_ERR_INVALID_ARG, "out partially overlaps B");
+  cudaError_t e = kda::launch_state_affine(M, S, B, out, count, reinterpret_cast<cudaStream_t>(stream_));
+  if (e != cudaSuccess) return cuda_fail(e, "state affine kernel launch");
+  return ok();
+}
 size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv) {
   if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
   if (dk != kda::kD || dv != kda::kD) return 0;

@@ -1,0 +1,65 @@
+// kda_affine.cu — out[i] = M[i] S[i] + B[i] for a batch of 128 x 128 fp32 matrices.
+//
+// The KDA state after a stretch of tokens is affine in the state before it
+// (S_end = M S_start + B, M acting on the key rows): the recurrence of the
+// Ling-3.0-flash article, section "KDA: constant-size memory over a very long
+// context", multiplies the state by (I - b k k^T) Diag(a) on the left and adds
+// b k v^T. Composing such maps lets the segments of one long sequence be prefilled
+// in parallel (context parallelism): this kernel applies one map to a state.
+//
+// fp32 FMA on CUDA cores (the matrices are few and small: 2 MFLOP each). One CTA of
+// 256 threads per 32-row band of one output; thread t takes row t / 8 of the band
+// and 16 consecutive columns.
+#include <cuda_runtime.h>
+
+#include "kda_internal.h"
+
+namespace kda {
+
+namespace {
+
+constexpr int kAffD = 128;
+
+__global__ void __launch_bounds__(256) state_affine_kernel(const float* __restrict__ M, const float* __restrict__ S,
+                                                           const float* B, float* out) {
+  const size_t mat = static_cast<size_t>(blockIdx.x) * kAffD * kAffD;
+  const int row = blockIdx.y * 32 + (threadIdx.x >> 3);
+  const int c0 = (threadIdx.x & 7) * 16;
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; e += 4) {
+    const float4 b = B ? *reinterpret_cast<const float4*>(B + mat + static_cast<size_t>(row) * kAffD + c0 + e)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    acc[e] = b.x; acc[e + 1] = b.y; acc[e + 2] = b.z; acc[e + 3] = b.w;
+  }
+  if (S) {
+    const float* Mr = M + mat + static_cast<size_t>(row) * kAffD;
+    const float* Sm = S + mat + c0;
+    for (int k = 0; k < kAffD; ++k) {
+      const float m = __ldg(Mr + k);
+#pragma unroll
+      for (int e = 0; e < 16; e += 4) {
+        const float4 s = __ldg(reinterpret_cast<const float4*>(Sm + static_cast<size_t>(k) * kAffD + e));
+        acc[e] = fmaf(m, s.x, acc[e]);
+        acc[e + 1] = fmaf(m, s.y, acc[e + 1]);
+        acc[e + 2] = fmaf(m, s.z, acc[e + 2]);
+        acc[e + 3] = fmaf(m, s.w, acc[e + 3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 16; e += 4)
+    *reinterpret_cast<float4*>(out + mat + static_cast<size_t>(row) * kAffD + c0 + e) =
+        make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+}
+
+}  // namespace
+
+cudaError_t launch_state_affine(const float* M, const float* S, const float* B, float* out, int64_t count,
+                                cudaStream_t stream) {
+  if (count == 0) return cudaSuccess;
+  state_affine_kernel<<<dim3(static_cast<unsigned>(count), kAffD / 32), 256, 0, stream>>>(M, S, B, out);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

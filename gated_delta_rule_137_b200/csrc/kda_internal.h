@@ -90,6 +90,10 @@ cudaError_t launch_mixer_decode_commit(const float* state_ckpt, const void* conv
                                        float* state_pool, void* conv_pool, const int32_t* state_indices,
                                        int pool_size, int N, int K, int H, uint32_t* status, cudaStream_t stream);
 
+// out[i] = M[i] S[i] + B[i] for `count` 128 x 128 fp32 matrices (S, B may be null: zero).
+cudaError_t launch_state_affine(const float* M, const float* S, const float* B, float* out, int64_t count,
+                                cudaStream_t stream);
+
 // Tensor-core chunked prefill on d = 128 operands (bf16 or fp32 q/k/v/out).
 cudaError_t launch_prefill_d128(const PrefillArgs& a, cudaStream_t stream);
 

@@ -219,6 +219,22 @@ KDA_API kda_status kda_mixer_decode_commit(const float* state_ckpt, const void* 
                                    const int32_t* state_indices, int pool_size, int N, int K, int H, int d,
                                    void* status, kda_stream_t stream);
 
+/*
+ * Affine map of states: out[i] = M[i] S[i] + B[i] for `count` d x d fp32 matrices
+ * (row-major, M acting on the key rows). The state after a stretch of tokens is
+ * affine in the state before it (same KDA section): S_end = M S_start + B, where M
+ * is the stretch's final state from the identity with zero values and B its final
+ * state from zero. Composing the maps of consecutive segments gives each segment
+ * its starting state, which lets one long sequence be prefilled in parallel across
+ * devices (context parallelism; see gated_delta_rule_137_b200.context_parallel).
+ *   M      device fp32 [count, d, d]
+ *   S, B   device fp32 [count, d, d] or NULL (zero)
+ *   out    device fp32 [count, d, d]; may be B (in-place add), not M or S
+ * d must be 128; pointers 16-byte aligned.
+ */
+KDA_API kda_status kda_state_affine(const float* M, const float* S, const float* B, float* out, int64_t count,
+                            int d, kda_stream_t stream);
+
 /* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes): the
  * status word plus the two-pass prefill's scratch, sized as for kda_chunk_fwd (the
  * conv/L2 stage runs inside the prefill's first pass and needs no buffer of its own). */

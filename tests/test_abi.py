@@ -177,3 +177,12 @@ def test_mixer_decode_tokens_and_commit_reject_bad_arguments(lib):
     assert lib.kda_mixer_decode_commit(*bad) == kda.KDA_ERR_INVALID_ARG
     bad = list(cbase); bad[10] = 64                 # d != 128
     assert lib.kda_mixer_decode_commit(*bad) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_state_affine_rejects_bad_arguments(lib):
+    assert lib.kda_state_affine(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, 2, 64, None) == kda.KDA_ERR_UNSUPPORTED
+    assert lib.kda_state_affine(None, FAKE * 2, FAKE * 3, FAKE * 4, 2, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_state_affine(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, -1, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_state_affine(FAKE, FAKE * 2, FAKE * 3, FAKE + 8, 2, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_state_affine(FAKE, FAKE * 2, None, FAKE * 2, 2, 128, None) == kda.KDA_ERR_INVALID_ARG  # out is S
+    assert lib.kda_state_affine(FAKE, None, None, FAKE * 4, 0, 128, None) == kda.KDA_OK  # nothing to do

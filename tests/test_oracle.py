@@ -382,3 +382,21 @@ def test_mixer_decode_tokens_checkpoints_equal_shorter_runs():
             np.testing.assert_allclose(out[:, j], o, rtol=0, atol=0)
         np.testing.assert_allclose(states[:, a - 1], S, rtol=0, atol=0)
         np.testing.assert_allclose(hists[:, a - 1], hist, rtol=0, atol=0)
+
+
+def test_final_state_is_affine_in_the_initial_state():
+    """S_end(S0) = M S0 + B with M the run from the identity with zero values and B the
+    run from zero: the fact a context-parallel prefill builds on (checked on random S0)."""
+    rng = np.random.default_rng(137104)
+    T, H, d = 40, 2, 8
+    q, k, v = (rng.standard_normal((T, H, d)) for _ in range(3))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    la = -np.log1p(np.exp(rng.standard_normal((T, H, d)))) / 8
+    b = 1 / (1 + np.exp(-rng.standard_normal((T, H))))
+    cu = np.array([0, T])
+    eye = np.broadcast_to(np.eye(d), (1, H, d, d)).copy()
+    _, M = O.kda_recurrence(q, k, np.zeros_like(v), la, b, eye, cu)
+    _, B = O.kda_recurrence(q, k, v, la, b, None, cu)
+    S0 = rng.standard_normal((1, H, d, d))
+    _, S = O.kda_recurrence(q, k, v, la, b, S0, cu)
+    np.testing.assert_allclose(S, M @ S0 + B, rtol=1e-11, atol=1e-12)
