@@ -471,6 +471,46 @@ def run_gpu(args):
                          "algorithmic_bytes_per_launch": kbytes}}
         del sp, cp, mtoks, ktok
 
+    # ---------------- context-parallel prefill, its pieces timed on one GPU ---------------
+    cpar = None
+    if not args.quick:
+        from gated_delta_rule_137_b200 import context_parallel as cpm
+        segs, Tc = 4, 4 * T1
+        ci = device_prefill_inputs(Tc, H, D, 1370006, device, state_N=1)
+        cargs = [ci[k] for k in ("q", "k", "v", "log_alpha", "beta")]
+        seg_of = lambda x, i: x[i * T1:(i + 1) * T1].contiguous()
+        last = [seg_of(x, segs - 1) for x in cargs]
+        maps = [cpm.segment_map(*[seg_of(x, i) for x in cargs], N=1) for i in range(segs)]
+
+        def timed(fn, n=5):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            return e0.elapsed_time(e1) / n
+
+        S_last = cpm.start_state(maps, segs - 1, ci["initial_state"])
+        t_map = timed(lambda: cpm.segment_map(*last, N=1))
+        t_fold = timed(lambda: cpm.start_state(maps, segs - 1, ci["initial_state"]))
+        t_final = timed(lambda: kda.chunk_fwd(*last, S_last, None, N=1))
+        t_emul = timed(lambda: cpm.context_parallel_emulate(*cargs, ci["initial_state"], N=1, segments=segs), 3)
+        t_plain = timed(lambda: kda.chunk_fwd(*cargs, ci["initial_state"], None, N=1), 3)
+        # timed calls x kernels: maps 5 x 2 prefills x 3, fold 5 x 3 affine, segment prefill 5 x 3,
+        # emulation 3 x (4 maps x 6 + 4 prefills x 3 + 6 affine), plain prefill 3 x 3
+        launches += 5 * 6 + 5 * 3 + 5 * 3 + 3 * (4 * 6 + 4 * 3 + 6) + 3 * 3
+        cpar = {"workload": f"context-parallel prefill of one {Tc}-token sequence (H={H} d={D}) in {segs} segments; "
+                            "pieces timed on one GPU with CUDA events (the exchange is not part of it)",
+                "segment_map_ms": t_map, "fold_ms": t_fold, "segment_prefill_ms": t_final,
+                "per_rank_path_ms": t_map + t_fold + t_final,
+                "emulated_on_one_gpu_ms": t_emul, "plain_prefill_ms": t_plain,
+                "exchange_bytes_per_rank": 2 * H * D * D * 4}
+        del ci, cargs, maps, last
+
     # ---------------- full mixer (conv4 + L2 + KDA + gate), B=2 x T=32768 ----------------
     mix = None
     if not args.quick:
@@ -547,7 +587,7 @@ def run_gpu(args):
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "pipelining": "2 device buffer sets; upload, kernels and download of consecutive steps overlap "
                                   "on three streams; every step's copies are inside the timed region"},
-            "decode": decode, "mixer_decode": mdec, "mixer": mix, "varlen": var,
+            "decode": decode, "mixer_decode": mdec, "context_parallel": cpar, "mixer": mix, "varlen": var,
             "clocks": clocks, "gpu_launches": launches, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -8,8 +8,8 @@
 // in parallel (context parallelism): this kernel applies one map to a state.
 //
 // fp32 FMA on CUDA cores (the matrices are few and small: 2 MFLOP each). One CTA of
-// 256 threads per 32-row band of one output; thread t takes row t / 8 of the band
-// and 16 consecutive columns.
+// 256 threads per 32-row band of one output stages S in shared memory; thread t takes
+// row t / 8 of the band and 16 consecutive columns.
 #include <cuda_runtime.h>
 
 #include "kda_internal.h"
@@ -22,6 +22,7 @@ constexpr int kAffD = 128;
 
 __global__ void __launch_bounds__(256) state_affine_kernel(const float* __restrict__ M, const float* __restrict__ S,
                                                            const float* B, float* out) {
+  extern __shared__ float4 s_S4[];  // S of this matrix, [128][128] fp32 (64 KB)
   const size_t mat = static_cast<size_t>(blockIdx.x) * kAffD * kAffD;
   const int row = blockIdx.y * 32 + (threadIdx.x >> 3);
   const int c0 = (threadIdx.x & 7) * 16;
@@ -33,17 +34,24 @@ __global__ void __launch_bounds__(256) state_affine_kernel(const float* __restri
     acc[e] = b.x; acc[e + 1] = b.y; acc[e + 2] = b.z; acc[e + 3] = b.w;
   }
   if (S) {
+    const float4* Sg = reinterpret_cast<const float4*>(S + mat);
+    for (int e = threadIdx.x; e < kAffD * kAffD / 4; e += blockDim.x) s_S4[e] = __ldg(Sg + e);
+    __syncthreads();
+    const float* s_S = reinterpret_cast<const float*>(s_S4);
     const float* Mr = M + mat + static_cast<size_t>(row) * kAffD;
-    const float* Sm = S + mat + c0;
-    for (int k = 0; k < kAffD; ++k) {
-      const float m = __ldg(Mr + k);
+    for (int k = 0; k < kAffD; k += 4) {
+      const float4 m4 = __ldg(reinterpret_cast<const float4*>(Mr + k));
+      const float mk[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-      for (int e = 0; e < 16; e += 4) {
-        const float4 s = __ldg(reinterpret_cast<const float4*>(Sm + static_cast<size_t>(k) * kAffD + e));
-        acc[e] = fmaf(m, s.x, acc[e]);
-        acc[e + 1] = fmaf(m, s.y, acc[e + 1]);
-        acc[e + 2] = fmaf(m, s.z, acc[e + 2]);
-        acc[e + 3] = fmaf(m, s.w, acc[e + 3]);
+      for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 sv = *reinterpret_cast<const float4*>(s_S + (k + kk) * kAffD + c0 + e);
+          acc[e] = fmaf(mk[kk], sv.x, acc[e]);
+          acc[e + 1] = fmaf(mk[kk], sv.y, acc[e + 1]);
+          acc[e + 2] = fmaf(mk[kk], sv.z, acc[e + 2]);
+          acc[e + 3] = fmaf(mk[kk], sv.w, acc[e + 3]);
+        }
       }
     }
   }
@@ -58,7 +66,10 @@ __global__ void __launch_bounds__(256) state_affine_kernel(const float* __restri
 cudaError_t launch_state_affine(const float* M, const float* S, const float* B, float* out, int64_t count,
                                 cudaStream_t stream) {
   if (count == 0) return cudaSuccess;
-  state_affine_kernel<<<dim3(static_cast<unsigned>(count), kAffD / 32), 256, 0, stream>>>(M, S, B, out);
+  constexpr int kSmem = kAffD * kAffD * 4;
+  static cudaError_t attr = cudaFuncSetAttribute(state_affine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (attr != cudaSuccess) return attr;
+  state_affine_kernel<<<dim3(static_cast<unsigned>(count), kAffD / 32), 256, S ? kSmem : 0, stream>>>(M, S, B, out);
   return cudaGetLastError();
 }
 
