@@ -35,6 +35,10 @@ What it computes (all in float64, from the exact input values upcast):
   same conv4 / L2 norm / recurrence / gate steps as ``kda_mixer`` applied to one
   new token, with the convolution's last three raw inputs kept per sequence (a
   conv history) instead of the whole sequence.
+* ``gate_log_alpha`` — the decay gate made from its pre-activation, read from
+  the article's "softplus" gate as log alpha = -scale_h * softplus(a) per channel
+  with one positive scale per head (the pages name the softplus, not its
+  parameters).
 * ``kda_mixer_decode_tokens`` — K consecutive tokens per sequence through
   ``kda_mixer_decode_step``, keeping the state and history after every token (the
   checkpoints a speculative decoder rolls back to when it accepts fewer tokens).
@@ -290,3 +294,13 @@ def kda_mixer_decode_tokens(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, 
         states.append(S)
         hists.append(hist)
     return np.stack(outs, axis=1), np.stack(states, axis=1), np.stack(hists, axis=1)
+
+
+def softplus(x) -> np.ndarray:
+    """log(1 + e^x), evaluated without overflow."""
+    return np.logaddexp(0.0, _f64(x))
+
+
+def gate_log_alpha(a_pre, a_scale) -> np.ndarray:
+    """log alpha [.., H, d] = -a_scale[h] * softplus(a_pre) (a_scale [H] > 0)."""
+    return -_f64(a_scale)[:, None] * softplus(a_pre)

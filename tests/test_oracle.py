@@ -400,3 +400,18 @@ def test_final_state_is_affine_in_the_initial_state():
     S0 = rng.standard_normal((1, H, d, d))
     _, S = O.kda_recurrence(q, k, v, la, b, S0, cu)
     np.testing.assert_allclose(S, M @ S0 + B, rtol=1e-11, atol=1e-12)
+
+
+def test_softplus_gate_closed_forms():
+    # softplus(0) = ln 2; large x -> x; very negative x -> e^x; -softplus <= 0 always
+    assert O.softplus(0.0) == pytest.approx(np.log(2.0), rel=1e-15)
+    assert O.softplus(50.0) == pytest.approx(50.0, rel=1e-15)
+    assert O.softplus(-40.0) == pytest.approx(np.exp(-40.0), rel=1e-12)
+    x = np.linspace(-30, 30, 601)
+    np.testing.assert_allclose(O.softplus(x), np.log1p(np.exp(x)), rtol=1e-12)
+    a = np.random.default_rng(137105).standard_normal((5, 3, 4))
+    s = np.array([0.5, 1.0, 2.0])
+    la = O.gate_log_alpha(a, s)
+    assert np.all(la < 0)
+    np.testing.assert_allclose(la[:, 1], -np.log1p(np.exp(a[:, 1])), rtol=1e-12)   # scale 1
+    np.testing.assert_allclose(la[:, 2], -2 * np.log1p(np.exp(a[:, 2])), rtol=1e-12)  # linear in the scale
