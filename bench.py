@@ -534,7 +534,27 @@ def run_gpu(args):
                "ms_per_call": mtot / msteps, "tokens_per_s": job_throughput(Bm * Tm * msteps, world, mtot / 1e3),
                "roofline": {"bound": "hbm", "achieved": mbytes / (mms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                             "frac": mbytes / (mms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_launch": mbytes}}
-        del mi, mo, mws
+        # the same mixer with the decay gate made on the device from its bf16 pre-activation
+        a_pre = torch.randn(Bm * Tm, H, D, generator=torch.Generator(device=device).manual_seed(1370007),
+                            device=device).bfloat16()
+        a_scale = torch.full((H,), 1 / 16, device=device)
+        gws = torch.empty(lib.kda_mixer_fwd_gate_workspace(Bm * Tm, Bm, H, D, D), dtype=torch.uint8, device=device)
+
+        def gstep(i):
+            kda.mixer_fwd_gate(mi["q"], mi["k"], mi["v"], mi["conv_w"], a_pre, a_scale, mi["beta"], mi["gate"], None,
+                               None, N=Bm, out=mo, final_state=mf, workspace=gws, stream=stream)
+
+        gper, gtot = time_region(gstep, msteps, 2, stream, device)
+        launches += 3 * msteps
+        gtot = max_over_ranks(gtot, device)
+        gbytes = mbytes - Bm * Tm * H * D * 2  # log_alpha fp32 -> a_pre bf16
+        gms = statistics.mean(gper)
+        mix["gate_from_preactivation"] = {
+            "workload": "same mixer, log_alpha = -scale_h softplus(a) made on the device from bf16 a",
+            "ms_per_call": gtot / msteps, "tokens_per_s": job_throughput(Bm * Tm * msteps, world, gtot / 1e3),
+            "roofline": {"bound": "hbm", "achieved": gbytes / (gms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbytes / (gms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_launch": gbytes}}
+        del mi, mo, mws, a_pre, gws
 
     # ---------------- varlen packed prefill, 64 sequences U[256, 8192] ------------------
     var = None

@@ -66,6 +66,9 @@ _SIGNATURES = {
                                        _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "kda_mixer_decode_commit": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "kda_state_affine": (_i32, [_vp, _vp, _vp, _vp, _i64, _i32, _vp]),
+    "kda_mixer_fwd_gate_workspace": (_sz, [_i64, _i32, _i32, _i32, _i32]),
+    "kda_mixer_fwd_gate": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
+                                  _vp, _vp, _vp, _sz, _vp]),
 }
 
 
@@ -265,6 +268,34 @@ def state_affine(M, S=None, B=None, *, out=None, stream=None):
         out = torch.empty_like(M)
     _check(lib.kda_state_affine(_ptr(M), _ptr(S), _ptr(B), _ptr(out), count, d, _stream(stream)))
     return out
+
+
+def mixer_fwd_gate(q_raw, k_raw, v_raw, conv_w, a_pre, a_scale, beta, gate=None, initial_state=None,
+                   cu_seqlens=None, *, N: Optional[int] = None, out=None, final_state=None,
+                   output_final_state: bool = True, workspace=None, stream=None, check_status: bool = False):
+    """Full mixer prefill with log_alpha = -a_scale[h] * softplus(a_pre) made on the
+    device (kda_mixer_fwd_gate); a_pre bf16 [T, H, 128], a_scale fp32 [H]."""
+    torch = _torch()
+    lib = load_library()
+    total_T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    if N is None:
+        if cu_seqlens is None:
+            raise ValueError("N is needed when cu_seqlens is not given")
+        N = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((total_T, H, dv), dtype=torch.bfloat16, device=q_raw.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q_raw.device)
+    need = int(lib.kda_mixer_fwd_gate_workspace(total_T, N, H, dk, dv))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q_raw.device)
+    _check(lib.kda_mixer_fwd_gate(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w), _ptr(a_pre), _ptr(a_scale),
+                                  _ptr(beta), _ptr(gate), _ptr(initial_state), _ptr(cu_seqlens), total_T, N, H, dk, dv,
+                                  _ptr(out), _ptr(final_state), _ptr(workspace), workspace.numel(), _stream(stream)))
+    if check_status:
+        workspace_status(workspace, stream)
+    return out, final_state
 
 
 def workspace_status(workspace, stream=None) -> int:

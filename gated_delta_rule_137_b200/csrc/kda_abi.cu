@@ -389,6 +389,47 @@ kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   return ok();
 }
 
+size_t kda_mixer_fwd_gate_workspace(int64_t total_T, int N, int H, int dk, int dv) {
+  if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
+  if (dk != kda::kD || dv != kda::kD) return 0;
+  if (total_T == 0 || N == 0) return kda::kStatusBytes;
+  const size_t split = kda::split_workspace_bytes(total_T, N, H, /*any_chains=*/true);
+  return split ? kda::kStatusBytes + split : 0;
+}
+kda_status kda_mixer_fwd_gate(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                              const void* a_pre, const float* a_scale, const float* beta, const void* gate,
+                              const float* initial_state, const int32_t* cu_seqlens, int64_t total_T, int N, int H,
+                              int dk, int dv, void* out, float* final_state, void* workspace, size_t workspace_bytes,
+                              kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  // a_pre stands where log_alpha stands in the shared checks (same shape, 16-byte aligned)
+  kda_status st = check_mixer(q_raw, k_raw, v_raw, conv_w, static_cast<const float*>(a_pre), beta, gate,
+                              initial_state, cu_seqlens, total_T, N, H, dk, dv, out, final_state);
+  if (st != KDA_OK) return st;
+  if (total_T > 0 && !a_scale) return fail(KDA_ERR_INVALID_ARG, "a_scale must be non-NULL");
+  if (a_scale && (reinterpret_cast<uintptr_t>(a_scale) & 3u)) return fail(KDA_ERR_INVALID_ARG, "a_scale is not 4-byte aligned");
+  if (N == 0) return ok();
+  if (workspace && !aligned16(workspace)) return fail(KDA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  const size_t need = kda_mixer_fwd_gate_workspace(total_T, N, H, dk, dv);
+  if (need == 0) return fail(KDA_ERR_UNSUPPORTED, "the two-pass scratch for these sizes exceeds the supported 32 GiB");
+  if (!workspace || workspace_bytes < need)
+    return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? workspace_bytes : 0, need);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  kda::PrefillArgs a{};
+  a.q = q_raw; a.k = k_raw; a.v = v_raw; a.log_alpha = nullptr; a.beta = beta; a.h0 = initial_state;
+  a.cu = cu_seqlens; a.gate = gate; a.conv_w = conv_w; a.out = out; a.ht = final_state; a.status = status;
+  a.total_T = total_T; a.N = N; a.H = H;
+  a.in_f32 = false;
+  a.out_f32 = false;
+  a.a_pre = a_pre;
+  a.a_scale = a_scale;
+  if (total_T > 0) a.split_ws = static_cast<char*>(workspace) + kda::kStatusBytes;
+  e = kda::launch_prefill_d128(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+  return ok();
+}
 kda_status kda_workspace_status(void* workspace, kda_stream_t stream_, uint32_t* flags) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!workspace) return fail(KDA_ERR_INVALID_ARG, "workspace is NULL");

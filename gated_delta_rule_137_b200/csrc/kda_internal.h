@@ -43,6 +43,9 @@ struct PrefillArgs {
   bool out_f32;           // out is fp32 (else bf16)
   void* split_ws;         // split_workspace_bytes() of scratch for the two-pass prefill, or
                           // null for the single-pass kernel
+  const void* a_pre;      // bf16 [total_T, H, 128] or null: the decay gate's pre-activation, with
+  const float* a_scale;   // fp32 [H]: log_alpha = -a_scale[h] * softplus(a_pre) (log_alpha null);
+                          // two-pass full mixer only
 };
 
 // ---- two-pass prefill (kda_split.cu) ---------------------------------------------------
@@ -64,9 +67,9 @@ inline int64_t split_max_chunks(int64_t total_T, int N) {
 }
 inline size_t split_plan_bytes(int N) { return align256((static_cast<size_t>(N) + 1) * sizeof(int32_t)); }
 constexpr int64_t kSplitMaxChains = 74;  // half of the 148 SMs: beyond it no slicing is needed
-inline size_t split_workspace_bytes(int64_t total_T, int N, int H) {
+inline size_t split_workspace_bytes(int64_t total_T, int N, int H, bool any_chains = false) {
   if (total_T <= 0 || N <= 0) return 0;
-  if (static_cast<int64_t>(N) * H > kSplitMaxChains) return 0;
+  if (!any_chains && static_cast<int64_t>(N) * H > kSplitMaxChains) return 0;
   const size_t items = static_cast<size_t>(split_max_chunks(total_T, N)) * static_cast<size_t>(H) * kItemBytes;
   if (items > kSplitMaxItemBytes) return 0;
   return split_plan_bytes(N) + items;

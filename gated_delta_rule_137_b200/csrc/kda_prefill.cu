@@ -676,6 +676,7 @@ cudaError_t launch_prefill_d128(const PrefillArgs& a, cudaStream_t stream) {
     return cudaGetLastError();
   }
   if (a.split_ws) return launch_prefill_split(a, stream);
+  if (a.a_pre) return cudaErrorInvalidValue;  // the pre-activation gate has only the two-pass form
   if (a.conv_w) {  // the fused full mixer: raw bf16 q/k/v, bf16 out
     if (a.in_f32 || a.out_f32) return cudaErrorInvalidValue;
     return launch_types<__nv_bfloat16, __nv_bfloat16, true>(a, stream);

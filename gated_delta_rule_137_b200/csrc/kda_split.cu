@@ -189,7 +189,9 @@ __device__ __forceinline__ ItemPos item_pos(int64_t it, const PrefillArgs& a, co
 // kConv: q, k, v are the raw inputs of the full mixer; the causal depthwise conv of
 // width 4 (zero history at each sequence start) is applied to all three and the L2
 // norm x / sqrt(sum x^2 + 1e-6) to q and k, in fp32, before anything else.
-template <typename TIn, bool kConv>
+// kPre: the decay gate arrives as its bf16 pre-activation and a per-head scale,
+// log_alpha = -a_scale[h] * softplus(a_pre), made here as it is loaded.
+template <typename TIn, bool kConv, bool kPre = false>
 __global__ void __launch_bounds__(kIntraThreads, 1)
     kda_intra_kernel(const PrefillArgs a, const SplitPlan p) {
   using SM = IntraSmem;
@@ -260,7 +262,10 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         if (r < nx.len) {
           const size_t o = static_cast<size_t>(nx.t0 + r) * tok_stride + static_cast<size_t>(nx.h) * kD;
           constexpr int kLine = 128 / sizeof(TIn);  // elements per 128-B line
-          prefetch_l2(a.log_alpha + o + part * 32);
+          if constexpr (kPre)
+            prefetch_l2(static_cast<const __nv_bfloat16*>(a.a_pre) + o + (part & 1) * 64);
+          else
+            prefetch_l2(a.log_alpha + o + part * 32);
           prefetch_l2((part < 2 ? kg : qg) + o + (part & 1) * kLine);
           prefetch_l2(vg + o + (part & 1) * kLine + (part >> 1) * (sizeof(TIn) == 4 ? 2 * kLine : 0));
         }
@@ -306,9 +311,19 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         for (int i = 0; i < 4; ++i) {
           const bool in = r0 + i < len;
           const size_t o = static_cast<size_t>(t0 + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
-          const float4 l4 = __ldg(reinterpret_cast<const float4*>(a.log_alpha + o));
-          la[s][i][0] = in ? l4.x : 0.f; la[s][i][1] = in ? l4.y : 0.f;
-          la[s][i][2] = in ? l4.z : 0.f; la[s][i][3] = in ? l4.w : 0.f;
+          if constexpr (kPre) {
+            // log alpha = -scale * softplus(x), softplus(x) = max(x, 0) + log1p(e^-|x|)
+            const float sc = __ldg(a.a_scale + h);
+            float x[4];
+            ld4_in(static_cast<const __nv_bfloat16*>(a.a_pre) + o, x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              la[s][i][e] = in ? -sc * (fmaxf(x[e], 0.f) + log1pf(__expf(-fabsf(x[e])))) : 0.f;
+          } else {
+            const float4 l4 = __ldg(reinterpret_cast<const float4*>(a.log_alpha + o));
+            la[s][i][0] = in ? l4.x : 0.f; la[s][i][1] = in ? l4.y : 0.f;
+            la[s][i][2] = in ? l4.z : 0.f; la[s][i][3] = in ? l4.w : 0.f;
+          }
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -1038,9 +1053,9 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
 }
 
 // ================================ host =================================================
-template <typename TIn, bool kConv>
+template <typename TIn, bool kConv, bool kPre = false>
 cudaError_t launch_intra(const PrefillArgs& a, const SplitPlan& p, int64_t max_chunks, cudaStream_t stream) {
-  auto kern = kda_intra_kernel<TIn, kConv>;
+  auto kern = kda_intra_kernel<TIn, kConv, kPre>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -1075,11 +1090,11 @@ cudaError_t launch_recur_dv(const PrefillArgs& a, const SplitPlan& p, cudaStream
 template <typename TOut>
 cudaError_t launch_recur(const PrefillArgs& a, const SplitPlan& p, cudaStream_t stream) {
   // value-column slices per chain: as many as a single wave of CTAs over the 148 SMs
-  // allows (one CTA per SM); the two-pass form is only chosen for <= 74 chains
+  // allows (one CTA per SM); beyond 74 chains (only the gate-from-pre-activation mixer
+  // takes the two passes there) 64-column slices in several waves
   const int64_t chains = static_cast<int64_t>(a.N) * a.H;
   if (4 * chains <= 148) return launch_recur_dv<32, TOut>(a, p, stream);
-  if (chains <= kSplitMaxChains) return launch_recur_dv<64, TOut>(a, p, stream);
-  return cudaErrorInvalidValue;
+  return launch_recur_dv<64, TOut>(a, p, stream);  // more than 74 chains: several waves
 }
 
 }  // namespace
@@ -1091,7 +1106,10 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t max_chunks = split_max_chunks(a.total_T, a.N);
-  if (a.conv_w) {
+  if (a.a_pre) {  // the full mixer with the decay gate made from its pre-activation
+    if (!a.conv_w || !a.a_scale || a.in_f32 || a.out_f32) return cudaErrorInvalidValue;
+    e = launch_intra<__nv_bfloat16, true, true>(a, p, max_chunks, stream);
+  } else if (a.conv_w) {
     if (a.in_f32 || a.out_f32) return cudaErrorInvalidValue;
     e = launch_intra<__nv_bfloat16, true>(a, p, max_chunks, stream);
   } else {

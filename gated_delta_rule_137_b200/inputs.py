@@ -194,6 +194,16 @@ def make_decode(N, H, dk, dv, steps, *, seed, state_std=0.02, name="decode") -> 
                           q=q, k=k, v=v, log_alpha=la, beta=beta, state=st)
 
 
+def make_gate_preactivation(total_T, H, d, *, seed):
+    """The decay gate as its pre-activation: a ~ N(0, 1) rounded to bf16 [total_T, H, d],
+    and one scale per head drawn uniformly from [1/32, 1/8] (fp32 [H])."""
+    rng = np.random.default_rng(seed)
+    a = _normal(rng, (total_T, H, d))
+    _bf16_round_inplace(a)
+    scale = rng.uniform(1 / 32, 1 / 8, H).astype(np.float64)
+    return a, scale
+
+
 @dataclasses.dataclass
 class MixerDecodeWorkload:
     """Serving decode of the full mixer: `steps` tokens for N sequences whose states and

@@ -263,6 +263,24 @@ KDA_API kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const voi
                          void* workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * Full mixer prefill with the decay gate made from its pre-activation (the article's
+ * KDA panel names a softplus for the gate; the form read here is one positive scale
+ * per head): log_alpha = -a_scale[h] * softplus(a_pre), computed in fp32 as the
+ * pre-activation is read, so the gate costs 2 bytes per channel instead of 4.
+ * Arguments as kda_mixer_fwd, with log_alpha replaced by
+ *   a_pre    device bf16 [total_T, H, dk]
+ *   a_scale  device fp32 [H], > 0
+ * and the workspace sized by kda_mixer_fwd_gate_workspace (this entry point always
+ * runs the two-pass prefill; 0 from the query means the sizes are too large for it).
+ */
+KDA_API size_t kda_mixer_fwd_gate_workspace(int64_t total_T, int N, int H, int dk, int dv);
+KDA_API kda_status kda_mixer_fwd_gate(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                              const void* a_pre, const float* a_scale, const float* beta, const void* gate,
+                              const float* initial_state, const int32_t* cu_seqlens, int64_t total_T,
+                              int N, int H, int dk, int dv, void* out, float* final_state,
+                              void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * Full mixer prefill without a workspace, for callers that cannot allocate device
  * memory where they run the mixer (a plugin whose host framework owns every device
  * allocation, a serving loop that may not call cudaMalloc). The paper has no

@@ -307,3 +307,21 @@ def test_mixer_full_size_sampled_heads(kda):
     ro, rf = _mixer_oracle_heads(w, heads)
     assert_prefill_close(out[:, heads], ro, "mixer out", stored_bf16=True)
     assert_prefill_close(fin[:, heads], rf, "mixer final")
+
+
+@pytest.mark.parametrize("lens,H", [([300, 77], 4), ([70] * 40, 2)])  # 8 chains; 80 chains (several waves)
+def test_mixer_gate_from_preactivation(kda, lens, H):
+    """kda_mixer_fwd_gate: log_alpha = -a_scale[h] softplus(a_pre) made on the device."""
+    import torch
+    w = I.make_prefill(lens, H, 128, 128, seed=sum(lens) + H + 7, normalise_qk=False, mixer=True)
+    a_pre, a_scale = I.make_gate_preactivation(w.q.shape[0], H, 128, seed=sum(lens) + 8)
+    dt = "bf16"
+    out, fin = kda.mixer_fwd_gate(to_device(w.q, dt), to_device(w.k, dt), to_device(w.v, dt),
+                                  to_device(w.conv_w, "f32"), to_device(a_pre, "bf16"), to_device(a_scale, "f32"),
+                                  to_device(w.beta, "f32"), to_device(w.gate, dt), to_device(w.initial_state, "f32"),
+                                  to_device(w.cu_seqlens, "i32"), N=w.N, check_status=True)
+    torch.cuda.synchronize()
+    la = O.gate_log_alpha(a_pre, a_scale)
+    ro, rf = O.kda_mixer(w.q, w.k, w.v, w.conv_w, la, w.beta, w.gate, w.cu_seqlens, w.initial_state)
+    assert_prefill_close(to_host(out), ro, "gate-from-pre-activation mixer out", stored_bf16=True)
+    assert_prefill_close(to_host(fin), rf, "gate-from-pre-activation mixer final state")
