@@ -35,6 +35,9 @@ What it computes (all in float64, from the exact input values upcast):
   same conv4 / L2 norm / recurrence / gate steps as ``kda_mixer`` applied to one
   new token, with the convolution's last three raw inputs kept per sequence (a
   conv history) instead of the whole sequence.
+* ``kda_backward`` — the gradients of ``kda_recurrence`` (of q, k, v, log_alpha,
+  beta and the initial state, given the gradients of the outputs and of the final
+  state): the chain rule through each token step, taken in reverse order.
 * ``gate_log_alpha`` — the decay gate made from its pre-activation, read from
   the article's "softplus" gate as log alpha = -scale_h * softplus(a) per channel
   with one positive scale per head (the pages name the softplus, not its
@@ -304,3 +307,52 @@ def softplus(x) -> np.ndarray:
 def gate_log_alpha(a_pre, a_scale) -> np.ndarray:
     """log alpha [.., H, d] = -a_scale[h] * softplus(a_pre) (a_scale [H] > 0)."""
     return -_f64(a_scale)[:, None] * softplus(a_pre)
+
+
+def kda_backward(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_out, d_final=None):
+    """Gradients of kda_recurrence over packed sequences.
+
+    One token step, written with P = Diag(alpha) S_prev, w = P^T k, u = beta (v - w):
+        S = P + k u^T,  o = S^T q.
+    Walking the tokens backwards with G the gradient of S (the final state's gradient,
+    or zero, at the end of each sequence):
+        G += q do^T;  dq = S do;  du = G^T k;  dv = beta du;  dbeta = du . (v - w);
+        dw = -beta du;  dk = G u + P dw;  dP = G + k dw^T;
+        dlog_alpha_i = sum_j dP_ij P_ij;  G <- Diag(alpha) dP  (the gradient of S_prev).
+    Returns (dq, dk, dv, dlog_alpha, dbeta, d_initial_state), float64, shapes of the inputs.
+    """
+    q, k, v, la, b = _f64(q), _f64(k), _f64(v), _f64(log_alpha), _f64(beta)
+    do = _f64(d_out)
+    TT, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    N = len(cu) - 1
+    S0 = np.zeros((N, H, dk, dv)) if initial_state is None else _f64(initial_state)
+    dq, dkk, dvv, dla, db = (np.zeros_like(x) for x in (q, k, v, la, b))
+    dS0 = np.zeros_like(S0)
+    for n in range(N):
+        s, e = cu[n], cu[n + 1]
+        # forward, keeping every state
+        states = [S0[n]]
+        for t in range(s, e):
+            S, _ = token_step(states[-1], q[t], k[t], v[t], la[t], b[t])
+            states.append(S)
+        G = np.zeros((H, dk, dv)) if d_final is None else _f64(d_final)[n].copy()
+        for i, t in enumerate(range(e - 1, s - 1, -1)):
+            S, Sp = states[len(states) - 1 - i], states[len(states) - 2 - i]
+            alpha = np.exp(la[t])                              # [H, dk]
+            P = alpha[:, :, None] * Sp                         # [H, dk, dv]
+            w = np.einsum("hij,hi->hj", P, k[t])               # [H, dv]
+            u = b[t][:, None] * (v[t] - w)
+            G = G + np.einsum("hi,hj->hij", q[t], do[t])
+            dq[t] = np.einsum("hij,hj->hi", S, do[t])
+            du = np.einsum("hij,hi->hj", G, k[t])
+            dvv[t] = b[t][:, None] * du
+            db[t] = np.sum(du * (v[t] - w), axis=1)
+            dw = -b[t][:, None] * du
+            dkk[t] = np.einsum("hij,hj->hi", G, u) + np.einsum("hij,hj->hi", P, dw)
+            dP = G + np.einsum("hi,hj->hij", k[t], dw)
+            dla[t] = np.sum(dP * P, axis=2)
+            G = alpha[:, :, None] * dP
+        dS0[n] = G
+    return dq, dkk, dvv, dla, db, dS0

@@ -415,3 +415,36 @@ def test_softplus_gate_closed_forms():
     assert np.all(la < 0)
     np.testing.assert_allclose(la[:, 1], -np.log1p(np.exp(a[:, 1])), rtol=1e-12)   # scale 1
     np.testing.assert_allclose(la[:, 2], -2 * np.log1p(np.exp(a[:, 2])), rtol=1e-12)  # linear in the scale
+
+
+def test_backward_matches_finite_differences():
+    """Every gradient of kda_backward against central differences of kda_recurrence
+    (tiny packed problem with two sequences, a loss mixing all outputs and the final
+    states with fixed random weights)."""
+    rng = np.random.default_rng(137106)
+    lens, H, d = [4, 3], 2, 3
+    TT = sum(lens)
+    cu = np.array([0, 4, 7])
+    q, k, v = (rng.standard_normal((TT, H, d)) for _ in range(3))
+    la = -np.log1p(np.exp(rng.standard_normal((TT, H, d))))
+    b = 1 / (1 + np.exp(-rng.standard_normal((TT, H))))
+    s0 = rng.standard_normal((2, H, d, d)) * 0.3
+    wo, wf = rng.standard_normal((TT, H, d)), rng.standard_normal((2, H, d, d))
+
+    def loss(q_, k_, v_, la_, b_, s0_):
+        o, f = O.kda_recurrence(q_, k_, v_, la_, b_, s0_, cu)
+        return np.sum(wo * o) + np.sum(wf * f)
+
+    grads = O.kda_backward(q, k, v, la, b, s0, cu, wo, wf)
+    args = [q, k, v, la, b, s0]
+    eps = 1e-6
+    for which, (x, g) in enumerate(zip(args, grads)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            xp, xm = [a.copy() for a in args], [a.copy() for a in args]
+            xp[which][i] += eps
+            xm[which][i] -= eps
+            num[i] = (loss(*xp) - loss(*xm)) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7, err_msg=f"gradient {which}")
