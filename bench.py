@@ -80,6 +80,14 @@ def mixer_decode_tokens_bytes(N: int, K: int, Hh: int = H, d: int = D) -> int:
     return N * Hh * (2 * d * d * 4 + 2 * 9 * d * 2 + K * (5 * d * 2 + d * 4 + 4)) + N * 4
 
 
+def backward_bytes(total_T: int, N: int, Hh: int = H, d: int = D) -> int:
+    """Algorithmic HBM bytes of one backward call: q, k, v, d_out (bf16), log_alpha (fp32),
+    beta read; dq, dk, dv, d_log_alpha (fp32), d_beta written; initial state and the
+    final state's gradient read, the initial state's gradient written."""
+    tok = total_T * Hh * (4 * d * 2 + d * 4 + 4 + 4 * d * 4 + 4)
+    return tok + 3 * N * Hh * d * d * 4
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -586,6 +594,32 @@ def run_gpu(args):
                "tensor_tflops": prefill_tc_flops(TT) / (vms * 1e-3) / 1e12}
         del vi, vo, vf, vws
 
+    # ---------------- backward of the recurrence, the model shape B=1 T=4096 H=32 ---------------
+    bwd = None
+    if not args.quick:
+        bi = device_prefill_inputs(T1, H, D, 1370008, device, state_N=1)
+        gen = torch.Generator(device=device).manual_seed(1370009)
+        d_out = torch.randn(T1, H, D, generator=gen, device=device).bfloat16()
+        d_fin = 0.1 * torch.randn(1, H, D, D, generator=gen, device=device)
+        bws = torch.empty(kda.chunk_bwd_workspace_bytes(T1, 1, H), dtype=torch.uint8, device=device)
+
+        def bstep(i):
+            kda.chunk_bwd(bi["q"], bi["k"], bi["v"], bi["log_alpha"], bi["beta"], d_out, bi["initial_state"], None,
+                          d_fin, N=1, workspace=bws, stream=stream)
+
+        bsteps = max(3, min(args.steps, 5))
+        bper, btot = time_region(bstep, bsteps, 3, stream, device)
+        launches += 2 * bsteps  # plan + backward kernel
+        btot = max_over_ranks(btot, device)
+        bbytes = backward_bytes(T1, 1)
+        bms = statistics.mean(bper)
+        bwd = {"workload": f"backward of the recurrence B=1 T={T1} H={H} d={D} (bf16 q/k/v/d_out, fp32 gradients, "
+                           "initial state and final-state gradient)",
+               "ms_per_call": btot / bsteps, "tokens_per_s": job_throughput(T1 * bsteps, world, btot / 1e3),
+               "roofline": {"bound": "hbm", "achieved": bbytes / (bms * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                            "frac": bbytes / (bms * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_launch": bbytes}}
+        del bi, d_out, d_fin, bws
+
     cpu = cpu_baseline(args) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
 
     if rank == 0:
@@ -608,7 +642,7 @@ def run_gpu(args):
                     "pipelining": "2 device buffer sets; upload, kernels and download of consecutive steps overlap "
                                   "on three streams; every step's copies are inside the timed region"},
             "decode": decode, "mixer_decode": mdec, "context_parallel": cpar, "mixer": mix, "varlen": var,
-            "clocks": clocks, "gpu_launches": launches, "cpu_baseline": cpu,
+            "backward": bwd, "clocks": clocks, "gpu_launches": launches, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -11,6 +11,7 @@ calls raise.
     out, final = mixer_fwd(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, ...)
     out        = mixer_decode_step(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate,
                                    state_pool, conv_pool, state_indices)  # pools in place
+    dq, dk, dv, dla, dbeta, dh0 = chunk_bwd(q, k, v, log_alpha, beta, d_out, ...)
 
 Shapes (token-major, packed): q, k, log_alpha [total_T, H, dk]; v [total_T, H, dv];
 beta [total_T, H]; states [N, H, dk, dv]; cu_seqlens int32 [N+1] (device).
@@ -69,6 +70,9 @@ _SIGNATURES = {
     "kda_mixer_fwd_gate_workspace": (_sz, [_i64, _i32, _i32, _i32, _i32]),
     "kda_mixer_fwd_gate": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
                                   _vp, _vp, _vp, _sz, _vp]),
+    "kda_chunk_bwd_workspace": (_sz, [_i64, _i32, _i32, _i32, _i32]),
+    "kda_chunk_bwd": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
+                             _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 
 
@@ -296,6 +300,41 @@ def mixer_fwd_gate(q_raw, k_raw, v_raw, conv_w, a_pre, a_scale, beta, gate=None,
     if check_status:
         workspace_status(workspace, stream)
     return out, final_state
+
+
+def chunk_bwd_workspace_bytes(total_T: int, N: int, H: int, dk: int = 128, dv: int = 128) -> int:
+    return int(load_library().kda_chunk_bwd_workspace(total_T, N, H, dk, dv))
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, d_out, initial_state=None, cu_seqlens=None, d_final_state=None, *,
+              N: Optional[int] = None, output_d_initial_state: bool = True, workspace=None, stream=None,
+              check_status: bool = False):
+    """Backward of the recurrence (kda_chunk_bwd). Packed [total_T, H, 128] inputs as for
+    chunk_fwd; d_out like v. Returns fp32 (dq, dk, dv, d_log_alpha, d_beta,
+    d_initial_state or None)."""
+    torch = _torch()
+    lib = load_library()
+    total_T, H, dk = q.shape
+    dv = v.shape[-1]
+    if N is None:
+        if cu_seqlens is None:
+            raise ValueError("N is needed when cu_seqlens is not given")
+        N = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dk_, dv_, dla = (torch.empty((total_T, H, n), **f32) for n in (dk, dk, dv, dk))
+    dbeta = torch.empty((total_T, H), **f32)
+    dh0 = torch.empty((N, H, dk, dv), **f32) if output_d_initial_state else None
+    need = int(lib.kda_chunk_bwd_workspace(total_T, N, H, dk, dv))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+                             _ptr(cu_seqlens), total_T, N, H, dk, dv, _ptr(d_out), _ptr(d_final_state), _ptr(dq),
+                             _ptr(dk_), _ptr(dv_), _ptr(dla), _ptr(dbeta), _ptr(dh0), _ptr(workspace),
+                             workspace.numel(), _stream(stream)))
+    if check_status:
+        workspace_status(workspace, stream)
+    return dq, dk_, dv_, dla, dbeta, dh0
 
 
 def workspace_status(workspace, stream=None) -> int:

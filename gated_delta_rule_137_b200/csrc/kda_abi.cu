@@ -430,6 +430,56 @@ kda_status kda_mixer_fwd_gate(const void* q_raw, const void* k_raw, const void* 
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return ok();
 }
+size_t kda_chunk_bwd_workspace(int64_t total_T, int N, int H, int dk, int dv) {
+  if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
+  if (dk != kda::kD || dv != kda::kD) return 0;
+  return kda::kStatusBytes + kda::bwd_workspace_bytes(total_T, N, H);
+}
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, kda_dtype qkv_dtype, const float* log_alpha,
+                         const float* beta, const float* initial_state, const int32_t* cu_seqlens, int64_t total_T,
+                         int N, int H, int dk, int dv, const void* d_out, const float* d_final_state, float* dq,
+                         float* dk_out, float* dv_out, float* d_log_alpha, float* d_beta, float* d_initial_state,
+                         void* workspace, size_t workspace_bytes, kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  kda_status st = check_common(total_T, N, H, dk, dv);
+  if (st != KDA_OK) return st;
+  if (dk != kda::kD || dv != kda::kD) return fail(KDA_ERR_UNSUPPORTED, "the backward needs dk == dv == 128");
+  if (qkv_dtype != KDA_DT_F32 && qkv_dtype != KDA_DT_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "qkv_dtype=%d is neither KDA_DT_F32 nor KDA_DT_BF16", static_cast<int>(qkv_dtype));
+  if (N == 0) {
+    if (total_T != 0) return fail(KDA_ERR_INVALID_ARG, "N=0 with total_T=%lld", static_cast<long long>(total_T));
+    return ok();
+  }
+  if (!cu_seqlens && total_T % N != 0)
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL but total_T=%lld is not a multiple of N=%d",
+                static_cast<long long>(total_T), N);
+  if (total_T > 0 && (!q || !k || !v || !log_alpha || !beta || !d_out || !dq || !dk_out || !dv_out ||
+                      !d_log_alpha || !d_beta))
+    return fail(KDA_ERR_INVALID_ARG, "inputs, d_out and the token gradients must be non-NULL");
+  const void* ptrs[] = {q, k, v, log_alpha, initial_state, d_out, d_final_state, dq, dk_out, dv_out,
+                        d_log_alpha, d_initial_state, workspace};
+  const char* names[] = {"q", "k", "v", "log_alpha", "initial_state", "d_out", "d_final_state", "dq", "dk",
+                         "dv", "d_log_alpha", "d_initial_state", "workspace"};
+  for (int i = 0; i < 13; ++i)
+    if (ptrs[i] && !aligned16(ptrs[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  if ((beta && (reinterpret_cast<uintptr_t>(beta) & 3u)) || (d_beta && (reinterpret_cast<uintptr_t>(d_beta) & 3u)))
+    return fail(KDA_ERR_INVALID_ARG, "beta and d_beta must be 4-byte aligned");
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+  const size_t need = kda_chunk_bwd_workspace(total_T, N, H, dk, dv);
+  if (!workspace || workspace_bytes < need)
+    return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? workspace_bytes : 0, need);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  e = kda::launch_backward(q, k, v, qkv_dtype == KDA_DT_BF16, log_alpha, beta, initial_state, cu_seqlens, total_T, N,
+                           H, d_out, d_final_state, dq, dk_out, dv_out, d_log_alpha, d_beta, d_initial_state,
+                           static_cast<char*>(workspace) + kda::kStatusBytes, status, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+  return ok();
+}
+
 kda_status kda_workspace_status(void* workspace, kda_stream_t stream_, uint32_t* flags) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!workspace) return fail(KDA_ERR_INVALID_ARG, "workspace is NULL");

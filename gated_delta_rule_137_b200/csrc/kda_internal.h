@@ -75,6 +75,17 @@ inline size_t split_workspace_bytes(int64_t total_T, int N, int H, bool any_chai
   return split_plan_bytes(N) + items;
 }
 cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream);
+// cu_seqlens (or N equal lengths) -> chunk_start[N + 1]: the first 64-token chunk of each
+// sequence, [N] = total; -1 there and the status flag on bad cu_seqlens.
+cudaError_t launch_plan(const int32_t* cu, int64_t total_T, int N, int32_t* chunk_start, uint32_t* status,
+                        cudaStream_t stream);
+
+// Backward of the recurrence (kda_backward.cu).
+size_t bwd_workspace_bytes(int64_t total_T, int N, int H);
+cudaError_t launch_backward(const void* q, const void* k, const void* v, bool bf16, const float* log_alpha,
+                            const float* beta, const float* h0, const int32_t* cu, int64_t total_T, int N, int H,
+                            const void* d_out, const float* d_final, float* dq, float* dk, float* dv, float* dla,
+                            float* dbeta, float* dh0, void* ws, uint32_t* status, cudaStream_t stream);
 
 // Sets the message kda_last_error() returns on this host thread.
 void set_last_error(const char* msg);

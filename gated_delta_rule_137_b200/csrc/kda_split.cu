@@ -1099,11 +1099,16 @@ cudaError_t launch_recur(const PrefillArgs& a, const SplitPlan& p, cudaStream_t 
 
 }  // namespace
 
+cudaError_t launch_plan(const int32_t* cu, int64_t total_T, int N, int32_t* chunk_start, uint32_t* status,
+                        cudaStream_t stream) {
+  kda_plan_kernel<<<1, 1024, 0, stream>>>(cu, total_T, N, chunk_start, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream) {
   uint8_t* ws = static_cast<uint8_t*>(a.split_ws);
   SplitPlan p{reinterpret_cast<const int32_t*>(ws), ws + split_plan_bytes(a.N)};
-  kda_plan_kernel<<<1, 1024, 0, stream>>>(a.cu, a.total_T, a.N, reinterpret_cast<int32_t*>(ws), a.status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_plan(a.cu, a.total_T, a.N, reinterpret_cast<int32_t*>(ws), a.status, stream);
   if (e != cudaSuccess) return e;
   const int64_t max_chunks = split_max_chunks(a.total_T, a.N);
   if (a.a_pre) {  // the full mixer with the decay gate made from its pre-activation

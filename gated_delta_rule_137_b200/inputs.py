@@ -204,6 +204,18 @@ def make_gate_preactivation(total_T, H, d, *, seed):
     return a, scale
 
 
+def make_cotangents(total_T, N, H, dv, *, seed, qkv_dtype="bf16", dk=None, final_std=0.1):
+    """Gradients fed to the backward: d_out ~ N(0, 1) [total_T, H, dv] (rounded to bf16
+    when the inputs are bf16) and d_final ~ N(0, final_std^2) fp32 [N, H, dk, dv]
+    (None when final_std is 0)."""
+    rng = np.random.default_rng(seed)
+    d_out = _normal(rng, (total_T, H, dv))
+    if qkv_dtype == "bf16":
+        _bf16_round_inplace(d_out)
+    d_final = _normal(rng, (N, H, dk or dv, dv), final_std) if final_std else None
+    return d_out, d_final
+
+
 @dataclasses.dataclass
 class MixerDecodeWorkload:
     """Serving decode of the full mixer: `steps` tokens for N sequences whose states and

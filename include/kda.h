@@ -304,6 +304,46 @@ KDA_API kda_status kda_mixer_fwd_noalloc(const void* q_raw, const void* k_raw, c
                                          float* final_state, kda_stream_t stream);
 
 /*
+ * Workspace for kda_chunk_bwd (bytes, multiple of 256; 0 for rejected sizes): the
+ * status word, a checkpoint of the state every 16 tokens (64 KB per 16 tokens and
+ * head, e.g. 545 MB for one 4096-token sequence of 32 heads) and 1 MB of scratch for
+ * each of min(N * H, 148) CTAs.
+ */
+KDA_API size_t kda_chunk_bwd_workspace(int64_t total_T, int N, int H, int dk, int dv);
+
+/*
+ * Backward of the recurrence (training): given the gradient of the loss with respect
+ * to the outputs (and optionally the final state), the gradients with respect to every
+ * input of kda_chunk_fwd. Defining passage: the same KDA section; the gradient is that
+ * of the token recurrence, which the chunked forward computes up to rounding. Writing
+ * one token with P = Diag(alpha) S_prev, w = P^T k, u = beta (v - w), S = P + k u^T,
+ * o = S^T q and walking the tokens backwards with G the gradient of S:
+ *     G += q do^T;  dq = S do;  du = G^T k;  dv = beta du;  dbeta = du . (v - w);
+ *     dk = G u - beta P du;  dP = G - beta k du^T;
+ *     dlog_alpha_i = sum_j dP_ij P_ij;  G <- Diag(alpha) dP.
+ * The states are recomputed from checkpoints taken every 16 tokens; arithmetic fp32.
+ *
+ *   q, k, v, log_alpha, beta, initial_state, cu_seqlens, total_T, N, H: as for
+ *              kda_chunk_fwd (dk == dv == 128 only: KDA_ERR_UNSUPPORTED otherwise).
+ *   d_out      device [total_T, H, dv], dtype qkv_dtype: gradient of the outputs.
+ *   d_final_state  device fp32 [N, H, dk, dv] or NULL (zero).
+ *   dq, dk, dv, d_log_alpha   device fp32 [total_T, H, 128], written.
+ *   d_beta     device fp32 [total_T, H], written.
+ *   d_initial_state  device fp32 [N, H, dk, dv] or NULL (not written): gradient of the
+ *              state before each sequence (d_final_state for an empty sequence).
+ *   workspace  device, >= kda_chunk_bwd_workspace(...) bytes, 16-byte aligned.
+ * Outputs must not overlap the inputs. Pointers 16-byte aligned (beta, d_beta: 4).
+ * Returns KDA_OK once the work is enqueued; bad cu_seqlens set KDA_DEVFLAG_BAD_SEQLENS
+ * in the workspace status word and leave the outputs unwritten.
+ */
+KDA_API kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, kda_dtype qkv_dtype,
+                                 const float* log_alpha, const float* beta, const float* initial_state,
+                                 const int32_t* cu_seqlens, int64_t total_T, int N, int H, int dk, int dv,
+                                 const void* d_out, const float* d_final_state, float* dq, float* dk_out,
+                                 float* dv_out, float* d_log_alpha, float* d_beta, float* d_initial_state,
+                                 void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * Reads the device status word kept in `workspace` (KDA_DEVFLAG_* bits) after
  * synchronising `stream`, and clears it. Returns KDA_ERR_RANGE when any bit
  * was set, KDA_OK otherwise; *flags (if not NULL) receives the bits.

@@ -58,3 +58,21 @@ def assert_decode_out_close(got, ref, what: str):
     bound = DECODE_TOL * np.max(np.abs(ref)) + BF16_HALF_ULP * np.abs(ref) * 1.0001
     over = np.abs(got - ref) - bound
     assert np.all(over <= 0), f"{what}: worst excess {float(np.max(over)):.3e}"
+
+
+# The backward runs token by token in fp32. Per step each gradient element is a sum of at
+# most 2 x 128 fp32 products (unit roundoff 2^-24 ~ 6e-8, so <= 1.5e-5 relative per step
+# in the worst case), and the gradient of the state is carried through maps of norm <= 1
+# (alpha <= 1, beta in (0, 1), |k| = 1), so rounding adds up at most linearly along a
+# sequence: T x 1.5e-5 bounds it (1.5e-3 at 100 tokens) and random signs make it grow like
+# sqrt(T). 1e-3 of the largest magnitude holds every case tested here with room, while a
+# dropped term, a wrong sign or a transposed operand moves gradients by O(1) of it.
+BWD_TOL = 1e-3
+
+
+def assert_backward_close(got, ref, what: str):
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = float(np.max(np.abs(got - ref)))
+    scale = float(np.max(np.abs(ref)))
+    assert err <= BWD_TOL * scale, f"{what}: max|err|={err:.3e} > {BWD_TOL}*max|ref|={BWD_TOL * scale:.3e}"
+    return err / scale

@@ -186,3 +186,38 @@ def test_state_affine_rejects_bad_arguments(lib):
     assert lib.kda_state_affine(FAKE, FAKE * 2, FAKE * 3, FAKE + 8, 2, 128, None) == kda.KDA_ERR_INVALID_ARG
     assert lib.kda_state_affine(FAKE, FAKE * 2, None, FAKE * 2, 2, 128, None) == kda.KDA_ERR_INVALID_ARG  # out is S
     assert lib.kda_state_affine(FAKE, None, None, FAKE * 4, 0, 128, None) == kda.KDA_OK  # nothing to do
+
+
+def test_chunk_bwd_workspace_formula(lib):
+    # status word + plan + one fp32 state per 16 tokens (4 per 64-token chunk bound) and
+    # head + 1 MB (16 states, 16 x 2 vectors) of scratch per CTA, at most 148 CTAs
+    def expect(T, N, H):
+        plan = -(-(N + 1) * 4 // 256) * 256
+        chunks = min(T // 64 + N, T)
+        ckpt = -(-(chunks * 4 * H * 128 * 128 * 4) // 256) * 256
+        scratch = min(N * H, 148) * (16 * 128 * 128 + 16 * 2 * 128) * 4
+        return 256 + plan + ckpt + scratch
+    assert lib.kda_chunk_bwd_workspace(0, 3, 2, 128, 128) == 256 + 256   # status + plan only
+    for T, N, H in [(4096, 1, 32), (300, 5, 2), (1, 1, 1), (262144, 64, 32)]:
+        assert lib.kda_chunk_bwd_workspace(T, N, H, 128, 128) == expect(T, N, H)
+    assert lib.kda_chunk_bwd_workspace(4096, 1, 32, 64, 128) == 0   # only dk == dv == 128
+    assert lib.kda_chunk_bwd_workspace(-1, 1, 32, 128, 128) == 0
+
+
+def test_chunk_bwd_rejects_bad_arguments(lib):
+    ws = lib.kda_chunk_bwd_workspace(128, 2, 2, 128, 128)
+    f = FAKE
+
+    def call(q=f, la=f * 2, beta=f * 3, d_out=f * 4, dq=f * 5, dbeta=f * 6, cu=None, T=128, N=2, dk=128,
+             ws_bytes=ws, dtype=kda.KDA_DT_BF16):
+        return lib.kda_chunk_bwd(q, f, f, dtype, la, beta, None, cu, T, N, 2, dk, 128, d_out, None, dq, f, f, f,
+                                 dbeta, None, f * 7, ws_bytes, None)
+    assert call(dk=64) == kda.KDA_ERR_UNSUPPORTED
+    assert call(dtype=7) == kda.KDA_ERR_INVALID_ARG
+    assert call(d_out=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(dbeta=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(q=f + 8) == kda.KDA_ERR_INVALID_ARG            # misaligned
+    assert call(beta=f + 2) == kda.KDA_ERR_INVALID_ARG         # beta needs 4-byte alignment
+    assert call(T=129) == kda.KDA_ERR_INVALID_ARG              # not a multiple of N without cu_seqlens
+    assert call(ws_bytes=ws - 256) == kda.KDA_ERR_WORKSPACE
+    assert call(T=0, N=0) == kda.KDA_OK                        # empty batch: nothing to do
