@@ -1,5 +1,4 @@
-// kda_backward.cu — gradients of the KDA recurrence (training), one CTA per (sequence,
-// head), fp32 on CUDA cores.
+// kda_backward.cu — gradients of the KDA recurrence (training), fp32 on CUDA cores.
 //
 // Recurrence (Ling-3.0-flash article, section "KDA: constant-size memory over a very
 // long context"), one token written with P = Diag(alpha) S_prev, w = P^T k,
@@ -9,53 +8,65 @@
 //   dw = -beta du;  dk = G u + P dw;  dP = G + k dw^T;
 //   dlog_alpha_i = sum_j dP_ij P_ij;  G <- Diag(alpha) dP.
 //
-// The states the walk needs are recomputed: pass 1 runs the forward with the state in
-// registers and stores it at the start of every 64-token chunk; pass 2 takes the chunks
-// in reverse, recomputes one from its checkpoint (keeping the state before each token,
-// and u and v - w, in a per-CTA scratch) and walks its tokens backwards. The checkpoints
-// come every 16 tokens so that the scratch a CTA writes and reads back (16 states of
-// 64 KB) stays in L2; the grid is persistent, each CTA taking (sequence, head) chains in
-// turn, so the scratch is bounded by the number of SMs.
+// Every column j of S (and of G) evolves on its own: w_j, u_j, du_j, dv_j, dw_j and the
+// updates of S[:, j] and G[:, j] read only column j and the token's row vectors (k, q,
+// alpha). Only dq, dk, dlog_alpha and dbeta sum over the columns. So a (sequence, head)
+// chain is cut into 4 slices of 32 value columns, one CTA each, the 4 CTAs of a chain
+// forming a thread-block cluster; their per-slice row sums meet through distributed
+// shared memory and are added in a fixed order (the result does not depend on timing).
 //
-// Layout as in the decode kernels: 256 threads, warp w holds state rows 16w..16w+15,
-// lane l columns 4l..4l+3. Column sums (over rows) go through shared memory across the
-// 8 warps; row sums (over columns) are a reduce-scatter inside the warp.
+// The states the backward walk needs are recomputed: pass 1 runs the forward and stores
+// the state at the start of every 8 tokens; pass 2 takes these stretches in reverse,
+// recomputes one from its checkpoint (keeping the state before each of its tokens, and
+// u and v - w, in shared memory) and walks its tokens backwards. Per token the inputs of
+// the next token are fetched while the current one computes (two buffers in shared
+// memory), so a token costs two block barriers and no exposed global load.
+//
+// Thread layout: 256 threads, warp w holds state rows 16w..16w+15, lane l column l of
+// the slice. Column sums (over rows) go through shared memory across the 8 warps; row
+// sums (over the slice's columns) are a reduce-scatter across the 32 lanes.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "kda_internal.h"
 
+namespace cg = cooperative_groups;
+
 namespace kda {
 
 namespace {
 
-constexpr int kBD = 128;          // head dim
-constexpr int kBRows = 16;        // rows per warp
-constexpr int kBChunk = 16;       // checkpoint interval (tokens): a CTA's scratch (1 MB) stays in L2
-constexpr int kBPerChunk = 64 / kBChunk;  // checkpoints per 64-token chunk of the plan
-constexpr int kBwdMaxCtas = 148;  // persistent grid: one CTA per SM (the registers allow no more)
+constexpr int kBD = 128;                  // head dim (rows of the state, and all its columns)
+constexpr int kBCols = 32;                // value columns of one slice
+constexpr int kBSlices = kBD / kBCols;    // CTAs (cluster size) per chain
+constexpr int kBRows = 16;                // rows per warp
+constexpr int kBStretch = 8;              // checkpoint interval (tokens)
+constexpr int kBPerChunk = 64 / kBStretch;  // checkpoints per 64-token chunk of the plan
+constexpr int kBThreads = 256;
+constexpr int kBMaxClusters = 37;         // 148 SMs / 4: an upper bound on resident clusters
 
 __device__ __forceinline__ float bload(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float bload(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// Row sums of a warp's 16 x 128 block: v[r] is this lane's partial (its 4 columns) for
-// row r. Returns the full sum of row `row` (set here), which lanes l and l ^ 1 share.
+// Row sums of a warp's 16 x 32 block: v[r] is this lane's element of row r. Returns the
+// full sum of row `row` (set here), which lanes l and l ^ 1 share.
 __device__ __forceinline__ float row_sums16(const float (&v)[16], int lane, int& row) {
   const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
   float a[8];
-  #pragma unroll
+#pragma unroll
   for (int r = 0; r < 8; ++r) {
     const float keep = b4 ? v[r + 8] : v[r], send = b4 ? v[r] : v[r + 8];
     a[r] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
   }
   float b[4];
-  #pragma unroll
+#pragma unroll
   for (int r = 0; r < 4; ++r) {
     const float keep = b3 ? a[r + 4] : a[r], send = b3 ? a[r] : a[r + 4];
     b[r] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
   }
   float c[2];
-  #pragma unroll
+#pragma unroll
   for (int r = 0; r < 2; ++r) {
     const float keep = b2 ? b[r + 2] : b[r], send = b2 ? b[r] : b[r + 2];
     c[r] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
@@ -74,37 +85,85 @@ struct BwdArgs {
   const float* h0;                // [N, H, 128, 128] or null
   const float* d_final;           // [N, H, 128, 128] or null
   const int32_t* cu;              // [N + 1] or null
-  const int32_t* chunk_start;     // [N + 1] from the plan kernel
+  const int32_t* chunk_start;     // [N + 1] from the plan kernel (64-token chunks)
   float *dq, *dk, *dv, *dla, *dbeta, *dh0;
-  float* ckpt;                    // [4 x 64-token chunks][H][128][128]: one state per 16 tokens
-  float* scratch;                 // per CTA: [16][128][128] states + [16][2][128] u, v - w
-  uint32_t* status;
+  float* ckpt;                    // [8 x 64-token chunks][H][128][128]: the state every 8 tokens
   int64_t total_T;
   int N, H;
 };
 
-constexpr size_t kBwdScratchFloats = static_cast<size_t>(kBChunk) * kBD * kBD + static_cast<size_t>(kBChunk) * 2 * kBD;
+// Shared memory of one CTA (dynamic).
+struct BwdSmem {
+  float st[kBStretch][kBD][kBCols];      // state before each token of the stretch (this slice)
+  float part[2][kBStretch][3][kBD];      // per-slice row sums dq, dk, dla (double-buffered)
+  float part_beta[2][kBStretch];         // per-slice dbeta
+  float u[kBStretch][kBCols], vw[kBStretch][kBCols];
+  float red[8][kBCols];                  // column sums across the 8 warps
+  float k[2][kBD], q[2][kBD], al[2][kBD];  // row vectors of the token (two buffers)
+  float v[2][kBCols], dout[2][kBCols];   // this slice's columns of v and d_out
+  float beta[2];
+};
+
+// The inputs of one token, held in registers between fetch and publish.
+struct TokRegs {
+  float k, q, la;  // row tid (tid < 128)
+  float x, y;      // v, d_out of column tid - 128 of the slice (128 <= tid < 160); beta (tid == 160)
+};
+
+template <typename TIn, bool kAll>
+__device__ __forceinline__ TokRegs fetch_token(const BwdArgs& a, int64_t t, int h, int c0, int tid) {
+  TokRegs r{0.f, 0.f, 0.f, 0.f, 0.f};
+  const size_t o = (static_cast<size_t>(t) * a.H + h) * kBD;
+  if (tid < kBD) {
+    r.k = bload(static_cast<const TIn*>(a.k) + o + tid);
+    r.la = __ldg(a.log_alpha + o + tid);
+    if (kAll) r.q = bload(static_cast<const TIn*>(a.q) + o + tid);
+  } else if (tid < kBD + kBCols) {
+    r.x = bload(static_cast<const TIn*>(a.v) + o + c0 + tid - kBD);
+    if (kAll) r.y = bload(static_cast<const TIn*>(a.d_out) + o + c0 + tid - kBD);
+  } else if (tid == kBD + kBCols) {
+    r.x = __ldg(a.beta + static_cast<size_t>(t) * a.H + h);
+  }
+  return r;
+}
+
+template <bool kAll>
+__device__ __forceinline__ void publish_token(BwdSmem& s, int b, const TokRegs& r, int tid) {
+  if (tid < kBD) {
+    s.k[b][tid] = r.k;
+    s.al[b][tid] = expf(r.la);
+    if (kAll) s.q[b][tid] = r.q;
+  } else if (tid < kBD + kBCols) {
+    s.v[b][tid - kBD] = r.x;
+    if (kAll) s.dout[b][tid - kBD] = r.y;
+  } else if (tid == kBD + kBCols) {
+    s.beta[b] = r.x;
+  }
+}
 
 template <typename TIn>
-__global__ void __launch_bounds__(256, 1) kda_bwd_kernel(const BwdArgs a) {
-  if (__ldg(a.chunk_start + a.N) < 0) return;  // bad cu_seqlens (flagged by the plan kernel)
+__global__ void __cluster_dims__(kBSlices, 1, 1) __launch_bounds__(kBThreads, 1) kda_bwd_kernel(const BwdArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  BwdSmem& s = *reinterpret_cast<BwdSmem*>(smem_raw);
+  cg::cluster_group cluster = cg::this_cluster();
+  const int slice = static_cast<int>(cluster.block_rank());
+  const int c0 = slice * kBCols;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int row0 = warp * kBRows;
   const int H = a.H;
   const int64_t chains = static_cast<int64_t>(a.N) * a.H;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  const int col = lane * 4, row0 = warp * kBRows;
-  const TIn* qg = static_cast<const TIn*>(a.q);
-  const TIn* kg = static_cast<const TIn*>(a.k);
-  const TIn* vg = static_cast<const TIn*>(a.v);
-  const TIn* dog = static_cast<const TIn*>(a.d_out);
-  float* scrS = a.scratch + static_cast<size_t>(blockIdx.x) * kBwdScratchFloats;  // [16][128][128]
-  float* scrU = scrS + static_cast<size_t>(kBChunk) * kBD * kBD;                  // [16][2][128]: u, v - w
+  const int64_t cluster_id = blockIdx.x / kBSlices, n_clusters = gridDim.x / kBSlices;
+  const bool bad = __ldg(a.chunk_start + a.N) < 0;  // bad cu_seqlens (flagged by the plan kernel)
+  const float* peer_part[kBSlices];
+  const float* peer_beta[kBSlices];
+#pragma unroll
+  for (int p = 0; p < kBSlices; ++p) {
+    peer_part[p] = cluster.map_shared_rank(&s.part[0][0][0][0], p);
+    peer_beta[p] = cluster.map_shared_rank(&s.part_beta[0][0], p);
+  }
+  int pb = 0;  // partial-sum buffer of the current stretch
 
-  __shared__ float s_k[kBD], s_q[kBD], s_al[kBD];   // row vectors of the current token
-  __shared__ float s_v[kBD], s_do[kBD];             // column vectors
-  __shared__ float s_beta;
-  __shared__ float4 s_red[8][32];
-
-  for (int64_t nh = blockIdx.x; nh < chains; nh += gridDim.x) {
+  for (int64_t nh = bad ? chains : cluster_id; nh < chains; nh += n_clusters) {
     const int n = static_cast<int>(nh / H), h = static_cast<int>(nh % H);
     int64_t bos, eos;
     if (a.cu) {
@@ -115,180 +174,181 @@ __global__ void __launch_bounds__(256, 1) kda_bwd_kernel(const BwdArgs a) {
       bos = static_cast<int64_t>(n) * L;
       eos = bos + L;
     }
-    const int nch = static_cast<int>((eos - bos + kBChunk - 1) / kBChunk);
+    const int nst = static_cast<int>((eos - bos + kBStretch - 1) / kBStretch);
     const int64_t cbase = static_cast<int64_t>(__ldg(a.chunk_start + n)) * kBPerChunk;
+    auto ckpt_of = [&](int c) { return a.ckpt + (static_cast<size_t>(cbase + c) * H + h) * kBD * kBD + c0 + lane; };
 
-    auto tok_off = [&](int64_t t) { return (static_cast<size_t>(t) * H + h) * kBD; };
-    auto state_at = [&](float* base, int r) { return base + static_cast<size_t>(row0 + r) * kBD + col; };
-
-    float4 S[kBRows];
+    float S[kBRows];
     {
-      const float* h0 = a.h0 ? a.h0 + static_cast<size_t>(nh) * kBD * kBD : nullptr;
-      #pragma unroll
-      for (int r = 0; r < kBRows; ++r)
-        S[r] = h0 ? *reinterpret_cast<const float4*>(h0 + static_cast<size_t>(row0 + r) * kBD + col)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float* h0 = a.h0 ? a.h0 + static_cast<size_t>(nh) * kBD * kBD + c0 + lane : nullptr;
+#pragma unroll
+      for (int r = 0; r < kBRows; ++r) S[r] = h0 ? __ldg(h0 + (row0 + r) * kBD) : 0.f;
     }
 
-    // one forward token step on S (registers); returns u and v - w for this lane's columns
-    auto fwd_step = [&](int64_t t, float4& u_out, float4& vw_out) {
-      const size_t o = tok_off(t);
-      if (tid < kBD) {
-        s_k[tid] = bload(kg + o + tid);
-        s_al[tid] = expf(a.log_alpha[o + tid]);
-      } else {
-        s_v[tid - kBD] = bload(vg + o + tid - kBD);
+    // one forward token step on S from buffer b; when i >= 0 keeps the state before it,
+    // and u, v - w, as token i of the stretch. Ends after the column-sum barrier.
+    auto fwd_compute = [&](int b, int i) {
+      if (i >= 0) {
+#pragma unroll
+        for (int r = 0; r < kBRows; ++r) s.st[i][row0 + r][lane] = S[r];
       }
-      if (tid == 0) s_beta = a.beta[static_cast<size_t>(t) * H + h];
-      __syncthreads();
-      float4 pw = make_float4(0.f, 0.f, 0.f, 0.f);
-      #pragma unroll
+      float pw = 0.f;
+#pragma unroll
       for (int r = 0; r < kBRows; ++r) {
-        const float al = s_al[row0 + r], kr = s_k[row0 + r];
-        S[r].x *= al; S[r].y *= al; S[r].z *= al; S[r].w *= al;
-        pw.x = fmaf(kr, S[r].x, pw.x); pw.y = fmaf(kr, S[r].y, pw.y);
-        pw.z = fmaf(kr, S[r].z, pw.z); pw.w = fmaf(kr, S[r].w, pw.w);
+        S[r] *= s.al[b][row0 + r];
+        pw = fmaf(s.k[b][row0 + r], S[r], pw);
       }
-      s_red[warp][lane] = pw;
+      s.red[warp][lane] = pw;
       __syncthreads();
-      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-      #pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const float4 p = s_red[x][lane];
-        w.x += p.x; w.y += p.y; w.z += p.z; w.w += p.w;
+      float w = 0.f;
+#pragma unroll
+      for (int x = 0; x < 8; ++x) w += s.red[x][lane];
+      const float vw = s.v[b][lane] - w, u = s.beta[b] * vw;
+#pragma unroll
+      for (int r = 0; r < kBRows; ++r) S[r] = fmaf(s.k[b][row0 + r], u, S[r]);
+      if (i >= 0 && warp == 0) {
+        s.u[i][lane] = u;
+        s.vw[i][lane] = vw;
       }
-      const float bt = s_beta;
-      vw_out = make_float4(s_v[col] - w.x, s_v[col + 1] - w.y, s_v[col + 2] - w.z, s_v[col + 3] - w.w);
-      u_out = make_float4(bt * vw_out.x, bt * vw_out.y, bt * vw_out.z, bt * vw_out.w);
-      #pragma unroll
-      for (int r = 0; r < kBRows; ++r) {
-        const float kr = s_k[row0 + r];
-        S[r].x = fmaf(kr, u_out.x, S[r].x); S[r].y = fmaf(kr, u_out.y, S[r].y);
-        S[r].z = fmaf(kr, u_out.z, S[r].z); S[r].w = fmaf(kr, u_out.w, S[r].w);
-      }
-      __syncthreads();  // s_k / s_al / s_v / s_red are rewritten by the next step
     };
 
-    // ---- pass 1: forward, a checkpoint at the start of every chunk ------------------------
-    for (int c = 0; c < nch; ++c) {
-      float* ck = a.ckpt + (static_cast<size_t>(cbase + c) * H + h) * kBD * kBD;
-      #pragma unroll
-      for (int r = 0; r < kBRows; ++r) *reinterpret_cast<float4*>(state_at(ck, r)) = S[r];
-      const int64_t t0 = bos + static_cast<int64_t>(c) * kBChunk;
-      const int clen = static_cast<int>(eos - t0 < kBChunk ? eos - t0 : kBChunk);
-      float4 u, vw;
-      for (int i = 0; i < clen; ++i) fwd_step(t0 + i, u, vw);
+    // ---- pass 1: forward, a checkpoint at the start of every stretch ------------------------
+    int b = 0;
+    if (nst > 0) {
+      publish_token<false>(s, b, fetch_token<TIn, false>(a, bos, h, c0, tid), tid);
+      __syncthreads();
     }
-
-    // ---- pass 2: chunks in reverse; recompute, then walk the tokens backwards -----------------
-    float4 G[kBRows];
-    {
-      const float* df = a.d_final ? a.d_final + static_cast<size_t>(nh) * kBD * kBD : nullptr;
-      #pragma unroll
-      for (int r = 0; r < kBRows; ++r)
-        G[r] = df ? *reinterpret_cast<const float4*>(df + static_cast<size_t>(row0 + r) * kBD + col)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int c = nch - 1; c >= 0; --c) {
-      const float* ck = a.ckpt + (static_cast<size_t>(cbase + c) * H + h) * kBD * kBD;
-      #pragma unroll
-      for (int r = 0; r < kBRows; ++r) S[r] = *reinterpret_cast<const float4*>(state_at(const_cast<float*>(ck), r));
-      const int64_t t0 = bos + static_cast<int64_t>(c) * kBChunk;
-      const int clen = static_cast<int>(eos - t0 < kBChunk ? eos - t0 : kBChunk);
-      for (int i = 0; i < clen; ++i) {  // the state before token i, and u, v - w of token i
-        float* sp = scrS + static_cast<size_t>(i) * kBD * kBD;
-        #pragma unroll
-        for (int r = 0; r < kBRows; ++r) *reinterpret_cast<float4*>(state_at(sp, r)) = S[r];
-        float4 u, vw;
-        fwd_step(t0 + i, u, vw);
-        if (warp == 0) {
-          *reinterpret_cast<float4*>(scrU + (static_cast<size_t>(i) * 2) * kBD + col) = u;
-          *reinterpret_cast<float4*>(scrU + (static_cast<size_t>(i) * 2 + 1) * kBD + col) = vw;
-        }
-      }
-      __syncthreads();  // the scratch rows of u, v - w written by warp 0 are read by every warp
-
-      // S now holds the state after the chunk: the state after its last token
-      for (int i = clen - 1; i >= 0; --i) {
-        const int64_t t = t0 + i;
-        const size_t o = tok_off(t);
-        if (tid < kBD) {
-          s_k[tid] = bload(kg + o + tid);
-          s_q[tid] = bload(qg + o + tid);
-          s_al[tid] = expf(a.log_alpha[o + tid]);
-        } else {
-          s_do[tid - kBD] = bload(dog + o + tid - kBD);
-        }
-        if (tid == 0) s_beta = a.beta[static_cast<size_t>(t) * H + h];
-        float4 Sp[kBRows];  // the state before token t
-        const float* sp = scrS + static_cast<size_t>(i) * kBD * kBD;
-        #pragma unroll
-        for (int r = 0; r < kBRows; ++r) Sp[r] = *reinterpret_cast<const float4*>(state_at(const_cast<float*>(sp), r));
-        const float4 u = *reinterpret_cast<const float4*>(scrU + (static_cast<size_t>(i) * 2) * kBD + col);
-        const float4 vw = *reinterpret_cast<const float4*>(scrU + (static_cast<size_t>(i) * 2 + 1) * kBD + col);
+    for (int c = 0; c < nst; ++c) {
+      float* ck = ckpt_of(c);
+#pragma unroll
+      for (int r = 0; r < kBRows; ++r) ck[(row0 + r) * kBD] = S[r];
+      const int64_t t0 = bos + static_cast<int64_t>(c) * kBStretch;
+      const int len = static_cast<int>(eos - t0 < kBStretch ? eos - t0 : kBStretch);
+      for (int i = 0; i < len; ++i) {
+        const int64_t tn = t0 + i + 1;
+        TokRegs nx{};
+        if (tn < eos) nx = fetch_token<TIn, false>(a, tn, h, c0, tid);
+        fwd_compute(b, -1);
+        if (tn < eos) publish_token<false>(s, b ^ 1, nx, tid);
         __syncthreads();
-        const float4 dov = make_float4(s_do[col], s_do[col + 1], s_do[col + 2], s_do[col + 3]);
-        const float bt = s_beta;
+        b ^= 1;
+      }
+    }
 
-        // G += q do^T;  dq = S do (rows);  du partial = G^T k
+    // ---- pass 2: stretches in reverse; recompute, then walk the tokens backwards --------------
+    float G[kBRows];
+    {
+      const float* df = a.d_final ? a.d_final + static_cast<size_t>(nh) * kBD * kBD + c0 + lane : nullptr;
+#pragma unroll
+      for (int r = 0; r < kBRows; ++r) G[r] = df ? __ldg(df + (row0 + r) * kBD) : 0.f;
+    }
+    if (nst > 0) {
+      const int64_t t0 = bos + static_cast<int64_t>(nst - 1) * kBStretch;
+      publish_token<true>(s, b, fetch_token<TIn, true>(a, t0, h, c0, tid), tid);
+      __syncthreads();
+    }
+    for (int c = nst - 1; c >= 0; --c) {
+      const float* ck = ckpt_of(c);
+#pragma unroll
+      for (int r = 0; r < kBRows; ++r) S[r] = ck[(row0 + r) * kBD];
+      const int64_t t0 = bos + static_cast<int64_t>(c) * kBStretch;
+      const int len = static_cast<int>(eos - t0 < kBStretch ? eos - t0 : kBStretch);
+      // recompute tokens t0 .. t0 + len - 1; the last one's inputs stay in their buffer,
+      // since the backward walk starts with the same token
+      for (int i = 0; i < len; ++i) {
+        const bool more = i + 1 < len;
+        TokRegs nx{};
+        if (more) nx = fetch_token<TIn, true>(a, t0 + i + 1, h, c0, tid);
+        fwd_compute(b, i);
+        if (more) publish_token<true>(s, b ^ 1, nx, tid);
+        __syncthreads();
+        if (more) b ^= 1;
+      }
+      // S holds the state after the stretch's last token
+      for (int i = len - 1; i >= 0; --i) {
+        const int64_t t = t0 + i;
+        // next: token t - 1, or, after the stretch's first token, the first token of the
+        // stretch before it (full, 8 tokens), whose recompute comes next
+        const bool more = i > 0 || c > 0;
+        TokRegs nx{};
+        if (more) nx = fetch_token<TIn, true>(a, i > 0 ? t - 1 : t0 - kBStretch, h, c0, tid);
+        const float dov = s.dout[b][lane], bt = s.beta[b];
+        const float u = s.u[i][lane], vw = s.vw[i][lane];
+
+        // G += q do^T;  dq = S do;  du = G^T k (column sum)
         float rs[kBRows];
-        float4 pdu = make_float4(0.f, 0.f, 0.f, 0.f);
-        #pragma unroll
+        float pdu = 0.f;
+#pragma unroll
         for (int r = 0; r < kBRows; ++r) {
-          const float qr = s_q[row0 + r], kr = s_k[row0 + r];
-          G[r].x = fmaf(qr, dov.x, G[r].x); G[r].y = fmaf(qr, dov.y, G[r].y);
-          G[r].z = fmaf(qr, dov.z, G[r].z); G[r].w = fmaf(qr, dov.w, G[r].w);
-          rs[r] = S[r].x * dov.x + S[r].y * dov.y + S[r].z * dov.z + S[r].w * dov.w;
-          pdu.x = fmaf(kr, G[r].x, pdu.x); pdu.y = fmaf(kr, G[r].y, pdu.y);
-          pdu.z = fmaf(kr, G[r].z, pdu.z); pdu.w = fmaf(kr, G[r].w, pdu.w);
+          G[r] = fmaf(s.q[b][row0 + r], dov, G[r]);
+          rs[r] = S[r] * dov;
+          pdu = fmaf(s.k[b][row0 + r], G[r], pdu);
         }
         int rr;
         float sum = row_sums16(rs, lane, rr);
-        if (!(lane & 1)) a.dq[o + row0 + rr] = sum;
-        s_red[warp][lane] = pdu;
+        if (!(lane & 1)) s.part[pb][i][0][row0 + rr] = sum;
+        s.red[warp][lane] = pdu;
         __syncthreads();
-        float4 du = make_float4(0.f, 0.f, 0.f, 0.f);
-        #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const float4 p = s_red[x][lane];
-          du.x += p.x; du.y += p.y; du.z += p.z; du.w += p.w;
-        }
-        if (warp == 0) {  // dv = beta du;  dbeta = du . (v - w)
-          *reinterpret_cast<float4*>(a.dv + o + col) = make_float4(bt * du.x, bt * du.y, bt * du.z, bt * du.w);
-          float db = du.x * vw.x + du.y * vw.y + du.z * vw.z + du.w * vw.w;
-          #pragma unroll
+        float du = 0.f;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) du += s.red[x][lane];
+        if (warp == 0) {  // dv = beta du (complete: column-local);  dbeta partial = du . (v - w)
+          a.dv[(static_cast<size_t>(t) * H + h) * kBD + c0 + lane] = bt * du;
+          float db = du * vw;
+#pragma unroll
           for (int off = 16; off > 0; off >>= 1) db += __shfl_xor_sync(0xffffffffu, db, off);
-          if (lane == 0) a.dbeta[static_cast<size_t>(t) * H + h] = db;
+          if (lane == 0) s.part_beta[pb][i] = db;
         }
-        const float4 dw = make_float4(-bt * du.x, -bt * du.y, -bt * du.z, -bt * du.w);
+        const float dw = -bt * du;
 
         // P = Diag(alpha) S_prev;  dk = G u + P dw;  dP = G + k dw^T;  dla = rowsum(dP * P);  G = alpha dP
         float rk[kBRows], rl[kBRows];
-        #pragma unroll
+#pragma unroll
         for (int r = 0; r < kBRows; ++r) {
-          const float al = s_al[row0 + r], kr = s_k[row0 + r];
-          const float4 P = make_float4(al * Sp[r].x, al * Sp[r].y, al * Sp[r].z, al * Sp[r].w);
-          rk[r] = G[r].x * u.x + G[r].y * u.y + G[r].z * u.z + G[r].w * u.w +
-                  P.x * dw.x + P.y * dw.y + P.z * dw.z + P.w * dw.w;
-          const float4 dP = make_float4(fmaf(kr, dw.x, G[r].x), fmaf(kr, dw.y, G[r].y), fmaf(kr, dw.z, G[r].z),
-                                        fmaf(kr, dw.w, G[r].w));
-          rl[r] = dP.x * P.x + dP.y * P.y + dP.z * P.z + dP.w * P.w;
-          G[r] = make_float4(al * dP.x, al * dP.y, al * dP.z, al * dP.w);
-          S[r] = Sp[r];  // the state after token t - 1
+          const float al = s.al[b][row0 + r], kr = s.k[b][row0 + r];
+          const float sp = s.st[i][row0 + r][lane];
+          const float P = al * sp;
+          rk[r] = fmaf(G[r], u, P * dw);
+          const float dP = fmaf(kr, dw, G[r]);
+          rl[r] = dP * P;
+          G[r] = al * dP;
+          S[r] = sp;  // the state after token t - 1
         }
         sum = row_sums16(rk, lane, rr);
-        if (!(lane & 1)) a.dk[o + row0 + rr] = sum;
+        if (!(lane & 1)) s.part[pb][i][1][row0 + rr] = sum;
         sum = row_sums16(rl, lane, rr);
-        if (!(lane & 1)) a.dla[o + row0 + rr] = sum;
-        __syncthreads();  // shared vectors and s_red are rewritten by the next token
+        if (!(lane & 1)) s.part[pb][i][2][row0 + rr] = sum;
+        if (more) publish_token<true>(s, b ^ 1, nx, tid);
+        __syncthreads();
+        if (more) b ^= 1;
       }
+
+      // the stretch's row sums of all 4 slices: slice p adds up rows 32p .. 32p + 31
+      cluster.sync();
+      for (int e = tid; e < len * 3 * kBCols; e += kBThreads) {
+        const int i = e / (3 * kBCols), which = (e / kBCols) % 3, row = c0 + e % kBCols;
+        const int off = ((pb * kBStretch + i) * 3 + which) * kBD + row;
+        float acc = 0.f;
+#pragma unroll
+        for (int p = 0; p < kBSlices; ++p) acc += peer_part[p][off];
+        float* dst = which == 0 ? a.dq : which == 1 ? a.dk : a.dla;
+        dst[(static_cast<size_t>(t0 + i) * H + h) * kBD + row] = acc;
+      }
+      if (slice == 0 && tid < len) {
+        float acc = 0.f;
+#pragma unroll
+        for (int p = 0; p < kBSlices; ++p) acc += peer_beta[p][pb * kBStretch + tid];
+        a.dbeta[static_cast<size_t>(t0 + tid) * H + h] = acc;
+      }
+      pb ^= 1;  // the next stretch writes the other buffer while peers may still read this one
     }
     if (a.dh0) {
-      float* d0 = a.dh0 + static_cast<size_t>(nh) * kBD * kBD;
-      #pragma unroll
-      for (int r = 0; r < kBRows; ++r) *reinterpret_cast<float4*>(state_at(d0, r)) = G[r];
+      float* d0 = a.dh0 + static_cast<size_t>(nh) * kBD * kBD + c0 + lane;
+#pragma unroll
+      for (int r = 0; r < kBRows; ++r) d0[(row0 + r) * kBD] = G[r];
     }
-  }  // chains
+  }
+  cluster.sync();  // no CTA leaves while a peer may still read its partial sums
 }
 
 }  // namespace
@@ -297,10 +357,7 @@ size_t bwd_workspace_bytes(int64_t total_T, int N, int H) {
   if (total_T < 0 || N <= 0 || H <= 0) return 0;
   if (total_T == 0) return split_plan_bytes(N);  // only the plan: no chain has a token
   const int64_t ckpts = split_max_chunks(total_T, N) * kBPerChunk;
-  const int64_t chains = static_cast<int64_t>(N) * H;
-  const int64_t ctas = chains < kBwdMaxCtas ? chains : kBwdMaxCtas;
-  return split_plan_bytes(N) + align256(static_cast<size_t>(ckpts) * H * kBD * kBD * sizeof(float)) +
-         static_cast<size_t>(ctas) * kBwdScratchFloats * sizeof(float);
+  return split_plan_bytes(N) + align256(static_cast<size_t>(ckpts) * H * kBD * kBD * sizeof(float));
 }
 
 cudaError_t launch_backward(const void* q, const void* k, const void* v, bool bf16, const float* log_alpha,
@@ -311,18 +368,37 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, bool bf
   int32_t* cs = reinterpret_cast<int32_t*>(w);
   cudaError_t e = launch_plan(cu, total_T, N, cs, status, stream);  // 64-token chunks per sequence
   if (e != cudaSuccess) return e;
-  const int64_t ckpts = split_max_chunks(total_T, N) * kBPerChunk;
   float* ckpt = reinterpret_cast<float*>(w + split_plan_bytes(N));
-  float* scratch = reinterpret_cast<float*>(w + split_plan_bytes(N) +
-                                            align256(static_cast<size_t>(ckpts) * H * kBD * kBD * sizeof(float)));
-  BwdArgs a{q, k, v, d_out, log_alpha, beta, h0, d_final, cu, cs, dq, dk, dv, dla, dbeta, dh0,
-            ckpt, scratch, status, total_T, N, H};
+  BwdArgs a{q, k, v, d_out, log_alpha, beta, h0, d_final, cu, cs, dq, dk, dv, dla, dbeta, dh0, ckpt, total_T, N, H};
+  const size_t smem = sizeof(BwdSmem);
+  auto kern = bf16 ? kda_bwd_kernel<__nv_bfloat16> : kda_bwd_kernel<float>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  // persistent grid: as many 4-CTA clusters as are resident at once (a cluster must fit in
+  // one GPC, so fewer than 148 / 4), each taking chains in turn
+  int resident = 0;
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(kBMaxClusters * kBSlices);
+    cfg.blockDim = dim3(kBThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = kBSlices;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&resident, kern, &cfg) != cudaSuccess || resident < 1) {
+      (void)cudaGetLastError();
+      resident = 1;
+    }
+  }
   const int64_t chains = static_cast<int64_t>(N) * H;
-  const unsigned grid = static_cast<unsigned>(chains < kBwdMaxCtas ? chains : kBwdMaxCtas);
-  if (bf16)
-    kda_bwd_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a);
-  else
-    kda_bwd_kernel<float><<<grid, 256, 0, stream>>>(a);
+  const int64_t cap = resident < kBMaxClusters ? resident : kBMaxClusters;
+  const unsigned clusters = static_cast<unsigned>(chains < cap ? chains : cap);
+  kern<<<clusters * kBSlices, kBThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 

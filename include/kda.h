@@ -305,9 +305,8 @@ KDA_API kda_status kda_mixer_fwd_noalloc(const void* q_raw, const void* k_raw, c
 
 /*
  * Workspace for kda_chunk_bwd (bytes, multiple of 256; 0 for rejected sizes): the
- * status word, a checkpoint of the state every 16 tokens (64 KB per 16 tokens and
- * head, e.g. 545 MB for one 4096-token sequence of 32 heads) and 1 MB of scratch for
- * each of min(N * H, 148) CTAs.
+ * status word and a checkpoint of the state every 8 tokens (64 KB per 8 tokens and
+ * head, e.g. 1.09 GB for one 4096-token sequence of 32 heads).
  */
 KDA_API size_t kda_chunk_bwd_workspace(int64_t total_T, int N, int H, int dk, int dv);
 
@@ -321,7 +320,8 @@ KDA_API size_t kda_chunk_bwd_workspace(int64_t total_T, int N, int H, int dk, in
  *     G += q do^T;  dq = S do;  du = G^T k;  dv = beta du;  dbeta = du . (v - w);
  *     dk = G u - beta P du;  dP = G - beta k du^T;
  *     dlog_alpha_i = sum_j dP_ij P_ij;  G <- Diag(alpha) dP.
- * The states are recomputed from checkpoints taken every 16 tokens; arithmetic fp32.
+ * The states are recomputed from checkpoints taken every 8 tokens; arithmetic fp32.
+ * Deterministic: the same inputs give bit-identical gradients.
  *
  *   q, k, v, log_alpha, beta, initial_state, cu_seqlens, total_T, N, H: as for
  *              kda_chunk_fwd (dk == dv == 128 only: KDA_ERR_UNSUPPORTED otherwise).

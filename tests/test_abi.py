@@ -189,14 +189,12 @@ def test_state_affine_rejects_bad_arguments(lib):
 
 
 def test_chunk_bwd_workspace_formula(lib):
-    # status word + plan + one fp32 state per 16 tokens (4 per 64-token chunk bound) and
-    # head + 1 MB (16 states, 16 x 2 vectors) of scratch per CTA, at most 148 CTAs
+    # status word + plan + one fp32 state per 8 tokens (8 per 64-token chunk bound) and head
     def expect(T, N, H):
         plan = -(-(N + 1) * 4 // 256) * 256
         chunks = min(T // 64 + N, T)
-        ckpt = -(-(chunks * 4 * H * 128 * 128 * 4) // 256) * 256
-        scratch = min(N * H, 148) * (16 * 128 * 128 + 16 * 2 * 128) * 4
-        return 256 + plan + ckpt + scratch
+        ckpt = -(-(chunks * 8 * H * 128 * 128 * 4) // 256) * 256
+        return 256 + plan + ckpt
     assert lib.kda_chunk_bwd_workspace(0, 3, 2, 128, 128) == 256 + 256   # status + plan only
     for T, N, H in [(4096, 1, 32), (300, 5, 2), (1, 1, 1), (262144, 64, 32)]:
         assert lib.kda_chunk_bwd_workspace(T, N, H, 128, 128) == expect(T, N, H)

@@ -1,5 +1,5 @@
 """kda_chunk_bwd (gradients of the recurrence) through the C ABI against the oracle's
-kda_backward, on packed sequences that span several 16-token checkpoint intervals with
+kda_backward, on packed sequences that span several 8-token checkpoint intervals with
 ragged tails, an empty and a one-token sequence, fp32 and bf16 inputs, with and without
 the initial state and the final state's gradient; and, at the model shape (one
 4096-token sequence of 32 heads), on sampled heads, which the oracle computes alone
@@ -65,7 +65,7 @@ def test_backward_equal_lengths_without_states(kda):
 
 
 def test_backward_many_chains_persistent_grid(kda):
-    # more (sequence, head) chains than the 148 CTAs of the persistent grid
+    # more (sequence, head) chains than the 37 four-CTA clusters of the persistent grid
     w = I.make_prefill([20] * 40, 4, 128, 128, seed=I.SEED_BASE + 64)
     d_out, d_final = I.make_cotangents(w.total_T, w.N, 4, 128, seed=I.SEED_BASE + 65)
     got = _gpu(kda, w, d_out, d_final)
