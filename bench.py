@@ -96,16 +96,19 @@ def load_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+# The sources the headline call's kernels (plan, intra-chunk, recurrence) are compiled from.
+HEADLINE_KERNEL_SOURCES = ("kda_split.cu", "kda_tile.cuh", "sm100_ptx.cuh")
+
+
 def kernel_sources_sha256() -> str:
-    """Hash of the CUDA sources (csrc/*.cu, *.cuh, *.h, sorted by name): identifies the
-    kernels an ncu traffic figure was captured from."""
+    """Hash of the headline call's kernel sources (HEADLINE_KERNEL_SOURCES, in that order):
+    identifies the kernels an ncu traffic figure was captured from."""
     import hashlib
     csrc = os.path.join(ROOT, "gated_delta_rule_137_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(name.encode())
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    for name in HEADLINE_KERNEL_SOURCES:
+        h.update(name.encode())
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()
 
 

@@ -20,7 +20,8 @@
 // recomputes one from its checkpoint (keeping the state before each of its tokens, and
 // u and v - w, in shared memory) and walks its tokens backwards. Per token the inputs of
 // the next token are fetched while the current one computes (two buffers in shared
-// memory), so a token costs two block barriers and no exposed global load.
+// memory), from L2: each stretch's inputs, and in pass 2 its checkpoint, are prefetched
+// into L2 one stretch ahead.
 //
 // Thread layout: 256 threads, warp w holds state rows 16w..16w+15, lane l column l of
 // the slice. Column sums (over rows) go through shared memory across the 8 warps; row
@@ -30,6 +31,7 @@
 #include <cuda_runtime.h>
 
 #include "kda_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -141,6 +143,33 @@ __device__ __forceinline__ void publish_token(BwdSmem& s, int b, const TokRegs& 
   }
 }
 
+// Brings a stretch's token inputs into L2 ahead of use (the rows are read from HBM
+// otherwise, one token ahead, which does not cover the latency): per token the k, log
+// alpha (and, for pass 2, q) rows of the head, this slice's 32 columns of v (and d_out),
+// and beta.
+template <typename TIn, bool kAll>
+__device__ __forceinline__ void prefetch_stretch(const BwdArgs& a, int64_t t0, int len, int h, int c0, int tid) {
+  if (tid >= kBStretch * 6) return;
+  const int i = tid / 6, which = tid % 6;
+  if (i >= len) return;
+  const size_t tok = static_cast<size_t>(t0 + i) * a.H + h;
+  const size_t o = tok * kBD;
+  switch (which) {
+    case 0: bulk_prefetch_l2(static_cast<const TIn*>(a.k) + o, kBD * sizeof(TIn)); break;
+    case 1: bulk_prefetch_l2(a.log_alpha + o, kBD * sizeof(float)); break;
+    case 2: bulk_prefetch_l2(static_cast<const TIn*>(a.v) + o + c0, kBCols * sizeof(TIn)); break;
+    case 3: asm volatile("prefetch.global.L2 [%0];" ::"l"(a.beta + tok)); break;
+    case 4: if (kAll) bulk_prefetch_l2(static_cast<const TIn*>(a.q) + o, kBD * sizeof(TIn)); break;
+    default: if (kAll) bulk_prefetch_l2(static_cast<const TIn*>(a.d_out) + o + c0, kBCols * sizeof(TIn)); break;
+  }
+}
+
+// Brings this slice's 128 x 32 block of a checkpoint into L2 (one 128-byte row segment
+// per thread of the upper half of the CTA). `state` is the checkpoint's [128][128] base.
+__device__ __forceinline__ void prefetch_ckpt(const float* state, int c0, int tid) {
+  if (tid >= kBD) bulk_prefetch_l2(state + static_cast<size_t>(tid - kBD) * kBD + c0, kBCols * sizeof(float));
+}
+
 template <typename TIn>
 __global__ void __cluster_dims__(kBSlices, 1, 1) __launch_bounds__(kBThreads, 1) kda_bwd_kernel(const BwdArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -218,12 +247,17 @@ __global__ void __cluster_dims__(kBSlices, 1, 1) __launch_bounds__(kBThreads, 1)
       publish_token<false>(s, b, fetch_token<TIn, false>(a, bos, h, c0, tid), tid);
       __syncthreads();
     }
+    if (nst > 0) prefetch_stretch<TIn, false>(a, bos, nst > 1 ? kBStretch : static_cast<int>(eos - bos), h, c0, tid);
     for (int c = 0; c < nst; ++c) {
       float* ck = ckpt_of(c);
 #pragma unroll
       for (int r = 0; r < kBRows; ++r) ck[(row0 + r) * kBD] = S[r];
       const int64_t t0 = bos + static_cast<int64_t>(c) * kBStretch;
       const int len = static_cast<int>(eos - t0 < kBStretch ? eos - t0 : kBStretch);
+      if (c + 1 < nst) {  // the next stretch (the last may be partial)
+        const int64_t t1 = t0 + kBStretch;
+        prefetch_stretch<TIn, false>(a, t1, static_cast<int>(eos - t1 < kBStretch ? eos - t1 : kBStretch), h, c0, tid);
+      }
       for (int i = 0; i < len; ++i) {
         const int64_t tn = t0 + i + 1;
         TokRegs nx{};
@@ -247,12 +281,20 @@ __global__ void __cluster_dims__(kBSlices, 1, 1) __launch_bounds__(kBThreads, 1)
       publish_token<true>(s, b, fetch_token<TIn, true>(a, t0, h, c0, tid), tid);
       __syncthreads();
     }
+    if (nst > 0) {
+      const int64_t tl = bos + static_cast<int64_t>(nst - 1) * kBStretch;
+      prefetch_stretch<TIn, true>(a, tl, static_cast<int>(eos - tl), h, c0, tid);
+    }
     for (int c = nst - 1; c >= 0; --c) {
       const float* ck = ckpt_of(c);
 #pragma unroll
       for (int r = 0; r < kBRows; ++r) S[r] = ck[(row0 + r) * kBD];
       const int64_t t0 = bos + static_cast<int64_t>(c) * kBStretch;
       const int len = static_cast<int>(eos - t0 < kBStretch ? eos - t0 : kBStretch);
+      if (c > 0) {  // the stretch before (full) and its checkpoint, used after this one
+        prefetch_stretch<TIn, true>(a, t0 - kBStretch, kBStretch, h, c0, tid);
+        prefetch_ckpt(a.ckpt + (static_cast<size_t>(cbase + c - 1) * H + h) * kBD * kBD, c0, tid);
+      }
       // recompute tokens t0 .. t0 + len - 1; the last one's inputs stay in their buffer,
       // since the backward walk starts with the same token
       for (int i = 0; i < len; ++i) {
