@@ -99,3 +99,12 @@ def test_mixer_decode_tokens_work_figure():
     assert bench.mixer_decode_tokens_bytes(256, 1) == bench.mixer_decode_bytes(256)
     per_token = 5 * 128 * 2 + 128 * 4 + 4
     assert bench.mixer_decode_tokens_bytes(256, 4) - bench.mixer_decode_tokens_bytes(256, 1) == 256 * 32 * 3 * per_token
+
+
+def test_backward_work_figure():
+    # per token-head: q, k, v, d_out bf16 and log_alpha fp32 + beta read; dq, dk, dv,
+    # d_log_alpha fp32 + d_beta written; per chain: initial state, d_final read, d_initial written
+    per_tok = 4 * 128 * 2 + 128 * 4 + 4 + 4 * 128 * 4 + 4
+    assert per_tok == 3592
+    assert bench.backward_bytes(4096, 1) == 4096 * 32 * per_tok + 3 * 32 * 128 * 128 * 4
+    assert bench.backward_bytes(0, 2) == 3 * 2 * 32 * 128 * 128 * 4

@@ -448,3 +448,31 @@ def test_backward_matches_finite_differences():
             xm[which][i] -= eps
             num[i] = (loss(*xp) - loss(*xm)) / (2 * eps)
         np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7, err_msg=f"gradient {which}")
+
+
+def test_backward_closed_form_without_writes():
+    """With beta = 0 and alpha = 1 nothing is written: S_t = S0 for every token, so
+    o_t = S0^T q_t and, with G_t = d_final + sum_{s >= t} q_s do_s^T (the gradient of the
+    state after token t), the gradients have closed forms: dq_t = S0 do_t, dk = dv = 0,
+    dS0 = G_first, dbeta_t = (G_t^T k_t) . (v_t - S0^T k_t), dlog_alpha_t,i =
+    sum_j (G_t)_ij (S0)_ij."""
+    rng = np.random.default_rng(137107)
+    T, H, dk, dv = 6, 2, 4, 3
+    q, k = rng.standard_normal((T, H, dk)), rng.standard_normal((T, H, dk))
+    v = rng.standard_normal((T, H, dv))
+    do = rng.standard_normal((T, H, dv))
+    s0 = rng.standard_normal((1, H, dk, dv))
+    df = rng.standard_normal((1, H, dk, dv))
+    la, b = np.zeros((T, H, dk)), np.zeros((T, H))
+    dq, dkk, dvv, dla, db, ds0 = O.kda_backward(q, k, v, la, b, s0, [0, T], do, df)
+    S = s0[0]
+    for h in range(H):
+        G = df[0, h].copy()
+        for t in range(T - 1, -1, -1):
+            G = G + np.outer(q[t, h], do[t, h])
+            np.testing.assert_allclose(dq[t, h], S[h] @ do[t, h], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(db[t, h], (G.T @ k[t, h]) @ (v[t, h] - S[h].T @ k[t, h]), rtol=1e-12,
+                                       atol=1e-12)
+            np.testing.assert_allclose(dla[t, h], np.sum(G * S[h], axis=1), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(ds0[0, h], G, rtol=1e-12, atol=1e-12)
+    assert np.all(dkk == 0) and np.all(dvv == 0)
