@@ -102,7 +102,7 @@ def test_mixer_decode_tokens_work_figure():
 
 
 def test_backward_work_figure():
-    bench = _bench()
+    import bench
     # per token-head: q, k, v, d_out bf16 and log_alpha fp32 + beta read; dq, dk, dv,
     # d_log_alpha fp32 + d_beta written; per chain: initial state, d_final read, d_initial written
     per_tok = 4 * 128 * 2 + 128 * 4 + 4 + 4 * 128 * 4 + 4
