@@ -467,6 +467,27 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, kda_dtype 
     return fail(KDA_ERR_INVALID_ARG, "beta and d_beta must be 4-byte aligned");
   if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
     return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+  {  // the gradients are written while the inputs are read: no output may overlap any
+     // input or another output
+    const size_t es = elem_size(qkv_dtype);
+    const size_t tok = static_cast<size_t>(total_T) * H * kda::kD;
+    const size_t n_st = static_cast<size_t>(N) * H * kda::kD * kda::kD * sizeof(float);
+    const size_t n_tb = static_cast<size_t>(total_T) * H * sizeof(float);
+    const void* in[] = {q, k, v, d_out, log_alpha, beta, initial_state, d_final_state, cu_seqlens};
+    const size_t in_n[] = {tok * es, tok * es, tok * es, tok * es, tok * 4, n_tb, n_st, n_st,
+                           (static_cast<size_t>(N) + 1) * sizeof(int32_t)};
+    const void* outp[] = {dq, dk_out, dv_out, d_log_alpha, d_beta, d_initial_state};
+    const size_t out_n[] = {tok * 4, tok * 4, tok * 4, tok * 4, n_tb, n_st};
+    const char* out_names[] = {"dq", "dk", "dv", "d_log_alpha", "d_beta", "d_initial_state"};
+    for (int i = 0; i < 6; ++i) {
+      for (int j = 0; j < 9; ++j)
+        if (ranges_overlap(outp[i], out_n[i], in[j], in_n[j]))
+          return fail(KDA_ERR_INVALID_ARG, "%s overlaps an input", out_names[i]);
+      for (int j = i + 1; j < 6; ++j)
+        if (ranges_overlap(outp[i], out_n[i], outp[j], out_n[j]))
+          return fail(KDA_ERR_INVALID_ARG, "%s overlaps %s", out_names[i], out_names[j]);
+    }
+  }
   const size_t need = kda_chunk_bwd_workspace(total_T, N, H, dk, dv);
   if (!workspace || workspace_bytes < need)
     return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? workspace_bytes : 0, need);

@@ -204,18 +204,39 @@ def test_chunk_bwd_workspace_formula(lib):
 
 def test_chunk_bwd_rejects_bad_arguments(lib):
     ws = lib.kda_chunk_bwd_workspace(128, 2, 2, 128, 128)
-    f = FAKE
+    # disjoint 16-byte aligned fake ranges, 1 MiB apart (each tensor here is < 1 MiB)
+    f = [0x10000000 + i * (1 << 20) for i in range(16)]
 
-    def call(q=f, la=f * 2, beta=f * 3, d_out=f * 4, dq=f * 5, dbeta=f * 6, cu=None, T=128, N=2, dk=128,
+    def call(q=f[0], la=f[1], beta=f[2], d_out=f[3], dq=f[4], dbeta=f[5], cu=None, T=128, N=2, dk=128,
              ws_bytes=ws, dtype=kda.KDA_DT_BF16):
-        return lib.kda_chunk_bwd(q, f, f, dtype, la, beta, None, cu, T, N, 2, dk, 128, d_out, None, dq, f, f, f,
-                                 dbeta, None, f * 7, ws_bytes, None)
+        return lib.kda_chunk_bwd(q, f[6], f[7], dtype, la, beta, None, cu, T, N, 2, dk, 128, d_out, None, dq, f[8],
+                                 f[9], f[10], dbeta, None, f[11], ws_bytes, None)
     assert call(dk=64) == kda.KDA_ERR_UNSUPPORTED
     assert call(dtype=7) == kda.KDA_ERR_INVALID_ARG
     assert call(d_out=None) == kda.KDA_ERR_INVALID_ARG
     assert call(dbeta=None) == kda.KDA_ERR_INVALID_ARG
-    assert call(q=f + 8) == kda.KDA_ERR_INVALID_ARG            # misaligned
-    assert call(beta=f + 2) == kda.KDA_ERR_INVALID_ARG         # beta needs 4-byte alignment
+    assert call(q=f[0] + 8) == kda.KDA_ERR_INVALID_ARG         # misaligned
+    assert call(beta=f[2] + 2) == kda.KDA_ERR_INVALID_ARG      # beta needs 4-byte alignment
     assert call(T=129) == kda.KDA_ERR_INVALID_ARG              # not a multiple of N without cu_seqlens
     assert call(ws_bytes=ws - 256) == kda.KDA_ERR_WORKSPACE
     assert call(T=0, N=0) == kda.KDA_OK                        # empty batch: nothing to do
+
+
+def test_chunk_bwd_rejects_overlapping_outputs(lib):
+    T, N, H = 64, 1, 2
+    tok = T * H * 128
+    ws = lib.kda_chunk_bwd_workspace(T, N, H, 128, 128)
+    # disjoint 16-byte aligned fake ranges, 1 MiB apart (each tensor here is < 1 MiB)
+    base = [0x10000000 + i * (1 << 20) for i in range(16)]
+    q, k, v, la, beta, dout, dq, dk, dv, dla, dbeta, wsp = base[:12]
+
+    def call(**kw):
+        a = dict(q=q, k=k, v=v, la=la, beta=beta, dout=dout, dq=dq, dk=dk, dv=dv, dla=dla, dbeta=dbeta)
+        a.update(kw)
+        return lib.kda_chunk_bwd(a["q"], a["k"], a["v"], kda.KDA_DT_BF16, a["la"], a["beta"], None, None, T, N, H,
+                                 128, 128, a["dout"], None, a["dq"], a["dk"], a["dv"], a["dla"], a["dbeta"], None,
+                                 wsp, ws, None)
+    assert call(dq=q) == kda.KDA_ERR_INVALID_ARG                  # an output on an input
+    assert call(dla=la + 16 * (tok // 8)) == kda.KDA_ERR_INVALID_ARG  # partly inside log_alpha
+    assert call(dk=dq) == kda.KDA_ERR_INVALID_ARG                 # two outputs on each other
+    assert call(dbeta=dv + 256) == kda.KDA_ERR_INVALID_ARG
