@@ -179,6 +179,106 @@ def kda_chunked(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, c
     return out, final
 
 
+def kda_chunked_backward(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_out, d_final=None,
+                         chunk: int = 64):
+    """The gradients of kda_backward, computed through the chunk-parallel rewrite of
+    kda_chunked (a blueprint for a tensor-core backward: per chunk only GEMMs, a
+    triangular inverse and elementwise work, and one state gradient carried between
+    chunks). The forward of one chunk (per head, pairwise decay D[r,i,c] =
+    exp(g[r,c] - g[i,c]) for i <= r) is
+      KK = sum_c K[r,c] K[i,c] D,  QK = sum_c Q[r,c] K[i,c] D,
+      A = Diag(beta) strict(KK),  P = incl(QK),  M = (I + A)^-1,  T = M Diag(beta),
+      W = T (K e^g),  U~ = T V,  U = U~ - W S,  O = (Q e^g) S + P U,
+      S' = Diag(e^g_last) S + Kdec^T U,  Kdec = K e^(g_last - g).
+    Its reverse, given dO and dS' (the next chunk's dS, or d_final):
+      dU = P^T dO + Kdec dS';  dS = (Q e^g)^T dO + Diag(e^g_last) dS' - W^T dU;
+      dP = incl(dO U^T);  dW = -dU S^T;  dT = dW (K e^g)^T + dU V^T;
+      d(K e^g) = T^T dW;  dV = T^T dU;  dM = dT Diag(beta);  dbeta_i += sum_r M[r,i] dT[r,i];
+      dA = strict(-M^T dM M^T);  dbeta_r += sum_i dA[r,i] KK[r,i];  dKK = Diag(beta) dA;
+    then through the products of K, Q, e^g and D to dK, dQ and dg, and
+    dlog_alpha = the reverse running sum of dg within the chunk.
+    """
+    q, k, v, la, b = _f64(q), _f64(k), _f64(v), _f64(log_alpha), _f64(beta)
+    do = _f64(d_out)
+    TT, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    N = len(cu) - 1
+    S0 = np.zeros((N, H, dk, dv)) if initial_state is None else _f64(initial_state)
+    dq, dkk, dvv, dla, db = (np.zeros_like(x) for x in (q, k, v, la, b))
+    dS0 = np.zeros_like(S0)
+    for n in range(N):
+        starts = list(range(cu[n], cu[n + 1], chunk))
+        # forward: the state at the start of every chunk
+        S_at, S = [], S0[n].copy()
+        for s in starts:
+            e = min(s + chunk, cu[n + 1])
+            S_at.append(S)
+            _, S = kda_chunked(q[s:e], k[s:e], v[s:e], la[s:e], b[s:e], S[None], [0, e - s], chunk=chunk)
+            S = S[0]
+        dS = np.zeros((H, dk, dv)) if d_final is None else _f64(d_final)[n].copy()
+        for s, S in zip(reversed(starts), reversed(S_at)):
+            e = min(s + chunk, cu[n + 1])
+            L = e - s
+            Q, K = q[s:e].transpose(1, 0, 2), k[s:e].transpose(1, 0, 2)     # [H, L, dk]
+            V, dO = v[s:e].transpose(1, 0, 2), do[s:e].transpose(1, 0, 2)   # [H, L, dv]
+            be = b[s:e].T                                                   # [H, L]
+            g = np.cumsum(la[s:e].transpose(1, 0, 2), axis=1)              # [H, L, dk]
+            strict = np.tril(np.ones((L, L), dtype=bool), -1)
+            incl = np.tril(np.ones((L, L), dtype=bool), 0)
+            diff = g[:, :, None, :] - g[:, None, :, :]
+            D = np.where(incl[None, :, :, None], np.exp(np.where(incl[None, :, :, None], diff, 0.0)), 0.0)
+            KK = np.einsum("hrc,hic,hric->hri", K, K, D)
+            QK = np.einsum("hrc,hic,hric->hri", Q, K, D)
+            A = be[:, :, None] * np.where(strict, KK, 0.0)
+            P = np.where(incl, QK, 0.0)
+            eye = np.eye(L)
+            M = np.linalg.solve(eye[None] + A, np.broadcast_to(eye, (H, L, L)))
+            T = M * be[:, None, :]
+            Gam = np.exp(g)
+            Kt, Qt = K * Gam, Q * Gam
+            W, Ut = T @ Kt, T @ V
+            U = Ut - W @ S
+            gl = g[:, -1, :]                                                # [H, dk]
+            gam = np.exp(gl)
+            Ed = np.exp(gl[:, None, :] - g)                                 # [H, L, dk]
+            Kdec = K * Ed
+            Tt = lambda x: x.transpose(0, 2, 1)
+            # reverse of O = Qt S + P U and S' = Diag(gam) S + Kdec^T U
+            dU = Tt(P) @ dO + Kdec @ dS
+            dS_prev = Tt(Qt) @ dO + gam[:, :, None] * dS - Tt(W) @ dU
+            dP = np.where(incl, dO @ Tt(U), 0.0)
+            dQt = dO @ Tt(S)
+            dKdec = U @ Tt(dS)
+            dgam = np.sum(dS * S, axis=2)                                   # [H, dk]
+            # reverse of U = U~ - W S, W = T Kt, U~ = T V
+            dW = -dU @ Tt(S)
+            dT = dW @ Tt(Kt) + dU @ Tt(V)
+            dKt = Tt(T) @ dW
+            dV = Tt(T) @ dU
+            # reverse of T = M Diag(beta), M = (I + A)^-1, A = Diag(beta) strict(KK)
+            dM = dT * be[:, None, :]
+            dbe = np.sum(M * dT, axis=1)                                    # over r: [H, i]
+            dA = np.where(strict, -Tt(M) @ dM @ Tt(M), 0.0)
+            dbe = dbe + np.sum(dA * KK, axis=2)                             # over i: [H, r]
+            dKK = be[:, :, None] * dA
+            # reverse of KK, QK (pairwise decay) and of the e^g, Kdec products
+            dQ = dQt * Gam + np.einsum("hri,hic,hric->hrc", dP, K, D)
+            dK = (dKt * Gam + dKdec * Ed + np.einsum("hri,hic,hric->hrc", dKK, K, D)
+                  + np.einsum("hri,hrc,hric->hic", dKK, K, D) + np.einsum("hri,hrc,hric->hic", dP, Q, D))
+            dD = dKK[:, :, :, None] * K[:, :, None, :] * K[:, None, :, :] + \
+                dP[:, :, :, None] * Q[:, :, None, :] * K[:, None, :, :]
+            dDD = dD * D
+            dg = dQt * Qt + dKt * Kt - dKdec * Kdec + np.sum(dDD, axis=2) - np.sum(dDD, axis=1)
+            dg[:, -1, :] += np.sum(dKdec * Kdec, axis=1) + dgam * gam
+            dla_c = np.cumsum(dg[:, ::-1, :], axis=1)[:, ::-1, :]          # reverse running sum
+            dq[s:e], dkk[s:e], dvv[s:e] = dQ.transpose(1, 0, 2), dK.transpose(1, 0, 2), dV.transpose(1, 0, 2)
+            dla[s:e], db[s:e] = dla_c.transpose(1, 0, 2), dbe.T
+            dS = dS_prev
+        dS0[n] = dS
+    return dq, dkk, dvv, dla, db, dS0
+
+
 def short_conv(x, w, cu_seqlens) -> np.ndarray:
     """Causal depthwise convolution of width 4 on packed [sum_T, C] channels.
 

@@ -476,3 +476,25 @@ def test_backward_closed_form_without_writes():
             np.testing.assert_allclose(dla[t, h], np.sum(G * S[h], axis=1), rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(ds0[0, h], G, rtol=1e-12, atol=1e-12)
     assert np.all(dkk == 0) and np.all(dvv == 0)
+
+
+@pytest.mark.parametrize("lens,chunk", [([9, 4, 0, 13], 4), ([70, 5, 64], 64)])
+def test_chunked_backward_matches_the_token_backward(lens, chunk):
+    """kda_chunked_backward (the chunk-parallel form: GEMMs, a triangular inverse and a
+    reverse running sum per chunk) against kda_backward (one token at a time): partial
+    and full chunks, an empty sequence, initial states and a final-state gradient."""
+    rng = np.random.default_rng(137108 + chunk)
+    H, dk, dv = 2, 5, 3
+    TT = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    q, k = rng.standard_normal((TT, H, dk)), rng.standard_normal((TT, H, dk))
+    v = rng.standard_normal((TT, H, dv))
+    la = -np.log1p(np.exp(rng.standard_normal((TT, H, dk)))) / 4
+    b = 1 / (1 + np.exp(-rng.standard_normal((TT, H))))
+    s0 = rng.standard_normal((len(lens), H, dk, dv)) * 0.3
+    do = rng.standard_normal((TT, H, dv))
+    df = rng.standard_normal((len(lens), H, dk, dv))
+    ref = O.kda_backward(q, k, v, la, b, s0, cu, do, df)
+    got = O.kda_chunked_backward(q, k, v, la, b, s0, cu, do, df, chunk=chunk)
+    for name, r, g in zip(("dq", "dk", "dv", "dla", "dbeta", "dS0"), ref, got):
+        np.testing.assert_allclose(g, r, rtol=0, atol=1e-10 * np.max(np.abs(r)), err_msg=name)
