@@ -703,6 +703,32 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_profile_case(args):
+    """A mid-size single-pass prefill for kernel captures: 8 packed sequences x 4096
+    tokens x 32 heads (256 chains, so the single-pass kernel; 1.6 GB of inputs, above L2),
+    W + K calls, then one line with the CUDA-event time per call."""
+    import torch
+    import gated_delta_rule_137_b200 as kda
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(device)
+    kda.load_library()
+    n, T = 8, 4096
+    x = device_prefill_inputs(n * T, H, D, 1370010, device, state_N=n)
+    out = torch.empty(n * T, H, D, dtype=torch.bfloat16, device=device)
+    fin = torch.empty(n, H, D, D, dtype=torch.float32, device=device)
+    ws = torch.empty(max(256, kda.chunk_fwd_workspace_bytes(n * T, n, H, D, D, kda.KDA_DT_BF16)), dtype=torch.uint8,
+                     device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def call(i):
+        kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"], None, N=n, out=out,
+                      final_state=fin, workspace=ws, stream=stream)
+
+    per, tot = time_region(call, args.steps, args.warmup, stream, device)
+    print(json.dumps({"case": f"single-pass prefill {n} x {T} tokens, H={H} d={D}", "ms_per_call": tot / args.steps,
+                      "bytes_per_call": prefill_bytes(n * T, n)}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -712,6 +738,8 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="headline and decode only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=32)
+    ap.add_argument("--profile-case", action="store_true",
+                    help="only a mid-size single-pass prefill (8 x 4096 tokens, 32 heads), for kernel captures")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per headline call to report instead of profiles/traffic.json")
     args = ap.parse_args(argv)
@@ -719,6 +747,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.profile_case:
+        run_profile_case(args)
     else:
         run_gpu(args)
 
