@@ -45,6 +45,14 @@ What it computes (all in float64, from the exact input values upcast):
 * ``kda_mixer_decode_tokens`` — K consecutive tokens per sequence through
   ``kda_mixer_decode_step``, keeping the state and history after every token (the
   checkpoints a speculative decoder rolls back to when it accepts fewer tokens).
+* ``kda_chunked_backward`` — the same gradients as ``kda_backward`` through the
+  chunk-parallel rewrite of ``kda_chunked`` (each chunk's forward reversed step by
+  step); a self-check of the algebra a chunked backward kernel would follow, equal
+  to ``kda_backward`` to rounding.
+
+Each function is pinned by tests that do not restate it: closed forms, special
+cases that reduce to a textbook computation, finite differences, and the agreement
+of two independent formulations (token and chunk).
 
 Readings where the pages are silent (the full list is kept with the design
 notes): no 1/sqrt(d_k) query scale; log_alpha is given directly (natural log,
