@@ -82,3 +82,35 @@ def test_backward_model_shape_sampled_heads(kda):
         ref = O.kda_backward(w.q[:, sl], w.k[:, sl], w.v[:, sl], w.log_alpha[:, sl], w.beta[:, sl],
                              w.initial_state[:, sl], w.cu_seqlens, d_out[:, sl], d_final[:, sl])
         _check([g[:, sl] for g in got], ref)
+
+
+def test_backward_of_only_empty_sequences(kda):
+    # no tokens at all: the initial state's gradient is the final state's, exactly
+    import torch
+    H = 2
+    z = lambda dt: torch.empty((0, H, 128), dtype=dt, device="cuda")
+    cu = torch.zeros(4, dtype=torch.int32, device="cuda")
+    d_final = torch.randn(3, H, 128, 128, device="cuda", generator=torch.Generator("cuda").manual_seed(5))
+    s0 = torch.zeros(3, H, 128, 128, device="cuda")
+    grads = kda.chunk_bwd(z(torch.bfloat16), z(torch.bfloat16), z(torch.bfloat16), z(torch.float32),
+                          torch.empty((0, H), device="cuda"), z(torch.bfloat16), s0, cu, d_final, N=3,
+                          check_status=True)
+    torch.cuda.synchronize()
+    assert all(g.numel() == 0 for g in grads[:5])
+    assert torch.equal(grads[5], d_final)
+
+
+def test_backward_flags_bad_seqlens(kda):
+    import torch
+    w = I.make_prefill([100, 100], 2, 128, 128, seed=I.SEED_BASE + 67)
+    d_out, _ = I.make_cotangents(w.total_T, w.N, 2, 128, seed=I.SEED_BASE + 68, final_std=0.0)
+    args = [to_device(x, "bf16") for x in (w.q, w.k, w.v)] + [to_device(w.log_alpha, "f32"),
+                                                             to_device(w.beta, "f32"), to_device(d_out, "bf16")]
+    bad_cu = torch.tensor([0, 150, 120], dtype=torch.int32, device="cuda")  # not monotone, short of total_T
+    with pytest.raises(kda.KdaError):
+        kda.chunk_bwd(*args, None, bad_cu, None, N=2, check_status=True)
+    # a valid call afterwards reports a clean status and matches the oracle
+    got = [to_host(g) for g in kda.chunk_bwd(*args, None, to_device(w.cu_seqlens, "i32"), None, N=2,
+                                              check_status=True)]
+    ref = O.kda_backward(w.q, w.k, w.v, w.log_alpha, w.beta, None, w.cu_seqlens, d_out, None)
+    _check(got, ref)
