@@ -188,7 +188,7 @@ def kda_chunked(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, c
 
 
 def kda_chunked_backward(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_out, d_final=None,
-                         chunk: int = 64):
+                         chunk: int = 64, factorized: bool = False):
     """The gradients of kda_backward, computed through the chunk-parallel rewrite of
     kda_chunked (a blueprint for a tensor-core backward: per chunk only GEMMs, a
     triangular inverse and elementwise work, and one state gradient carried between
@@ -205,6 +205,11 @@ def kda_chunked_backward(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_
       dA = strict(-M^T dM M^T);  dbeta_r += sum_i dA[r,i] KK[r,i];  dKK = Diag(beta) dA;
     then through the products of K, Q, e^g and D to dK, dQ and dg, and
     dlog_alpha = the reverse running sum of dg within the chunk.
+
+    With ``factorized`` the decay-weighted products are taken as a tensor-core kernel
+    would take them, KK = Kt Kh^T and QK = Qt Kh^T with Kt = K e^g, Qt = Q e^g and
+    Kh = K e^-g (finite while a chunk's summed decay stays moderate), and their reverse
+    is dKt += dKK Kh, dQt += dP Kh, dKh = dKK^T Kt + dP^T Qt.
     """
     q, k, v, la, b = _f64(q), _f64(k), _f64(v), _f64(log_alpha), _f64(beta)
     do = _f64(d_out)
@@ -270,14 +275,24 @@ def kda_chunked_backward(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_
             dA = np.where(strict, -Tt(M) @ dM @ Tt(M), 0.0)
             dbe = dbe + np.sum(dA * KK, axis=2)                             # over i: [H, r]
             dKK = be[:, :, None] * dA
-            # reverse of KK, QK (pairwise decay) and of the e^g, Kdec products
-            dQ = dQt * Gam + np.einsum("hri,hic,hric->hrc", dP, K, D)
-            dK = (dKt * Gam + dKdec * Ed + np.einsum("hri,hic,hric->hrc", dKK, K, D)
-                  + np.einsum("hri,hrc,hric->hic", dKK, K, D) + np.einsum("hri,hrc,hric->hic", dP, Q, D))
-            dD = dKK[:, :, :, None] * K[:, :, None, :] * K[:, None, :, :] + \
-                dP[:, :, :, None] * Q[:, :, None, :] * K[:, None, :, :]
-            dDD = dD * D
-            dg = dQt * Qt + dKt * Kt - dKdec * Kdec + np.sum(dDD, axis=2) - np.sum(dDD, axis=1)
+            if factorized:
+                # reverse of KK = Kt Kh^T, QK = Qt Kh^T, then of Kt, Qt, Kh and Kdec
+                Kh = K / Gam
+                dKt = dKt + dKK @ Kh
+                dQt = dQt + dP @ Kh
+                dKh = Tt(dKK) @ Kt + Tt(dP) @ Qt
+                dQ = dQt * Gam
+                dK = dKt * Gam + dKh / Gam + dKdec * Ed
+                dg = dQt * Qt + dKt * Kt - dKh * Kh - dKdec * Kdec
+            else:
+                # reverse of KK, QK (pairwise decay) and of the e^g, Kdec products
+                dQ = dQt * Gam + np.einsum("hri,hic,hric->hrc", dP, K, D)
+                dK = (dKt * Gam + dKdec * Ed + np.einsum("hri,hic,hric->hrc", dKK, K, D)
+                      + np.einsum("hri,hrc,hric->hic", dKK, K, D) + np.einsum("hri,hrc,hric->hic", dP, Q, D))
+                dD = dKK[:, :, :, None] * K[:, :, None, :] * K[:, None, :, :] + \
+                    dP[:, :, :, None] * Q[:, :, None, :] * K[:, None, :, :]
+                dDD = dD * D
+                dg = dQt * Qt + dKt * Kt - dKdec * Kdec + np.sum(dDD, axis=2) - np.sum(dDD, axis=1)
             dg[:, -1, :] += np.sum(dKdec * Kdec, axis=1) + dgam * gam
             dla_c = np.cumsum(dg[:, ::-1, :], axis=1)[:, ::-1, :]          # reverse running sum
             dq[s:e], dkk[s:e], dvv[s:e] = dQ.transpose(1, 0, 2), dK.transpose(1, 0, 2), dV.transpose(1, 0, 2)

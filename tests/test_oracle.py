@@ -478,11 +478,13 @@ def test_backward_closed_form_without_writes():
     assert np.all(dkk == 0) and np.all(dvv == 0)
 
 
+@pytest.mark.parametrize("factorized", [False, True])
 @pytest.mark.parametrize("lens,chunk", [([9, 4, 0, 13], 4), ([70, 5, 64], 64)])
-def test_chunked_backward_matches_the_token_backward(lens, chunk):
+def test_chunked_backward_matches_the_token_backward(lens, chunk, factorized):
     """kda_chunked_backward (the chunk-parallel form: GEMMs, a triangular inverse and a
-    reverse running sum per chunk) against kda_backward (one token at a time): partial
-    and full chunks, an empty sequence, initial states and a final-state gradient."""
+    reverse running sum per chunk; pairwise or factorized decay) against kda_backward
+    (one token at a time): partial and full chunks, an empty sequence, initial states
+    and a final-state gradient."""
     rng = np.random.default_rng(137108 + chunk)
     H, dk, dv = 2, 5, 3
     TT = sum(lens)
@@ -495,6 +497,6 @@ def test_chunked_backward_matches_the_token_backward(lens, chunk):
     do = rng.standard_normal((TT, H, dv))
     df = rng.standard_normal((len(lens), H, dk, dv))
     ref = O.kda_backward(q, k, v, la, b, s0, cu, do, df)
-    got = O.kda_chunked_backward(q, k, v, la, b, s0, cu, do, df, chunk=chunk)
+    got = O.kda_chunked_backward(q, k, v, la, b, s0, cu, do, df, chunk=chunk, factorized=factorized)
     for name, r, g in zip(("dq", "dk", "dv", "dla", "dbeta", "dS0"), ref, got):
         np.testing.assert_allclose(g, r, rtol=0, atol=1e-10 * np.max(np.abs(r)), err_msg=name)
