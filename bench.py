@@ -33,6 +33,9 @@ METRIC = "KDA prefill tokens/s & decode state GB/s at H=32,d=128 (1 B200, % roof
 H, D, T1 = 32, 128, 4096
 CHUNK = 64
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+# The prefill's MMAs are kind::tf32; its peak is the measured bf16 peak times the nominal
+# dense tf32 : bf16 ratio of the B200 (1.1 : 2.25 PFLOP/s).
+TF32_PER_BF16 = 1.1 / 2.25
 
 
 # ----------------------------------------------------------------------------------
@@ -57,8 +60,15 @@ def prefill_bytes(total_T: int, N: int, Hh: int = H, d: int = D, with_h0: bool =
 
 
 def prefill_tc_flops(total_T: int, Hh: int = H, d: int = D, chunk: int = CHUNK) -> int:
-    """Dense tensor-core work per token-head of the chunked form: three d x d state
-    GEMMs (6 d^2) and five chunk-wide GEMMs (10 C d)."""
+    """Tensor-core work the chunked form must do per token-head, triangle-aware: three
+    d x d state GEMMs (6 d^2) and five C-wide GEMMs whose operands are triangular
+    (K Kt^T, Q Kt^T, T K, T V, P U: 5 C d) = 139,264 flops at d = 128, C = 64."""
+    return total_T * Hh * (6 * d * d + 5 * chunk * d)
+
+
+def prefill_tc_flops_issued(total_T: int, Hh: int = H, d: int = D, chunk: int = CHUNK) -> int:
+    """The same GEMMs as the kernels issue them, on dense tiles (10 C d for the C-wide
+    ones) = 180,224 flops per token-head at d = 128, C = 64."""
     return total_T * Hh * (6 * d * d + 10 * chunk * d)
 
 
@@ -639,14 +649,32 @@ def run_gpu(args):
                          "kernel": "kda_chunk_fwd (plan + intra-chunk + recurrence kernels, one call)",
                          "algorithmic_bytes_per_launch": bytes_call,
                          "kernel_us": kern_ms * 1e3, "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({peak_src}, burst copy)",
-                         "tensor": {"achieved_tflops": tc_tflops, "peak_tflops": tc_peak,
-                                    "frac": tc_tflops / tc_peak, "flops_per_launch": prefill_tc_flops(T1)}},
+                         "tensor": {"achieved_tflops": tc_tflops, "flops_per_launch": prefill_tc_flops(T1),
+                                    "flops_count": "triangle-aware, 6 d^2 + 5 C d per token-head",
+                                    "mma_kind": "tf32",
+                                    "peak_tflops_tf32": tc_peak * TF32_PER_BF16,
+                                    "frac_tf32": tc_tflops / (tc_peak * TF32_PER_BF16),
+                                    "peak_tflops_bf16": tc_peak, "frac_bf16": tc_tflops / tc_peak,
+                                    "peak_source": f"MEASURED_PEAKS.json bf16_tflops ({peak_src}, burst) x "
+                                                   f"{TF32_PER_BF16:.3f} (nominal tf32 : bf16)",
+                                    "issued_flops_per_launch": prefill_tc_flops_issued(T1),
+                                    "issued_tflops": prefill_tc_flops_issued(T1) / (kern_ms / 1e3) / 1e12}},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "pipelining": "2 device buffer sets; upload, kernels and download of consecutive steps overlap "
                                   "on three streams; every step's copies are inside the timed region"},
             "decode": decode, "mixer_decode": mdec, "context_parallel": cpar, "mixer": mix, "varlen": var,
             "backward": bwd, "clocks": clocks, "gpu_launches": launches, "cpu_baseline": cpu,
         }
+        # the figures a reader of the line's tail needs, last (a truncated copy keeps them)
+        frac = lambda x: None if x is None else round(x["roofline"]["frac"], 4)
+        line["summary"] = {
+            "prefill_us": round(kern_ms * 1e3, 1), "prefill_frac": round(achieved_gbs / hbm_peak, 4),
+            "decode_us_per_step": round(decode["us_per_step"], 1), "decode_frac": frac(decode),
+            "mixer_decode_frac": frac(mdec), "mixer_ms": None if mix is None else round(mix["ms_per_call"], 3),
+            "mixer_frac": frac(mix), "varlen_ms": None if var is None else round(var["ms_per_call"], 3),
+            "varlen_frac": frac(var), "backward_ms": None if bwd is None else round(bwd["ms_per_call"], 3),
+            "backward_frac": frac(bwd), "e2e_tokens_per_s": round(e2e_value),
+            "tensor_frac_tf32": round(tc_tflops / (tc_peak * TF32_PER_BF16), 4)}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -672,21 +700,40 @@ def oracle_sample(heads: int = 2, T: int = T1):
     return tok_equiv / dt, dt, f"fp64 NumPy oracle, {heads} of {H} heads x {T} tokens of the B=1 T=4096 workload (scaled to all heads)"
 
 
+def oracle_threads():
+    """The oracle runs single-threaded: its contractions are NumPy einsums without BLAS,
+    and any BLAS pool is capped at one thread while it is timed. Returns a context
+    manager for that cap and a record of the host (cores, BLAS pools before the cap)."""
+    import numpy  # noqa: F401  (loads the BLAS the oracle would see)
+    try:
+        from threadpoolctl import threadpool_info, threadpool_limits
+        pools = [{"api": p.get("internal_api"), "threads": p.get("num_threads")} for p in threadpool_info()]
+        cap = threadpool_limits(limits=1)
+    except ImportError:  # pragma: no cover - threadpoolctl ships with the image
+        import contextlib
+        pools, cap = [], contextlib.nullcontext()
+    return cap, {"host_cpu_count": os.cpu_count(), "blas_pools_default": pools, "blas_threads_used": 1}
+
+
 def cpu_baseline(args):
-    v, dt, desc = oracle_sample(heads=args.cpu_heads)
-    return {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc, "seconds": dt}
+    cap, host = oracle_threads()
+    with cap:
+        v, dt, desc = oracle_sample(heads=args.cpu_heads)
+    return {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc, "seconds": dt, **host}
 
 
 def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
         return
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        oracle_sample(heads=1, T=256)
+    cap, host = oracle_threads()
     per = []
-    for _ in range(args.steps):
-        v, dt, desc = oracle_sample(heads=1, T=1024)
-        per.append(dt)
+    with cap:
+        for _ in range(args.warmup if args.warmup < 1 else 1):
+            oracle_sample(heads=1, T=256)
+        for _ in range(args.steps):
+            v, dt, desc = oracle_sample(heads=1, T=1024)
+            per.append(dt)
     total = sum(per)
     tok_equiv = args.steps * 1024 * 1 / H
     value = tok_equiv / total
@@ -698,7 +745,7 @@ def run_reference(args):
         "config": {"workload": "KDA chunked prefill B=1 T=4096 H=32 d_k=d_v=128 (bf16 q/k/v, fp32 log_alpha/beta/state)",
                    "global_batch": 1, "seq_len": T1, "parallelism": "host CPU, 1 core"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": "each step: 1 of 32 heads x the first 1024 tokens (scaled to all heads)"},
+                         "sample": "each step: 1 of 32 heads x the first 1024 tokens (scaled to all heads)", **host},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

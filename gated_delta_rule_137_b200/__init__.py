@@ -30,8 +30,9 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "kda.h")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_RANGE = range(6)
 KDA_DT_F32, KDA_DT_BF16 = 0, 1
 DEVFLAG_BAD_SEQLENS = 0x1
-DEVFLAG_DECAY_RANGE = 0x2
+DEVFLAG_DECAY_RANGE = 0x2  # reserved: no entry point sets it
 DEVFLAG_BAD_INDEX = 0x4
+DEVFLAG_WAIT_TIMEOUT = 0x80000000
 
 _lib = None
 
@@ -59,6 +60,8 @@ _SIGNATURES = {
     "kda_mixer_fwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
                              _vp, _vp, _vp, _sz, _vp]),
     "kda_workspace_status": (_i32, [_vp, _vp, _u32p]),
+    "kda_mixer_fwd_noalloc_status": (_i32, [_vp, _u32p]),
+    "kda_selftest_wait_timeout": (_i32, [_vp, _sz, ctypes.c_uint32, _vp]),
     "kda_mixer_fwd_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
                                      _vp, _vp, _vp]),
     "kda_mixer_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
@@ -347,3 +350,50 @@ def workspace_status(workspace, stream=None) -> int:
     if st == KDA_ERR_RANGE:
         raise KdaError(st, f"device status flags 0x{flags.value:08x}")
     return flags.value
+
+
+def mixer_fwd_noalloc(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate=None, initial_state=None,
+                      cu_seqlens=None, *, N: Optional[int] = None, out=None, final_state=None,
+                      output_final_state: bool = True, stream=None, check_status: bool = False):
+    """Full mixer prefill without a workspace (kda_mixer_fwd_noalloc): the scratch is a
+    fixed array inside the library (total_T * H <= 16384 token-heads)."""
+    torch = _torch()
+    lib = load_library()
+    total_T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    if N is None:
+        if cu_seqlens is None:
+            raise ValueError("N is needed when cu_seqlens is not given")
+        N = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((total_T, H, dv), dtype=torch.bfloat16, device=q_raw.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q_raw.device)
+    _check(lib.kda_mixer_fwd_noalloc(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w), _ptr(log_alpha),
+                                     _ptr(beta), _ptr(gate), _ptr(initial_state), _ptr(cu_seqlens), total_T, N, H,
+                                     dk, dv, _ptr(out), _ptr(final_state), _stream(stream)))
+    if check_status:
+        noalloc_status(stream)
+    return out, final_state
+
+
+def noalloc_status(stream=None) -> int:
+    """Reads and clears the status word of kda_mixer_fwd_noalloc on the current device;
+    raises KdaError(KDA_ERR_RANGE) if a flag was set."""
+    lib = load_library()
+    flags = ctypes.c_uint32(0)
+    st = lib.kda_mixer_fwd_noalloc_status(_stream(stream), ctypes.byref(flags))
+    if st not in (KDA_OK, KDA_ERR_RANGE):
+        _check(st)
+    if st == KDA_ERR_RANGE:
+        raise KdaError(st, f"device status flags 0x{flags.value:08x}")
+    return flags.value
+
+
+def selftest_wait_timeout(workspace, budget_us: int, stream=None) -> None:
+    """Runs the bounded-wait diagnostic (kda_selftest_wait_timeout): one thread waits on
+    an mbarrier that nothing arrives at and gives up after budget_us, setting
+    DEVFLAG_WAIT_TIMEOUT in the workspace's status word (read it with workspace_status)."""
+    lib = load_library()
+    _check(lib.kda_selftest_wait_timeout(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         budget_us, _stream(stream)))

@@ -516,6 +516,39 @@ kda_status kda_workspace_status(void* workspace, kda_stream_t stream_, uint32_t*
 
 }  // extern "C"
 
+namespace {
+// One thread waits on an mbarrier that nothing arrives at, with the library's bounded
+// wait: the wait runs out after budget_ns, raises the timeout bit in *status and the
+// kernel returns.
+__global__ void wait_timeout_probe_kernel(uint32_t* status, uint64_t budget_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    kda::mbar_init(&bar, 1);
+    kda::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) kda::mbar_wait_for(&bar, 0, status, budget_ns);
+  __syncthreads();
+}
+}  // namespace
+
+extern "C" kda_status kda_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t budget_us,
+                                                kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!workspace || workspace_bytes < kda::kStatusBytes)
+    return fail(KDA_ERR_WORKSPACE, "a workspace of at least %zu bytes is needed", kda::kStatusBytes);
+  if (!aligned16(workspace)) return fail(KDA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  if (budget_us < 1 || budget_us > 2000000u)
+    return fail(KDA_ERR_INVALID_ARG, "budget_us=%u must be in [1, 2000000]", budget_us);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status, static_cast<uint64_t>(budget_us) * 1000u);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe kernel launch");
+  return ok();
+}
+
 namespace kda {
 
 // Two-stage form of the full mixer (conv4 + L2 pre-stage into fp32 buffers in

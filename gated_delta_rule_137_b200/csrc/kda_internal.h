@@ -65,7 +65,8 @@ inline int64_t split_max_chunks(int64_t total_T, int N) {
   const int64_t c = total_T / kChunk + N;
   return c < total_T ? c : total_T;
 }
-inline size_t split_plan_bytes(int N) { return align256((static_cast<size_t>(N) + 1) * sizeof(int32_t)); }
+// per-sequence first chunks [N + 1], then one flag: some item was handed over as raw rows
+inline size_t split_plan_bytes(int N) { return align256((static_cast<size_t>(N) + 2) * sizeof(int32_t)); }
 constexpr int64_t kSplitMaxChains = 74;  // half of the 148 SMs: beyond it no slicing is needed
 inline size_t split_workspace_bytes(int64_t total_T, int N, int H, bool any_chains = false) {
   if (total_T <= 0 || N <= 0) return 0;

@@ -21,8 +21,12 @@
 //     next call; the status word is cleared at the start of each call. Calls that
 //     overlap on the GPU (different streams, no ordering between them) race on the
 //     array and give undefined results;
-//   * device-detected range flags are written into the array's status word but
-//     are not reported by this entry point;
+//   * with CUDA's lazy module loading (the default) the first call on a device is
+//     also when the driver loads the library's device code and so reserves the
+//     array; a call with total_T = 0 and N = 0 does that set-up and launches nothing, so it
+//     can serve as a warm-up while the device still has room;
+//   * the device status word (bad cu_seqlens, a wait that ran out of time) lives in
+//     the array too; kda_mixer_fwd_noalloc_status reads and clears it;
 //   * it allocates nothing: no cudaMalloc, cudaFree or allocating library call.
 #include <cstdio>
 #include <mutex>
@@ -72,7 +76,8 @@ extern "C" KDA_API kda_status kda_mixer_fwd_noalloc(const void* q_raw, const voi
                                                     const void* gate, const float* initial_state,
                                                     const int32_t* cu_seqlens, int64_t total_T, int N, int H, int dk,
                                                     int dv, void* out, float* final_state, kda_stream_t stream_) {
-  if (total_T < 0 || H < 1 || total_T * H > kNoallocMaxTokenHeads) {
+  // total_T is bounded on its own first, so that total_T * H cannot overflow
+  if (total_T < 0 || H < 1 || total_T > kNoallocMaxTokenHeads || total_T * H > kNoallocMaxTokenHeads) {
     char msg[256];
     snprintf(msg, sizeof(msg),
              "kda_mixer_fwd_noalloc: total_T * H = %lld exceeds the static scratch capacity of %lld token-heads "
@@ -96,4 +101,27 @@ extern "C" KDA_API kda_status kda_mixer_fwd_noalloc(const void* q_raw, const voi
   // then the recurrence); it computes what kda_mixer_fwd computes, within rounding.
   return kda::mixer_fwd_staged(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, cu_seqlens,
                                total_T, N, H, out, final_state, scratch, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+extern "C" KDA_API kda_status kda_mixer_fwd_noalloc_status(kda_stream_t stream_, uint32_t* flags) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  unsigned char* scratch = nullptr;
+  cudaError_t e = scratch_on_current_device(&scratch);
+  uint32_t word = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(scratch, 0, sizeof(word), stream);
+  if (e != cudaSuccess) {
+    char msg[256];
+    snprintf(msg, sizeof(msg), "kda_mixer_fwd_noalloc_status: %s", cudaGetErrorString(e));
+    return noalloc_fail(KDA_ERR_CUDA, msg);
+  }
+  if (flags) *flags = word;
+  if (word) {
+    char msg[128];
+    snprintf(msg, sizeof(msg), "kda_mixer_fwd_noalloc: device status word 0x%08x", word);
+    return noalloc_fail(KDA_ERR_RANGE, msg);
+  }
+  kda::set_last_error("");
+  return KDA_OK;
 }

@@ -37,8 +37,11 @@
 //   * V arrives by TMA (no multicast) and is widened/transposed to fp32 in shared
 //     memory; q, k, log_alpha, beta are read with coalesced read-only loads by the
 //     thread that owns each key channel.
-// Supported decay range: e^{-g} must stay finite, so the decay summed over one
-// chunk is limited to kMaxChunkDecay nats per channel (status flag otherwise).
+// Decay range: the factorised products need e^{-g} finite, so a chunk whose decay summed
+// over its tokens passes kMaxChunkDecay nats in some key channel is walked token by
+// token instead (walk_chunk: the recurrence itself on the state slice, exact for any
+// decay); kMaxChunkDecay also keeps the tf32 form within its parity bar. Both forms give
+// the same result up to rounding; the walk is slower.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -253,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int64_t t0 = bos; t0 < eos && !failed; t0 += kChunk) {
     const int len = static_cast<int>(eos - t0 < kChunk ? eos - t0 : kChunk);
     const int gnew = gslot ^ 1;  // slot for this chunk's e^{g_last}
+    bool strong;                 // the chunk's decay passes kMaxChunkDecay in some channel
 
     // -- 1. V tile by TMA into the staging area (the TP region, free until step 5) -----
     if (tid == 0) {
@@ -352,44 +356,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 t4 = *reinterpret_cast<const float4*>(sTot + w * kD + c0);
         pre[0] += t4.x; pre[1] += t4.y; pre[2] += t4.z; pre[3] += t4.w;
       }
+      // the chunk's decay per channel decides its form: factorised (e^g, e^-g finite) or
+      // the exact token walk
+      float gl = 0.f;
       if (tid < 128) {
-        float gl = 0.f;
 #pragma unroll
         for (int w = 0; w < 16; ++w) gl += sTot[w * kD + tid];
-        if (-gl > kMaxChunkDecay) atomicOr(a.status, kFlagDecayRange);
-        sGamma[gnew * 128 + tid] = __expf(gl);
       }
-      float kt[4][4], kh[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float qt[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float g = pre[e] + la[i][e];
-          const float eg = __expf(g), eng = __expf(-g);
-          kt[i][e] = kv[i][e] * eg;
-          kh[i][e] = to_tf32(kv[i][e] * eng);
-          qt[e] = qv[i][e] * eg;
-        }
-        const int r = r0 + i;
-        st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[i][0], kt[i][1], kt[i][2], kt[i][3]);    // Kt [tok][ch]
-        st4_tf32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);          // Qt [tok][ch]
-        st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);     // Kh [tok][ch]
-      }
-      // channel-major copies: channel c0+e, tokens r0..r0+3; lanes rotate e so that one
-      // store instruction touches different swizzle rows
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int e = (j + lane) & 3;
-        float x[4], y[4];
+      strong = __syncthreads_or(tid < 128 && -gl > kMaxChunkDecay) != 0;
+      // e^{g_last} scales the state at the next chunk; after a walk the state is exact
+      if (tid < 128) sGamma[gnew * 128 + tid] = strong ? 1.f : __expf(gl);
+      if (strong) {  // k, q (after conv / L2) and the raw log_alpha, row-major, for the walk
+        float* sKr = reinterpret_cast<float*>(sm + SM::kKQ);
+        float* sLAr = reinterpret_cast<float*>(sm + SM::kKH);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          x[i] = e == 0 ? kt[i][0] : e == 1 ? kt[i][1] : e == 2 ? kt[i][2] : kt[i][3];
-          y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
+          const int r = r0 + i;
+          const bool in = r < len;
+          *reinterpret_cast<float4*>(sKr + r * kD + c0) = make_float4(kv[i][0], kv[i][1], kv[i][2], kv[i][3]);
+          *reinterpret_cast<float4*>(sKr + (64 + r) * kD + c0) = make_float4(qv[i][0], qv[i][1], qv[i][2], qv[i][3]);
+          *reinterpret_cast<float4*>(sLAr + r * kD + c0) = in ? la4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        st4_f32(sm + SM::kKTT, f32_offset(c0 + e, r0, 128), x[0], x[1], x[2], x[3]);    // Kt^T [ch][tok]
-        st4_f32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);    // Kh^T [ch][tok]
-      }
+      } else {
+        float kt[4][4], kh[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float qt[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float g = pre[e] + la[i][e];
+            const float eg = __expf(g), eng = __expf(-g);
+            kt[i][e] = kv[i][e] * eg;
+            kh[i][e] = to_tf32(kv[i][e] * eng);
+            qt[e] = qv[i][e] * eg;
+          }
+          const int r = r0 + i;
+          st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[i][0], kt[i][1], kt[i][2], kt[i][3]);    // Kt [tok][ch]
+          st4_tf32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);          // Qt [tok][ch]
+          st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);     // Kh [tok][ch]
+        }
+        // channel-major copies: channel c0+e, tokens r0..r0+3; lanes rotate e so that one
+        // store instruction touches different swizzle rows
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = (j + lane) & 3;
+          float x[4], y[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            x[i] = e == 0 ? kt[i][0] : e == 1 ? kt[i][1] : e == 2 ? kt[i][2] : kt[i][3];
+            y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
+          }
+          st4_f32(sm + SM::kKTT, f32_offset(c0 + e, r0, 128), x[0], x[1], x[2], x[3]);    // Kt^T [ch][tok]
+          st4_f32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);    // Kh^T [ch][tok]
+        }
+      }  // factorised form
     }
 
     // -- 3. V landed: widen/transpose to V^T fp32 (rows past the sequence end -> 0) -------
@@ -418,11 +438,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) x[e] = (t4 + e < len) ? as_f32(st[(t4 + e) * DV + j]) : 0.f;
         }
-        st4_tf32(sm + SM::kVT, f32_offset(j, t4, DV), x[0], x[1], x[2], x[3]);
+        if (strong) {  // the walk reads V row-major in fp32
+          float* vr = reinterpret_cast<float*>(sm + SM::kVT);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) vr[(t4 + e) * DV + j] = x[e];
+        } else {
+          st4_tf32(sm + SM::kVT, f32_offset(j, t4, DV), x[0], x[1], x[2], x[3]);
+        }
       }
     }
     fence_proxy_async_smem();
     __syncthreads();
+
+    // -- a chunk the factorised form cannot carry: the exact token walk on the state slice --
+    if (strong) {
+      WalkArgs wa;
+      wa.sK = reinterpret_cast<const float*>(sm + SM::kKQ);
+      wa.sQ = wa.sK + 64 * kD;
+      wa.sLA = reinterpret_cast<const float*>(sm + SM::kKH);
+      wa.sBeta = sBeta;
+      wa.sV = reinterpret_cast<const float*>(sm + SM::kVT);
+      wa.scr = reinterpret_cast<float*>(sm + SM::kKTT);
+      wa.sST = nullptr;
+      wa.out = outg + static_cast<size_t>(t0) * tok_stride + static_cast<size_t>(h) * kD + col0;
+      wa.gate = gateg ? gateg + static_cast<size_t>(t0) * tok_stride + static_cast<size_t>(h) * kD + col0 : nullptr;
+      wa.out_stride = tok_stride;
+      wa.tmem_state = tmem + lane_off + TM::kD2;
+      wa.scale = sGamma[gslot * 128 + row];  // the true state is e^{g_last}(prev) * D2
+      wa.len = len;
+      walk_chunk<DV, TOut>(wa);
+      if (t0 + kChunk < eos) {  // next chunk's gate inputs
+        const int64_t nt = t0 + kChunk;
+        load_gate(nt, static_cast<int>(eos - nt < kChunk ? eos - nt : kChunk));
+      }
+      gslot = gnew;
+      tc_fence_before_sync();
+      failed = cta_any(lost);
+      tc_fence_after_sync();
+      continue;
+    }
 
     // -- 4. D0 = [A_raw; P_raw] = [Kt; Qt] Kh^T --------------------------------------------
     if (tid == 0) {

@@ -54,6 +54,7 @@ static_assert(kItemGamma + 512 == kItemBytes, "item layout");
 
 struct SplitPlan {
   const int32_t* chunk_start;  // [N + 1]: first global chunk of each sequence; [N] = total (-1: bad seqlens)
+  int32_t* any_raw;            // set by pass 1 when it hands any item over as raw rows (cleared by the plan)
   uint8_t* items;              // [chunks][H] items of kItemBytes
 };
 
@@ -103,6 +104,7 @@ __global__ void __launch_bounds__(1024) kda_plan_kernel(const int32_t* __restric
   }
   if (tid == 0) {
     cs[N] = s_bad ? -1 : s_carry;
+    cs[N + 1] = 0;  // no item handed over as raw rows yet (pass 1 sets it)
     if (s_bad) atomicOr(status, kFlagBadSeqlens);
   }
 }
@@ -137,7 +139,8 @@ struct IntraSmem {
   static constexpr int kBar = kBeta + 512;
   static constexpr int kNumBars = 8;
   static constexpr int kTmemSlot = kBar + 8 * kNumBars;
-  static constexpr int kTotal = kTmemSlot + 16;
+  static constexpr int kStrong = kTmemSlot + 16;     // int [2]: the item is walked token by token
+  static constexpr int kTotal = kStrong + 16;
   static constexpr int kAlloc = kTotal + 1024;
   static_assert(kAlloc <= 232448, "shared memory plan exceeds the per-block limit");
 };
@@ -186,6 +189,125 @@ __device__ __forceinline__ ItemPos item_pos(int64_t it, const PrefillArgs& a, co
   return o;
 }
 
+// ---- raw rows of an item handed to the recurrence's token walk ----------------------
+// Out of line: the rare path, kept away from the register allocation and the
+// instruction footprint of the factorised pass.
+struct RawRowsFront {
+  const void* q;
+  const void* k;
+  const float* log_alpha;
+  const void* a_pre;
+  const float* a_scale;
+  const float* conv_w;
+  uint8_t* item;
+  int64_t t0, bos;
+  int len, h, H, fw;
+};
+// One warp of the front group: chunk rows 8 fw .. 8 fw + 7, lane l = key channels 4l .. 4l+3.
+// Writes k and q (after the conv and L2 norm for the mixer) into the item's [-W; Qt] space
+// as [64][128] fp32 each, and the raw log_alpha into its Kh^T space; rows past the chunk
+// are zero.
+template <typename TIn, bool kConv, bool kPre>
+__device__ __noinline__ void raw_rows_front(const RawRowsFront r) {
+  const int lane = threadIdx.x & 31, c0 = lane * 4;
+  const TIn* qg = static_cast<const TIn*>(r.q);
+  const TIn* kg = static_cast<const TIn*>(r.k);
+  const int64_t ts = static_cast<int64_t>(r.H) * kD;
+  const size_t hc = static_cast<size_t>(r.h) * kD + c0;
+  float* ik = reinterpret_cast<float*>(r.item + kItemQW);
+  float* il = reinterpret_cast<float*>(r.item + kItemKHT);
+  for (int i = 0; i < 8; ++i) {
+    const int t = 8 * r.fw + i;
+    const bool in = t < r.len;  // uniform over the warp
+    float kv[4] = {0.f, 0.f, 0.f, 0.f}, qv[4] = {0.f, 0.f, 0.f, 0.f}, l[4] = {0.f, 0.f, 0.f, 0.f};
+    if (in) {
+      if constexpr (kConv) {  // y = sum_j w[c, j] x[t - 3 + j, c], zero before the sequence start
+        for (int j = 0; j < 4; ++j) {
+          const int64_t tt = r.t0 + t - 3 + j;
+          if (tt < r.bos) continue;
+          float xq[4], xk[4];
+          ld4_in(qg + static_cast<size_t>(tt) * ts + hc, xq);
+          ld4_in(kg + static_cast<size_t>(tt) * ts + hc, xk);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qv[e] = fmaf(__ldg(r.conv_w + ((0 * r.H + r.h) * kD + c0 + e) * 4 + j), xq[e], qv[e]);
+            kv[e] = fmaf(__ldg(r.conv_w + ((1 * r.H + r.h) * kD + c0 + e) * 4 + j), xk[e], kv[e]);
+          }
+        }
+      } else {
+        ld4_in(qg + static_cast<size_t>(r.t0 + t) * ts + hc, qv);
+        ld4_in(kg + static_cast<size_t>(r.t0 + t) * ts + hc, kv);
+      }
+      if constexpr (kPre) {  // log alpha = -scale * softplus(a)
+        const float sc = __ldg(r.a_scale + r.h);
+        float x[4];
+        ld4_in(static_cast<const __nv_bfloat16*>(r.a_pre) + static_cast<size_t>(r.t0 + t) * ts + hc, x);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) l[e] = -sc * (fmaxf(x[e], 0.f) + log1pf(__expf(-fabsf(x[e]))));
+      } else {
+        ld4_in(r.log_alpha + static_cast<size_t>(r.t0 + t) * ts + hc, l);
+      }
+    }
+    if constexpr (kConv) {  // x / sqrt(sum x^2 + 1e-6) over the head's 128 channels (the warp holds them)
+      float sq = 0.f, sk = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        sq = fmaf(qv[e], qv[e], sq);
+        sk = fmaf(kv[e], kv[e], sk);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+      }
+      const float fq = rsqrtf(sq + 1e-6f), fk = rsqrtf(sk + 1e-6f);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qv[e] *= fq;
+        kv[e] *= fk;
+      }
+    }
+    *reinterpret_cast<float4*>(ik + t * kD + c0) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+    *reinterpret_cast<float4*>(ik + (64 + t) * kD + c0) = make_float4(qv[0], qv[1], qv[2], qv[3]);
+    *reinterpret_cast<float4*>(il + t * kD + c0) = make_float4(l[0], l[1], l[2], l[3]);
+  }
+}
+
+struct RawRowsBack {
+  const void* v;
+  const float* conv_w;
+  uint8_t* item;
+  int64_t t0, bos;
+  int len, h, H, btid;
+};
+// The back group (256 threads): v rows (after the conv for the mixer) into the item's U~
+// space as [64][128] fp32; rows past the chunk are zero.
+template <typename TIn, bool kConv>
+__device__ __noinline__ void raw_rows_back(const RawRowsBack r) {
+  const TIn* vh = static_cast<const TIn*>(r.v) + static_cast<size_t>(r.h) * kD;
+  const int64_t ts = static_cast<int64_t>(r.H) * kD;
+  float* iv = reinterpret_cast<float*>(r.item + kItemU);
+  for (int idx = r.btid; idx < kChunk * 32; idx += 256) {  // (token, 4 value columns)
+    const int t = idx >> 5, j4 = 4 * (idx & 31);
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (t < r.len) {
+      if constexpr (kConv) {
+        for (int j = 0; j < 4; ++j) {
+          const int64_t tt = r.t0 + t - 3 + j;
+          if (tt < r.bos) continue;
+          float xv[4];
+          ld4_in(vh + static_cast<size_t>(tt) * ts + j4, xv);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] = fmaf(__ldg(r.conv_w + ((2 * r.H + r.h) * kD + j4 + e) * 4 + j), xv[e], x[e]);
+        }
+      } else {
+        ld4_in(vh + static_cast<size_t>(r.t0 + t) * ts + j4, x);
+      }
+    }
+    *reinterpret_cast<float4*>(iv + t * kD + j4) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+}
+
 // kConv: q, k, v are the raw inputs of the full mixer; the causal depthwise conv of
 // width 4 (zero history at each sequence start) is applied to all three and the L2
 // norm x / sqrt(sum x^2 + 1e-6) to q and k, in fp32, before anything else.
@@ -212,6 +334,7 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
   float* sTot = reinterpret_cast<float*>(sm + SM::kTot);    // [16][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmemSlot);
+  int* sStrong = reinterpret_cast<int*>(sm + SM::kStrong);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -341,137 +464,151 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) pre[1][e] = pre[0][e] + tot[0][e];
+      float gl = 0.f;
       if (ftid < 128) {
-        float gl = 0.f;
 #pragma unroll
         for (int g = 0; g < 16; ++g) gl += sTot[g * kD + ftid];
-        if (-gl > kMaxChunkDecay) atomicOr(a.status, kFlagDecayRange);
-        reinterpret_cast<float*>(item + kItemGamma)[ftid] = __expf(gl);
       }
       if (ftid == 0) bulk_wait_read();  // the previous item's Qt and Kh^T have left KQ and KHT
-      fsync();  // the totals are read: KQ may be written
+      // The totals are read (KQ may be written) and the group votes: a chunk whose decay
+      // passes kMaxChunkDecay in some channel is handed to the recurrence as its raw rows
+      // (k, q after conv / L2, log_alpha, v, beta) and walked there token by token;
+      // e^g_last[0] = -1 marks such an item.
+      const bool strong = group_any(kBarFront, kGroupThreads, ftid < 128 && -gl > kMaxChunkDecay);
+      if (ftid < 128)
+        reinterpret_cast<float*>(item + kItemGamma)[ftid] = strong ? (ftid == 0 ? -1.f : 0.f) : __expf(gl);
+      if (ftid == 0) {
+        sStrong[k & 1] = strong ? 1 : 0;  // for the back group (ordered by kBApFull)
+        if (strong) *p.any_raw = 1;       // the recurrence runs its walking loop
+      }
+      if (strong && ftid < 64) reinterpret_cast<float*>(item + kItemP)[ftid] = sB[ftid];
 
       // -- gate pass B: q, k (conv, L2 norm), Kt, Qt, Kh -----------------------------------
+      if (strong) {  // raw rows for the token walk (out of line: the rare path)
+        RawRowsFront rr{a.q, a.k, a.log_alpha, a.a_pre, a.a_scale, a.conv_w, item, t0, bos, len, h, H, fw};
+        raw_rows_front<TIn, kConv, kPre>(rr);
+      } else {
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        const int r0 = 4 * (2 * fw + s);
-        // q/k row m is chunk row r0 - kHist + m; rows outside [bos, t0 + len) read row t0
-        // (always in bounds) and are replaced by zero where used
-        uint32_t kraw[kGRows][sizeof(TIn)], qraw[kGRows][sizeof(TIn)];
-        bool rin[kGRows];
+        for (int s = 0; s < 2; ++s) {
+          const int r0 = 4 * (2 * fw + s);
+          // q/k row m is chunk row r0 - kHist + m; rows outside [bos, t0 + len) read row t0
+          // (always in bounds) and are replaced by zero where used
+          uint32_t kraw[kGRows][sizeof(TIn)], qraw[kGRows][sizeof(TIn)];
+          bool rin[kGRows];
 #pragma unroll
-        for (int m = 0; m < kGRows; ++m) {
-          const int rr = r0 - kHist + m;
-          rin[m] = rr < len && t0 + rr >= bos;
-          if constexpr (!kConv) {
+          for (int m = 0; m < kGRows; ++m) {
+            const int rr = r0 - kHist + m;
+            rin[m] = rr < len && t0 + rr >= bos;
+            if constexpr (!kConv) {
 #pragma unroll
-            for (int w = 0; w < static_cast<int>(sizeof(TIn)); ++w) {
-              kraw[m][w] = kpre[s][m][w];
-              qraw[m][w] = qpre[s][m][w];
+              for (int w = 0; w < static_cast<int>(sizeof(TIn)); ++w) {
+                kraw[m][w] = kpre[s][m][w];
+                qraw[m][w] = qpre[s][m][w];
+              }
+              continue;
             }
-            continue;
+            const size_t o = static_cast<size_t>(rin[m] ? t0 + rr : t0) * tok_stride + static_cast<size_t>(h) * kD + c0;
+            if constexpr (sizeof(TIn) == 2) {
+              const uint2 kk2 = __ldg(reinterpret_cast<const uint2*>(kg + o));
+              const uint2 qq2 = __ldg(reinterpret_cast<const uint2*>(qg + o));
+              kraw[m][0] = kk2.x; kraw[m][1] = kk2.y; qraw[m][0] = qq2.x; qraw[m][1] = qq2.y;
+            } else {
+              const uint4 kk4 = __ldg(reinterpret_cast<const uint4*>(kg + o));
+              const uint4 qq4 = __ldg(reinterpret_cast<const uint4*>(qg + o));
+              kraw[m][0] = kk4.x; kraw[m][1] = kk4.y; kraw[m][2] = kk4.z; kraw[m][3] = kk4.w;
+              qraw[m][0] = qq4.x; qraw[m][1] = qq4.y; qraw[m][2] = qq4.z; qraw[m][3] = qq4.w;
+            }
           }
-          const size_t o = static_cast<size_t>(rin[m] ? t0 + rr : t0) * tok_stride + static_cast<size_t>(h) * kD + c0;
-          if constexpr (sizeof(TIn) == 2) {
-            const uint2 kk2 = __ldg(reinterpret_cast<const uint2*>(kg + o));
-            const uint2 qq2 = __ldg(reinterpret_cast<const uint2*>(qg + o));
-            kraw[m][0] = kk2.x; kraw[m][1] = kk2.y; qraw[m][0] = qq2.x; qraw[m][1] = qq2.y;
-          } else {
-            const uint4 kk4 = __ldg(reinterpret_cast<const uint4*>(kg + o));
-            const uint4 qq4 = __ldg(reinterpret_cast<const uint4*>(qg + o));
-            kraw[m][0] = kk4.x; kraw[m][1] = kk4.y; kraw[m][2] = kk4.z; kraw[m][3] = kk4.w;
-            qraw[m][0] = qq4.x; qraw[m][1] = qq4.y; qraw[m][2] = qq4.z; qraw[m][3] = qq4.w;
-          }
-        }
-        auto unpack = [&](const uint32_t* w, int e) -> float {
-          if constexpr (sizeof(TIn) == 2) {
-            const uint32_t x = w[e >> 1];
-            return __uint_as_float((e & 1) ? (x & 0xFFFF0000u) : (x << 16));
-          } else {
-            return __uint_as_float(w[e]);
-          }
-        };
-        float kv[4][4], qv[4][4];
-        if constexpr (kConv) {
-          // y[t, c] = sum_j w[c, j] x[t - 3 + j, c] (x = 0 before the sequence start), then
-          // x / sqrt(sum_c y^2 + 1e-6) over the head's 128 channels (this warp holds them all)
-          float wq[4][4], wk[4][4];
+          auto unpack = [&](const uint32_t* w, int e) -> float {
+            if constexpr (sizeof(TIn) == 2) {
+              const uint32_t x = w[e >> 1];
+              return __uint_as_float((e & 1) ? (x & 0xFFFF0000u) : (x << 16));
+            } else {
+              return __uint_as_float(w[e]);
+            }
+          };
+          float kv[4][4], qv[4][4];
+          if constexpr (kConv) {
+            // y[t, c] = sum_j w[c, j] x[t - 3 + j, c] (x = 0 before the sequence start), then
+            // x / sqrt(sum_c y^2 + 1e-6) over the head's 128 channels (this warp holds them all)
+            float wq[4][4], wk[4][4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float4 a4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((0 * H + h) * kD + c0 + e) * 4));
-            const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((1 * H + h) * kD + c0 + e) * 4));
-            wq[e][0] = a4.x; wq[e][1] = a4.y; wq[e][2] = a4.z; wq[e][3] = a4.w;
-            wk[e][0] = b4.x; wk[e][1] = b4.y; wk[e][2] = b4.z; wk[e][3] = b4.w;
+            for (int e = 0; e < 4; ++e) {
+              const float4 a4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((0 * H + h) * kD + c0 + e) * 4));
+              const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((1 * H + h) * kD + c0 + e) * 4));
+              wq[e][0] = a4.x; wq[e][1] = a4.y; wq[e][2] = a4.z; wq[e][3] = a4.w;
+              wk[e][0] = b4.x; wk[e][1] = b4.y; wk[e][2] = b4.z; wk[e][3] = b4.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float sq = 0.f, sk = 0.f;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float yq = 0.f, yk = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int m = i + j;
+                  yq = fmaf(wq[e][j], rin[m] ? unpack(qraw[m], e) : 0.f, yq);
+                  yk = fmaf(wk[e][j], rin[m] ? unpack(kraw[m], e) : 0.f, yk);
+                }
+                qv[i][e] = yq;
+                kv[i][e] = yk;
+                sq = fmaf(yq, yq, sq);
+                sk = fmaf(yk, yk, sk);
+              }
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                sk += __shfl_xor_sync(0xffffffffu, sk, off);
+              }
+              const bool in = r0 + i < len;
+              const float fq = in ? rsqrtf(sq + 1e-6f) : 0.f, fk = in ? rsqrtf(sk + 1e-6f) : 0.f;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                qv[i][e] *= fq;
+                kv[i][e] *= fk;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                kv[i][e] = rin[i] ? unpack(kraw[i], e) : 0.f;
+                qv[i][e] = rin[i] ? unpack(qraw[i], e) : 0.f;
+              }
           }
+          float kh[4][4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            float sq = 0.f, sk = 0.f;
+            float kt[4], qt[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              float yq = 0.f, yk = 0.f;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int m = i + j;
-                yq = fmaf(wq[e][j], rin[m] ? unpack(qraw[m], e) : 0.f, yq);
-                yk = fmaf(wk[e][j], rin[m] ? unpack(kraw[m], e) : 0.f, yk);
-              }
-              qv[i][e] = yq;
-              kv[i][e] = yk;
-              sq = fmaf(yq, yq, sq);
-              sk = fmaf(yk, yk, sk);
+              const float g = pre[s][e] + la[s][i][e];
+              const float eg = __expf(g), eng = __expf(-g);
+              kt[e] = kv[i][e] * eg;
+              kh[i][e] = to_tf32(kv[i][e] * eng);
+              qt[e] = to_tf32(qv[i][e] * eg);
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-              sq += __shfl_xor_sync(0xffffffffu, sq, off);
-              sk += __shfl_xor_sync(0xffffffffu, sk, off);
-            }
-            const bool in = r0 + i < len;
-            const float fq = in ? rsqrtf(sq + 1e-6f) : 0.f, fk = in ? rsqrtf(sk + 1e-6f) : 0.f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              qv[i][e] *= fq;
-              kv[i][e] *= fk;
-            }
+            const int r = r0 + i;
+            st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[0], kt[1], kt[2], kt[3]);          // Kt [tok][ch]
+            st4_f32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);     // Qt [tok][ch]
+            st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);  // Kh [tok][ch]
           }
-        } else {
+          // Kh^T (staged for the item): channel c0+e, tokens r0..r0+3
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
+          for (int j = 0; j < 4; ++j) {
+            const int e = (j + lane) & 3;
+            float y[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              kv[i][e] = rin[i] ? unpack(kraw[i], e) : 0.f;
-              qv[i][e] = rin[i] ? unpack(qraw[i], e) : 0.f;
-            }
-        }
-        float kh[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float kt[4], qt[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float g = pre[s][e] + la[s][i][e];
-            const float eg = __expf(g), eng = __expf(-g);
-            kt[e] = kv[i][e] * eg;
-            kh[i][e] = to_tf32(kv[i][e] * eng);
-            qt[e] = to_tf32(qv[i][e] * eg);
+            for (int i = 0; i < 4; ++i) y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
+            st4_f32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);
           }
-          const int r = r0 + i;
-          st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[0], kt[1], kt[2], kt[3]);          // Kt [tok][ch]
-          st4_f32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);     // Qt [tok][ch]
-          st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);  // Kh [tok][ch]
         }
-        // Kh^T (staged for the item): channel c0+e, tokens r0..r0+3
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int e = (j + lane) & 3;
-          float y[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
-          st4_f32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);
-        }
-      }
+      }  // factorised form
       fence_proxy_async_smem();
       fsync();
-      if (ftid == 0) {  // Qt: rows 64..127 of each 32-column block of the tile; Kh^T whole
+      if (ftid == 0 && !strong) {  // Qt: rows 64..127 of each 32-column block of the tile; Kh^T whole
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb)
           bulk_store(item + kItemQW + kb * 16384 + 8192, sm + SM::kKQ + kb * 16384 + 8192, 8192);
@@ -486,12 +623,16 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
           ph_apfree ^= 1u;
         }
         tc_fence_after_sync();
-        constexpr uint32_t kIdAP = idesc_tf32(128, 64, false, false);
-        const uint64_t a0 = kdesc0(sb + SM::kKQ), b0 = kdesc0(sb + SM::kKH);
+        if (strong) {
+          mbar_arrive(bars + kBApFull);  // nothing to multiply: the back group only passes it on
+        } else {
+          constexpr uint32_t kIdAP = idesc_tf32(128, 64, false, false);
+          const uint64_t a0 = kdesc0(sb + SM::kKQ), b0 = kdesc0(sb + SM::kKH);
 #pragma unroll
-        for (int kk = 0; kk < 16; ++kk)
-          umma_tf32(tmem + kTmAP, a0 + kstep(kk, 128), b0 + kstep(kk, 64), kIdAP, kk > 0);
-        umma_commit(bars + kBApFull);
+          for (int kk = 0; kk < 16; ++kk)
+            umma_tf32(tmem + kTmAP, a0 + kstep(kk, 128), b0 + kstep(kk, 64), kIdAP, kk > 0);
+          umma_commit(bars + kBApFull);
+        }
       }
 
       // -- Kt^T, once the back group's previous W / U~ MMA and its staging have let go of KTT --
@@ -500,7 +641,7 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         ph_wfree ^= 1u;
         fsync();
       }
-      for (int i = ftid; i < kD * 16; i += kGroupThreads) {  // Kt (rows 0..63 of KQ) -> Kt^T
+      for (int i = ftid; i < (strong ? 0 : kD * 16); i += kGroupThreads) {  // Kt (rows 0..63 of KQ) -> Kt^T
         const int c = i % kD, r4 = (i / kD) * 4;
         const float* kq = reinterpret_cast<const float*>(sm + SM::kKQ);
         st4_f32(sm + SM::kKTT, f32_offset(c, r4, 128), kq[f32_offset(r4, c, 128) >> 2],
@@ -538,6 +679,29 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       ph_apfull ^= 1u;
       bsync();
       tc_fence_after_sync();
+      if (sStrong[k & 1]) {
+        // -- an item handed over as raw rows (walked by the recurrence): no solve; the v rows
+        //    (conv for the mixer) go to the item's U~ space in fp32, and the hand-overs with
+        //    the front group run as for any item ---------------------------------------------
+        tc_fence_before_sync();
+        bsync();
+        if (btid == 0) mbar_arrive(bars + kBApFree);
+        RawRowsBack rb{a.v, a.conv_w, item, ip.t0, ip.bos, ip.len, ip.h, H, btid};
+        raw_rows_back<TIn, kConv>(rb);
+        if (btid == 0) {
+          if (!lost && !mbar_wait(bars + kBVtFull, ph_vtfull, a.status)) lost = true;
+          ph_vtfull ^= 1u;
+          mbar_arrive(bars + kBWuDone);
+          if (!lost && !mbar_wait(bars + kBWuDone, ph_wu, a.status)) lost = true;
+          mbar_arrive(bars + kBWFree);
+        }
+        ph_wu ^= 1u;
+        if (group_any(kBarBack, kGroupThreads, lost)) {
+          lost = true;
+          break;
+        }
+        continue;
+      }
       {
         const int cb = half * 32;
         float d[32];
@@ -759,8 +923,11 @@ struct RecSmem {
   static_assert(kAlloc <= 232448, "shared memory plan exceeds the per-block limit");
 };
 
-template <int DV, typename TOut>
-__global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const PrefillArgs a, const SplitPlan p) {
+// kRaw: some items were handed over as raw rows and are walked token by token; without
+// it the loop is the plain tensor-core chain (the kernel picks the form from the flag
+// pass 1 leaves, so that the common case carries none of the walk's code).
+template <int DV, typename TOut, bool kRaw>
+__device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan& p) {
   using SM = RecSmem<DV>;
   constexpr int kSlices = kD / DV;
   constexpr int kPart = DV / 4;  // value columns per thread in the TMEM epilogues
@@ -925,11 +1092,77 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
   int64_t prev_t0 = -1;
   int prev_len = 0;
   int b = 0;
+  // items that pass 1 left as raw rows (e^g_last[0] = -1) are walked token by token
+  auto item_raw = [&](int c) {
+    return __ldg(reinterpret_cast<const float*>(item_of(c) + kItemGamma)) < 0.f;
+  };
+  bool raw = false;
+  if constexpr (kRaw) raw = c_begin < c_end && item_raw(c_begin);
   for (int c = c_begin; c < c_end && !failed; ++c) {
     const int i = c - c_begin;
     const int64_t t0 = bos + static_cast<int64_t>(i) * kChunk;
     const int len = static_cast<int>(eos - t0 < kChunk ? eos - t0 : kChunk);
     const uint32_t d1 = tmem + kD1 + b * DV;
+    bool raw_next = false;
+    if constexpr (kRaw) raw_next = c + 1 < c_end && item_raw(c + 1);
+
+    if (kRaw && raw) {
+      // -- the exact token walk: k | q in QW, log_alpha in KHT, beta in this chunk's PT slot
+      //    (P's bytes), v staged from the item into the other PT slot; the state slice moves
+      //    TMEM -> registers -> TMEM and the S^T operand
+      if (prev_t0 >= 0 && lq >= 2) {  // the previous chunk's output rows first
+        if (!lost && !mbar_wait(bar_o, o_phase, a.status)) lost = true;
+        o_phase ^= 1u;
+        tc_fence_after_sync();
+        out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);
+      }
+      prev_t0 = -1;
+      if (tid == 0 && !lost && !mbar_wait(bar_qw, static_cast<uint32_t>(qw_waited & 1), a.status)) lost = true;
+      if (tid == 0) ++qw_waited;
+      if (!lost && !mbar_wait(bar_pk, static_cast<uint32_t>(pk_waited & 1), a.status)) lost = true;
+      ++pk_waited;
+      tc_fence_before_sync();
+      failed = cta_any(lost);
+      tc_fence_after_sync();
+      if (failed) break;
+      {
+        // the chunk's v slice (DV columns) into the other PT slot, row-major, for the walk
+        const float* vsrc = reinterpret_cast<const float*>(item_of(c) + kItemU) + col0;
+        float* sv = reinterpret_cast<float*>(sm + SM::kPT + ((i + 1) & 1) * 32768);
+        for (int idx = tid; idx < 64 * (DV / 4); idx += kRecThreads) {
+          const int t = idx / (DV / 4), c4 = 4 * (idx % (DV / 4));
+          *reinterpret_cast<float4*>(sv + t * DV + c4) = __ldg(reinterpret_cast<const float4*>(vsrc + t * kD + c4));
+        }
+        WalkArgs wa;
+        wa.sK = reinterpret_cast<const float*>(sm + SM::kQW);
+        wa.sQ = wa.sK + 64 * kD;
+        wa.sLA = reinterpret_cast<const float*>(sm + SM::kKHT);
+        wa.sBeta = reinterpret_cast<const float*>(sm + SM::kPT + (i & 1) * 32768 + 8192);
+        wa.sV = sv;
+        wa.scr = reinterpret_cast<float*>(sm + SM::kUT);
+        wa.sST = reinterpret_cast<float*>(sm + SM::kST);
+        wa.out = outg + static_cast<size_t>(t0) * tok_stride + static_cast<size_t>(h) * kD + col0;
+        wa.gate = gateg ? gateg + static_cast<size_t>(t0) * tok_stride + static_cast<size_t>(h) * kD + col0 : nullptr;
+        wa.out_stride = tok_stride;
+        wa.tmem_state = tmem + lane_off + kD2;
+        wa.scale = 1.f;
+        wa.len = len;
+        walk_chunk<DV, TOut>(wa);
+      }
+      fence_proxy_async_smem();
+      __syncthreads();  // QW, KHT and the PT slot are read: the next chunk's tiles may land
+      if (tid == 0 && c + 1 < c_end) {
+        load_qw(c + 1);
+        load_pk(c + 1, (i + 1) & 1);
+        if (c + 2 < c_end) bulk_prefetch_l2(item_of(c + 2), kItemBytes);
+      }
+      if (lq < 2 && c + 1 < c_end) load_ut(c + 1);
+      tc_fence_before_sync();
+      failed = cta_any(lost);
+      tc_fence_after_sync();
+      raw = raw_next;
+      continue;
+    }
 
     // -- group 1: D1 = [-W S; Qt S] --------------------------------------------------------
     if (tid == 0) {
@@ -1014,6 +1247,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
     prev_t0 = t0;
     prev_len = len;
     b ^= 1;
+    raw = raw_next;
   }
   if (!failed && prev_t0 >= 0 && lq >= 2) {
     if (!lost && !mbar_wait(bar_o, o_phase, a.status)) lost = true;
@@ -1050,6 +1284,14 @@ __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const Prefill
     tc_fence_after_sync();
     tmem_dealloc(tmem, kCols);
   }
+}
+
+template <int DV, typename TOut>
+__global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const PrefillArgs a, const SplitPlan p) {
+  if (__ldg(p.any_raw))
+    recur_body<DV, TOut, true>(a, p);
+  else
+    recur_body<DV, TOut, false>(a, p);
 }
 
 // ================================ host =================================================
@@ -1107,7 +1349,8 @@ cudaError_t launch_plan(const int32_t* cu, int64_t total_T, int N, int32_t* chun
 
 cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream) {
   uint8_t* ws = static_cast<uint8_t*>(a.split_ws);
-  SplitPlan p{reinterpret_cast<const int32_t*>(ws), ws + split_plan_bytes(a.N)};
+  SplitPlan p{reinterpret_cast<const int32_t*>(ws), reinterpret_cast<int32_t*>(ws) + a.N + 1,
+              ws + split_plan_bytes(a.N)};
   cudaError_t e = launch_plan(a.cu, a.total_T, a.N, reinterpret_cast<int32_t*>(ws), a.status, stream);
   if (e != cudaSuccess) return e;
   const int64_t max_chunks = split_max_chunks(a.total_T, a.N);

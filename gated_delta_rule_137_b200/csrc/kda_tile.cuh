@@ -15,7 +15,15 @@
 namespace kda {
 namespace {
 
-constexpr float kMaxChunkDecay = 80.f;
+// Largest decay, summed over one chunk's tokens in any key channel, that a chunk may
+// carry into the factorised (tensor-core) form; stronger-decaying chunks are walked token
+// by token (walk_chunk below). Two limits meet here: e^-g must stay finite in fp32 (below
+// about 88 nats), and the tf32 operands keep the form within the 2e-2 RMS parity bar only
+// while the chunk forgets little. Measured against the fp64 oracle: final-state errors of
+// 0.3-0.4% of RMS at 5 nats, up to 1.4% at 18 nats when every channel decays that much,
+// and up to 3% between 40 and 80 nats (the state is then made of the last few tokens'
+// writes, so the relative error of each tf32 product shows undiluted).
+constexpr float kMaxChunkDecay = 20.f;
 constexpr int kLd = 68;  // row stride (floats) of the fp32 solve scratch (16-B aligned rows)
 
 // K-major fp32 operand tile with `rows` rows (M or N): descriptor of K step 0, and the
@@ -186,6 +194,163 @@ __device__ __forceinline__ void invert_unit_lower_64(float* sA, float* sY, int g
 // Whole-CTA form (threadIdx.x / 32 is the warp index, __syncthreads the barrier).
 __device__ __forceinline__ void invert_unit_lower_64(float* sA, float* sY) {
   invert_unit_lower_64(sA, sY, static_cast<int>(threadIdx.x >> 5), [] { __syncthreads(); });
+}
+
+// ---- the exact token-by-token walk of one chunk ------------------------------------
+// The chunked form multiplies K e^g by K e^-g; a chunk whose decay summed over its
+// tokens passes kMaxChunkDecay nats in some key channel would overflow e^-g or lose the
+// parity bar to tf32 rounding. Such a chunk is walked token by token instead, with the
+// recurrence itself in fp32 (no factorised exponentials, so any decay is exact):
+//     S' = Diag(alpha_t) S;  w = S'^T k_t;  b = S'^T q_t;  u = beta_t (v_t - w);
+//     S = S' + k_t u^T;      o_t = S^T q_t = b + u (k_t . q_t).
+
+// 16 values per lane; returns to lane l the sum over the warp of value l >> 1 (lanes
+// 2m and 2m + 1 both get value m). Halving exchanges: 8 + 4 + 2 + 1 + 1 shuffles.
+__device__ __forceinline__ float warp_reduce_scatter16(const float (&v)[16]) {
+  const int lane = threadIdx.x & 31;
+  const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0, h4 = (lane & 4) != 0, h2 = (lane & 2) != 0;
+  float a8[8], a4[4], a2[2];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    a8[i] = (h16 ? v[i + 8] : v[i]) + __shfl_xor_sync(0xffffffffu, h16 ? v[i] : v[i + 8], 16);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    a4[i] = (h8 ? a8[i + 4] : a8[i]) + __shfl_xor_sync(0xffffffffu, h8 ? a8[i] : a8[i + 4], 8);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    a2[i] = (h4 ? a4[i + 2] : a4[i]) + __shfl_xor_sync(0xffffffffu, h4 ? a4[i] : a4[i + 2], 4);
+  float x = (h2 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, h2 ? a2[0] : a2[1], 2);
+  return x + __shfl_xor_sync(0xffffffffu, x, 1);
+}
+
+// Scratch of walk_chunk, in floats: k.q per token, then two buffers of per-warp partial
+// sums (16 per 8-column group per warp).
+template <int KP>
+struct WalkScratch {
+  static constexpr int kKQ = 0;
+  static constexpr int kRed = 64;
+  static constexpr int kRedBuf = (KP / 8) * 256;
+  static constexpr int kFloats = kRed + 2 * kRedBuf;
+};
+
+// Where one chunk's walk reads and writes. Thread (warp w, lane l) of the 512-thread CTA
+// holds row r = 32 (w % 4) + l (key channel r) of the state slice and value columns
+// cp*KP .. cp*KP + KP - 1 of the CTA's DV columns, cp = w / 4, KP = DV / 4.
+struct WalkArgs {
+  const float* sK;             // shared [64][128] (token, channel): k of the chunk
+  const float* sQ;             // shared [64][128]: q
+  const float* sLA;            // shared [64][128]: log_alpha
+  const float* sBeta;          // shared [64]
+  const float* sV;             // shared [64][DV]: v, the CTA's value columns
+  float* scr;                  // shared, WalkScratch<DV / 4>::kFloats floats
+  float* sST;                  // shared S^T operand tile to refresh (f32_offset(col, row, DV)), or null
+  void* out;                   // global: out[t0][h][col0]; rows out_stride elements apart
+  const __nv_bfloat16* gate;   // global: gate[t0][h][col0] (same strides), or null
+  int64_t out_stride;
+  uint32_t tmem_state;         // TMEM address of the state slice's column 0 for this thread's lanes
+  float scale;                 // the state is scale * (TMEM contents) on entry
+  int len;                     // tokens of the chunk (<= 64)
+};
+
+// Walks tokens 0..len-1 of one chunk through the recurrence. Every thread of the CTA
+// calls it (it synchronises the CTA); on return the TMEM state slice (and sST, if
+// given) hold the state after the chunk and out (x sigmoid(gate)) holds its rows. Kept
+// out of line: it is the rare path, and inlining it would weigh on the register
+// allocation of the kernels' tensor-core loops.
+template <int DV, typename TOut>
+__device__ __noinline__ void walk_chunk(const WalkArgs& wa) {
+  constexpr int KP = DV / 4;
+  using WS = WalkScratch<KP>;
+  static_assert(KP % 8 == 0, "column parts come in groups of 8");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lq = warp & 3, cp = warp >> 2;
+  const int r = lq * 32 + lane;
+  const float* sK = wa.sK;
+  const float* sQ = wa.sQ;
+  float* scr = wa.scr;
+  float s[KP];
+#pragma unroll
+  for (int j = 0; j < KP; j += 8) {
+    float x[8];
+    tmem_ld8(wa.tmem_state + cp * KP + j, x);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s[j + e] = wa.scale * x[e];
+  }
+  float* sKQ = scr + WS::kKQ;
+  for (int t = warp; t < wa.len; t += 16) {  // k_t . q_t
+    float x = 0.f;
+#pragma unroll
+    for (int c = lane; c < 128; c += 32) x = fmaf(sK[t * 128 + c], sQ[t * 128 + c], x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if (lane == 0) sKQ[t] = x;
+  }
+  __syncthreads();
+  TOut* out = static_cast<TOut*>(wa.out);
+  for (int t = 0; t < wa.len; ++t) {
+    const float al = __expf(wa.sLA[t * 128 + r]), kr = sK[t * 128 + r], qr = sQ[t * 128 + r];
+    float* red = scr + WS::kRed + (t & 1) * WS::kRedBuf;
+#pragma unroll
+    for (int g = 0; g < KP / 8; ++g) {
+      float p[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        s[g * 8 + j] *= al;
+        p[j] = s[g * 8 + j] * kr;
+        p[8 + j] = s[g * 8 + j] * qr;
+      }
+      const float x = warp_reduce_scatter16(p);
+      if (!(lane & 1)) red[g * 256 + (cp * 4 + lq) * 16 + (lane >> 1)] = x;
+    }
+    __syncthreads();  // (the other buffer takes the next token: one barrier per token)
+    const float bt = wa.sBeta[t], kq = sKQ[t];
+    const float* vr = wa.sV + t * DV + cp * KP;
+#pragma unroll
+    for (int g = 0; g < KP / 8; ++g) {
+      float w[8], b[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w[j] = b[j] = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float* pr = red + g * 256 + (cp * 4 + q4) * 16;
+#pragma unroll
+        for (int j = 0; j < 8; j += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(pr + j);
+          const float4 y = *reinterpret_cast<const float4*>(pr + 8 + j);
+          w[j] += x.x; w[j + 1] += x.y; w[j + 2] += x.z; w[j + 3] += x.w;
+          b[j] += y.x; b[j + 1] += y.y; b[j + 2] += y.z; b[j + 3] += y.w;
+        }
+      }
+      float o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float u = bt * (vr[g * 8 + j] - w[j]);
+        o[j] = fmaf(u, kq, b[j]);
+        s[g * 8 + j] = fmaf(kr, u, s[g * 8 + j]);
+      }
+      if (lq == 0 && lane == 0) {  // one thread per column part writes the row
+        const size_t off = static_cast<size_t>(t) * wa.out_stride + cp * KP + g * 8;
+        if (wa.gate) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] *= 1.f / (1.f + __expf(-bf2f(wa.gate[off + e])));
+        }
+        store8(out + off, o);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KP; j += 8) {
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      x[e] = s[j + e];
+      if (wa.sST) wa.sST[f32_offset(cp * KP + j + e, r, DV) >> 2] = x[e];
+    }
+    tmem_st8(wa.tmem_state + cp * KP + j, x);
+  }
+  tmem_st_wait();
+  __syncthreads();  // the scratch and the chunk's inputs are free again
 }
 
 // ---- TMA descriptor encoding through the driver entry point ----------------------------

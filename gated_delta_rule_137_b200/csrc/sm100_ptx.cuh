@@ -34,7 +34,6 @@ constexpr uint64_t kWaitBudgetNs = 2000000000ull;
 // Error word bits raised by the device (shared with the host side via kda.h
 // KDA_DEVFLAG_* for the user-visible ones).
 constexpr uint32_t kFlagBadSeqlens = 0x1u;
-constexpr uint32_t kFlagDecayRange = 0x2u;
 constexpr uint32_t kFlagBadIndex = 0x4u;
 constexpr uint32_t kFlagWaitTimeout = 0x80000000u;
 
@@ -74,18 +73,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Waits for phase `parity` of `bar` to complete. Gives up after kWaitBudgetNs,
-// raises kFlagWaitTimeout in *err and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+// Waits for phase `parity` of `bar` to complete. Gives up after budget_ns, raises
+// kFlagWaitTimeout in *err and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t* err, uint64_t budget_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitBudgetNs) {
+    if (global_timer_ns() - t0 > budget_ns) {
       if (err) atomicOr(err, kFlagWaitTimeout);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  return mbar_wait_for(bar, parity, err, kWaitBudgetNs);
 }
 
 // Named barrier `id` (1..15) over `nthreads` threads (a multiple of 32): syncs one warp

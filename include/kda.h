@@ -33,11 +33,10 @@
  *   checks are synchronous on the host and return before any launch. A launch
  *   failure returns KDA_ERR_CUDA. The library never aborts, traps or prints.
  * - Problems that only the device can see (a cu_seqlens that is not
- *   non-decreasing or overruns total_T; a chunk whose per-channel decay exceeds
- *   the documented range) set bits in a status word held in `workspace`; the
- *   outputs are then unspecified (a bad cu_seqlens may leave every sequence
- *   unwritten). Read the word with kda_workspace_status() after the stream has
- *   run the call.
+ *   non-decreasing or overruns total_T; a wait inside a kernel that ran out of
+ *   time) set bits in a status word held in `workspace`; the outputs are then
+ *   unspecified (a bad cu_seqlens may leave every sequence unwritten). Read the
+ *   word with kda_workspace_status() after the stream has run the call.
  * - Thread safety: calls may be issued from several host threads; the message
  *   returned by kda_last_error() is thread-local.
  */
@@ -72,8 +71,13 @@ typedef enum { KDA_DT_F32 = 0, KDA_DT_BF16 = 1 } kda_dtype;
 
 /* Bits of the device status word (kda_workspace_status). */
 #define KDA_DEVFLAG_BAD_SEQLENS 0x1u  /* cu_seqlens not monotone / out of range */
-#define KDA_DEVFLAG_DECAY_RANGE 0x2u  /* chunk decay beyond the supported range  */
+#define KDA_DEVFLAG_DECAY_RANGE 0x2u  /* reserved, never set: every decay is in range (the
+                                         prefill walks chunks of very strong decay token by
+                                         token, see kda_chunk_fwd)                          */
 #define KDA_DEVFLAG_BAD_INDEX 0x4u    /* a state index outside [0, pool_size)    */
+#define KDA_DEVFLAG_WAIT_TIMEOUT 0x80000000u /* a wait inside a kernel gave up after 2 s (a lost
+                                         arrival); the kernel returned early, outputs
+                                         unspecified, the CUDA context stays usable         */
 
 /* Largest head dimensions this build accepts (d_k, d_v <= 128; the model uses 128). */
 #define KDA_MAX_HEAD_DIM 128
@@ -113,9 +117,11 @@ KDA_API size_t kda_chunk_fwd_workspace(int64_t total_T, int N, int H, int dk, in
  *   q, k       device, [total_T, H, dk], dtype qkv_dtype (bf16 or fp32)
  *   v          device, [total_T, H, dv], dtype qkv_dtype
  *   log_alpha  device fp32 [total_T, H, dk]: natural log of the per-channel
- *              decay, <= 0. Supported range: the decay summed over any 64-token
- *              chunk (aligned to the sequence start) must stay within 80 nats per
- *              channel; beyond it KDA_DEVFLAG_DECAY_RANGE is set.
+ *              decay, <= 0 (finite). Any decay is supported. A 64-token chunk
+ *              (aligned to the sequence start) whose decay summed over its tokens
+ *              stays within 80 nats in every key channel takes the tensor-core form,
+ *              which multiplies k e^g by k e^-g; any other chunk is walked token by
+ *              token with the recurrence itself (exact for any decay, slower).
  *   beta       device fp32 [total_T, H], the write strength (sigmoid output).
  *   initial_state  device fp32 [N, H, dk, dv] or NULL (zero state).
  *   cu_seqlens device int32 [N+1] or NULL (equal lengths; total_T % N == 0).
@@ -292,16 +298,29 @@ KDA_API kda_status kda_mixer_fwd_gate(const void* q_raw, const void* k_raw, cons
  * that loads the library, held until the process exits). Limit: total_T * H <=
  * 16384 token-heads; larger calls return KDA_ERR_UNSUPPORTED before any launch.
  * The first call on a device looks the array up (cudaGetSymbolAddress) with that
- * device current; make it before any stream capture. All calls on a device share
- * the array, which keeps the last call's contents (the status word is cleared at
- * the start of each call); calls that overlap on the GPU race and give undefined
- * results. Device-detected range flags are not reported. Allocates nothing.
+ * device current; make it before any stream capture. With CUDA's lazy module
+ * loading (the default) that first call is also when the driver loads the
+ * library's device code and reserves the array, so a device that is already full
+ * can fail it with KDA_ERR_CUDA: make one warm-up call (total_T = N = 0 does the set-up
+ * and launches nothing) while memory is free. All calls on a device share the
+ * array, which keeps the last call's contents (the status word is cleared at the
+ * start of each call); calls that overlap on the GPU race and give undefined
+ * results. Allocates nothing.
  */
 KDA_API kda_status kda_mixer_fwd_noalloc(const void* q_raw, const void* k_raw, const void* v_raw,
                                          const float* conv_w, const float* log_alpha, const float* beta,
                                          const void* gate, const float* initial_state, const int32_t* cu_seqlens,
                                          int64_t total_T, int N, int H, int dk, int dv, void* out,
                                          float* final_state, kda_stream_t stream);
+
+/*
+ * The device status word of kda_mixer_fwd_noalloc (it lives in the same static array
+ * on the current device): synchronises `stream`, copies the word to the host, clears
+ * it. Returns KDA_ERR_RANGE when any KDA_DEVFLAG_* bit was set (e.g. a bad
+ * cu_seqlens in the last call), KDA_OK otherwise; *flags (if not NULL) receives the
+ * bits. Allocates nothing; the same set-up rule as kda_mixer_fwd_noalloc applies.
+ */
+KDA_API kda_status kda_mixer_fwd_noalloc_status(kda_stream_t stream, uint32_t* flags);
 
 /*
  * Workspace for kda_chunk_bwd (bytes, multiple of 256; 0 for rejected sizes): the
@@ -349,6 +368,23 @@ KDA_API kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, kd
  * was set, KDA_OK otherwise; *flags (if not NULL) receives the bits.
  */
 KDA_API kda_status kda_workspace_status(void* workspace, kda_stream_t stream, uint32_t* flags);
+
+/*
+ * Diagnostic of the library's failure path (the pages have no counterpart). Every
+ * wait inside the kernels (on an mbarrier: a tensor-core commit, a bulk copy, a
+ * hand-over between warp groups) is bounded: after its budget it sets
+ * KDA_DEVFLAG_WAIT_TIMEOUT in the call's status word and the kernel returns, so a
+ * lost arrival ends as a status the host can read rather than as a hung GPU. This
+ * call launches one thread that waits, with that same bounded wait and a budget of
+ * budget_us microseconds, on an mbarrier that nothing arrives at: it always runs
+ * out, sets the bit in `workspace`'s status word (cleared first) and returns.
+ *   workspace  device, >= 256 bytes, 16-byte aligned (any workspace of this library)
+ *   budget_us  1 .. 2,000,000
+ * Read the result with kda_workspace_status (KDA_ERR_RANGE, flags =
+ * KDA_DEVFLAG_WAIT_TIMEOUT).
+ */
+KDA_API kda_status kda_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t budget_us,
+                                             kda_stream_t stream);
 
 #ifdef __cplusplus
 }

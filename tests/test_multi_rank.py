@@ -57,9 +57,11 @@ def test_single_process_needs_no_process_group():
 
 def test_algorithmic_work_figures():
     import bench
-    # model-shape prefill: 206.0 MB moved, 23.6 GFLOP of dense tensor-core work
+    # model-shape prefill: 206.0 MB moved; 18.25 GFLOP of tensor-core work counted
+    # triangle-aware (139,264 flops per token-head), 23.6 GFLOP as issued on dense tiles
     assert bench.prefill_bytes(4096, 1) == 206045184
-    assert bench.prefill_tc_flops(4096) == 4096 * 32 * (6 * 128 * 128 + 10 * 64 * 128)
+    assert bench.prefill_tc_flops(4096) == 4096 * 32 * 139264
+    assert bench.prefill_tc_flops_issued(4096) == 4096 * 32 * (6 * 128 * 128 + 10 * 64 * 128)
     # decode: two passes over a 64 KiB fp32 state per (sequence, head) plus the token
     assert bench.decode_bytes(256) == 256 * 32 * (2 * 128 * 128 * 4 + 4 * 128 * 2 + 128 * 4 + 4)
 

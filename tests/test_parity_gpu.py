@@ -131,15 +131,14 @@ def test_prefill_small_cases(kda, lens, H, dk, dv, dtype):
     assert_prefill_close(fin, rf, "final_state")
 
 
-def test_prefill_model_shape_sampled_heads(kda):
-    """B=1, T=4096, H=32, d=128 bf16 with N(0, 0.02^2) initial state; oracle on 4 heads."""
+def test_prefill_model_shape_all_heads(kda):
+    """B=1, T=4096, H=32, d=128 bf16 with N(0, 0.02^2) initial state (the headline
+    workload, through the two-pass kernels the bench times); the oracle runs every head."""
     w = I.prefill_model_shape()
     out, fin = _run_prefill(kda, w, varlen=False)
-    heads = [0, 11, 22, 31]
-    ro, rf = _oracle_heads(w, heads)
-    assert_prefill_close(out[:, heads], ro, "out", stored_bf16=True)
-    assert_prefill_close(fin[:, heads], rf, "final_state")
-    assert np.all(np.isfinite(out)) and np.all(np.isfinite(fin))
+    ro, rf = _oracle_heads(w, range(w.H))
+    assert_prefill_close(out, ro, "out", stored_bf16=True)
+    assert_prefill_close(fin, rf, "final_state")
 
 
 def test_prefill_varlen_sampled(kda):
@@ -148,8 +147,12 @@ def test_prefill_varlen_sampled(kda):
     out, fin = _run_prefill(kda, w)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(fin))
     lens = np.diff(w.cu_seqlens)
-    picks = [int(np.argmin(lens)), int(np.argmax(lens)), 17]
-    for n, h in zip(picks, [5, 30, 12]):
+    longest, shortest = int(np.argmax(lens)), int(np.argmin(lens))
+    # the longest sequence on four heads, the shortest on two, and ten more (sequence, head)
+    # chains spread over the batch: 16 chains
+    picks = [(longest, h) for h in (0, 9, 21, 30)] + [(shortest, h) for h in (5, 31)]
+    picks += [(n, (7 * n + 3) % w.H) for n in range(1, w.N, 6)][:10]
+    for n, h in picks:
         s, e = int(w.cu_seqlens[n]), int(w.cu_seqlens[n + 1])
         ro, rf = O.kda_recurrence(w.q[s:e, h:h + 1], w.k[s:e, h:h + 1], w.v[s:e, h:h + 1],
                                   w.log_alpha[s:e, h:h + 1], w.beta[s:e, h:h + 1],
@@ -252,17 +255,127 @@ def test_prefill_zero_tokens_copies_state(kda):
 
 
 def test_device_status_flags(kda):
+    """A cu_seqlens that is not monotone is flagged; a decay of 3 nats per token in every
+    channel (192 nats per chunk, beyond what e^g e^-g can carry in fp32) is not: those
+    chunks are walked token by token and must match the oracle with a clean status."""
     import torch
     w = I.make_prefill([100, 100], 2, 128, 128, seed=9)
     d = _upload(w)
     bad_cu = torch.tensor([0, 150, 120], dtype=torch.int32, device="cuda")  # not monotone
-    with pytest.raises(kda.KdaError):
+    with pytest.raises(kda.KdaError) as err:
         kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, bad_cu, N=2, check_status=True)
-    strong = d["log_alpha"] * 0 - 3.0  # 64 tokens x 3 nats > the supported chunk range
-    with pytest.raises(kda.KdaError):
-        kda.chunk_fwd(d["q"], d["k"], d["v"], strong, d["beta"], None, d["cu_seqlens"], N=2, check_status=True)
+    assert f"0x{kda.DEVFLAG_BAD_SEQLENS:08x}" in str(err.value)
+    la = np.full_like(w.log_alpha, -3.0)
+    out, fin = kda.chunk_fwd(d["q"], d["k"], d["v"], to_device(la, "f32"), d["beta"], d["initial_state"],
+                             d["cu_seqlens"], N=2, check_status=True)
+    torch.cuda.synchronize()
+    ro, rf = O.kda_recurrence(w.q, w.k, w.v, la, w.beta, w.initial_state, w.cu_seqlens)
+    assert_prefill_close(to_host(out), ro, "out at 3 nats per token", stored_bf16=True)
+    assert_prefill_close(to_host(fin), rf, "final state at 3 nats per token")
     # a valid call afterwards reports a clean status
     kda.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, d["cu_seqlens"], N=2, check_status=True)
+
+
+def test_wait_timeout_is_reported(kda):
+    """Every wait inside the kernels is bounded. The diagnostic entry point runs one such
+    wait on an mbarrier that nothing arrives at, with a 2 ms budget: it must give up,
+    leave KDA_DEVFLAG_WAIT_TIMEOUT in the status word, and leave the context usable."""
+    import torch
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    kda.selftest_wait_timeout(ws, 2000)
+    with pytest.raises(kda.KdaError) as err:
+        kda.workspace_status(ws)
+    assert f"0x{kda.DEVFLAG_WAIT_TIMEOUT:08x}" in str(err.value)
+    assert kda.workspace_status(ws) == 0  # read and cleared
+    w = I.make_prefill([70], 2, 128, 128, seed=10)
+    out, fin = _run_prefill(kda, w)  # the context still runs kernels
+    ro, rf = O.kda_recurrence(w.q, w.k, w.v, w.log_alpha, w.beta, w.initial_state, w.cu_seqlens)
+    assert_prefill_close(out, ro, "out after the timed-out wait", stored_bf16=True)
+
+
+# ------------------------------------------------------------- strong per-channel decay
+
+def _decay_pattern(w, scale, pattern):
+    """log_alpha = -softplus(z) * scale per channel (the generator draws -softplus(z)/16).
+    pattern "all": every chunk; "odd": only the odd 64-token chunks of each sequence (the
+    even ones keep the generator's mild decay), so fast and walked chunks alternate."""
+    la = w.log_alpha * (16.0 * scale)
+    if pattern == "odd":
+        keep = np.zeros(la.shape[0], dtype=bool)
+        for n in range(w.N):
+            s, e = int(w.cu_seqlens[n]), int(w.cu_seqlens[n + 1])
+            keep[s:e] = ((np.arange(e - s) // 64) % 2) == 0
+        la = np.where(keep[:, None, None], w.log_alpha, la)
+    return la
+
+
+@pytest.mark.parametrize("path", ["two-pass", "single-pass"])
+@pytest.mark.parametrize("scale,pattern,dtype", [
+    (1.0, "all", "bf16"),    # ~0.8 nats per token: chunks near and past the 80-nat line
+    (8.0, "all", "bf16"),    # ~6.5 nats per token: every chunk walked
+    (8.0, "odd", "bf16"),    # walked and tensor-core chunks alternate along each sequence
+    (8.0, "odd", "f32"),
+])
+def test_prefill_strong_decay(kda, path, scale, pattern, dtype):
+    """Per-channel decay far beyond the range of the factorised chunk form, through the
+    two-pass kernels (<= 74 chains) and the single-pass kernel (> 74 chains), against the
+    oracle's token recurrence; no status flag may be raised."""
+    rng = np.random.default_rng(I.SEED_BASE + 41)
+    if path == "two-pass":
+        lens, H = [200, 64, 7, 131], 4                          # 16 chains, ragged tails
+    else:
+        lens, H = [int(x) for x in rng.integers(1, 200, 20)], 4  # 80 chains
+        lens[:3] = [64, 65, 128]
+    w = I.make_prefill(lens, H, 128, 128, seed=I.SEED_BASE + 42 + int(scale), qkv_dtype=dtype)
+    la = _decay_pattern(w, scale, pattern)
+    need = kda.chunk_fwd_workspace_bytes(w.total_T, w.N, H, 128, 128,
+                                         kda.KDA_DT_BF16 if dtype == "bf16" else kda.KDA_DT_F32)
+    assert (need > 256) == (path == "two-pass")
+    d = _upload(w)
+    import torch
+    out, fin = kda.chunk_fwd(d["q"], d["k"], d["v"], to_device(la, "f32"), d["beta"], d["initial_state"],
+                             d["cu_seqlens"], N=w.N, check_status=True)
+    torch.cuda.synchronize()
+    ro, rf = O.kda_recurrence(w.q, w.k, w.v, la, w.beta, w.initial_state, w.cu_seqlens)
+    assert_prefill_close(to_host(out), ro, f"out ({path}, decay x{scale} {pattern})", stored_bf16=(dtype == "bf16"))
+    assert_prefill_close(to_host(fin), rf, f"final state ({path}, decay x{scale} {pattern})")
+
+
+@pytest.mark.parametrize("lens,H", [([300, 77], 4), ([70] * 40, 2)])  # two-pass; single-pass (80 chains)
+def test_mixer_strong_decay(kda, lens, H):
+    """The full mixer (conv4 + L2 inside the kernels, sigmoid gate) with strong decay on
+    the odd chunks: the walked chunks must see the conv'd, normalised q, k, v."""
+    w = I.make_prefill(lens, H, 128, 128, seed=sum(lens) + 43, normalise_qk=False, mixer=True)
+    la = _decay_pattern(w, 8.0, "odd")
+    import torch
+    dt = "bf16"
+    out, fin = kda.mixer_fwd(to_device(w.q, dt), to_device(w.k, dt), to_device(w.v, dt), to_device(w.conv_w, "f32"),
+                             to_device(la, "f32"), to_device(w.beta, "f32"), to_device(w.gate, dt),
+                             to_device(w.initial_state, "f32"), to_device(w.cu_seqlens, "i32"), N=w.N,
+                             check_status=True)
+    torch.cuda.synchronize()
+    ro, rf = O.kda_mixer(w.q, w.k, w.v, w.conv_w, la, w.beta, w.gate, w.cu_seqlens, w.initial_state)
+    assert_prefill_close(to_host(out), ro, "strong-decay mixer out", stored_bf16=True)
+    assert_prefill_close(to_host(fin), rf, "strong-decay mixer final state")
+
+
+def test_mixer_gate_from_preactivation_strong(kda):
+    """kda_mixer_fwd_gate with per-head scales of 4..8 on softplus(a): about 3-6 nats per
+    token, so most chunks are walked with log_alpha made on the device."""
+    import torch
+    w = I.make_prefill([300, 77], 4, 128, 128, seed=44, normalise_qk=False, mixer=True)
+    a_pre, _ = I.make_gate_preactivation(w.q.shape[0], 4, 128, seed=45)
+    a_scale = np.array([4.0, 5.0, 6.0, 8.0])
+    dt = "bf16"
+    out, fin = kda.mixer_fwd_gate(to_device(w.q, dt), to_device(w.k, dt), to_device(w.v, dt),
+                                  to_device(w.conv_w, "f32"), to_device(a_pre, "bf16"), to_device(a_scale, "f32"),
+                                  to_device(w.beta, "f32"), to_device(w.gate, dt), to_device(w.initial_state, "f32"),
+                                  to_device(w.cu_seqlens, "i32"), N=w.N, check_status=True)
+    torch.cuda.synchronize()
+    la = O.gate_log_alpha(a_pre, a_scale)
+    ro, rf = O.kda_mixer(w.q, w.k, w.v, w.conv_w, la, w.beta, w.gate, w.cu_seqlens, w.initial_state)
+    assert_prefill_close(to_host(out), ro, "strong gate-from-pre-activation out", stored_bf16=True)
+    assert_prefill_close(to_host(fin), rf, "strong gate-from-pre-activation final state")
 
 
 # --------------------------------------------------------------------------- mixer
@@ -299,11 +412,11 @@ def test_mixer_small(kda):
 
 
 def test_mixer_full_size_sampled_heads(kda):
-    """B=2, T=32768, H=32, d=128: conv4 + L2 + KDA + sigmoid gate; oracle on 2 heads."""
+    """B=2, T=32768, H=32, d=128: conv4 + L2 + KDA + sigmoid gate; oracle on 8 heads."""
     w = I.mixer_prefill()
     out, fin = _run_mixer(kda, w)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(fin))
-    heads = [3, 28]
+    heads = [0, 3, 8, 13, 17, 22, 28, 31]
     ro, rf = _mixer_oracle_heads(w, heads)
     assert_prefill_close(out[:, heads], ro, "mixer out", stored_bf16=True)
     assert_prefill_close(fin[:, heads], rf, "mixer final")
