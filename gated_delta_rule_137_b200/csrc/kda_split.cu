@@ -900,7 +900,12 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
 }
 
 // ================================ pass 2 =============================================
-constexpr int kRecThreads = 512;  // 16 warps; warp w reads TMEM lanes 32*(w%4).. and column part w/4
+// 17 warps: warps 0..15 run the epilogues (warp w reads TMEM lanes 32*(w%4).. and value
+// column part w/4); warp 16 waits for the tiles and issues the MMAs, so that an issue
+// that blocks on the tensor pipe never holds up an epilogue.
+constexpr int kRecEpiThreads = 512;
+constexpr int kRecThreads = kRecEpiThreads + 32;
+constexpr uint32_t kRecBarU = 1;  // named barrier: U^T written (epilogue warps + the issuer warp)
 
 //  region   size        holds
 //  QW       64 KB       [-W; Qt] of the current chunk
@@ -916,13 +921,20 @@ struct RecSmem {
   static constexpr int kKHT = 131072;
   static constexpr int kST = 163840;
   static constexpr int kUT = kST + DV * 512;
-  static constexpr int kBar = kUT + DV * 256;  // 4 mbarriers
-  static constexpr int kTmemSlot = kBar + 32;
+  static constexpr int kBar = kUT + DV * 256;  // 5 mbarriers
+  static constexpr int kTmemSlot = kBar + 48;
   static constexpr int kTotal = kTmemSlot + 16;
   static constexpr int kAlloc = kTotal + 1024;
   static_assert(kAlloc <= 232448, "shared memory plan exceeds the per-block limit");
 };
 
+// Per chunk, with S the state slice (TMEM D2 and the S^T operand in shared memory):
+//   issuer:   QW landed -> G1: D1 = [-W; Qt] S -> (G1 done) next chunk's QW on its way
+//   epilogue: (G1 done) U = U~ + D1[0:64] -> U^T operand                  [barrier U]
+//   issuer:   PK landed -> G2a: D2 += Kh^T U ; G2b: D1 += [.; P] U (output rows, read a
+//             chunk later) -> (G2a done) next chunk's P, Kh^T, e^g_last on their way
+//   epilogue: (G2a done) S <- e^g_last D2 (TMEM and S^T)                 [end barrier]
+// The state chain waits only for G1, the U epilogue, G2a and the S epilogue.
 // kRaw: some items were handed over as raw rows and are walked token by token; without
 // it the loop is the plain tensor-core chain (the kernel picks the form from the flag
 // pass 1 leaves, so that the common case carries none of the walk's code).
@@ -938,6 +950,8 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const bool issuer_warp = warp == 16;
+  const bool issuer = issuer_warp && lane == 0;
   const int lq = warp & 3;
   const int cp = warp >> 2;
   const int row = lq * 32 + lane;
@@ -964,17 +978,15 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
-  uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + SM::kBar);
-  uint64_t* bar_qw = bar_mma + 1;
-  uint64_t* bar_pk = bar_mma + 2;
-  uint64_t* bar_o = bar_mma + 3;  // the chunk's P U is done: its output rows may be read
+  uint64_t* bar_g1 = reinterpret_cast<uint64_t*>(sm + SM::kBar);  // G1 done
+  uint64_t* bar_qw = bar_g1 + 1;                                    // QW landed
+  uint64_t* bar_pk = bar_g1 + 2;                                    // P, Kh^T, e^g_last landed
+  uint64_t* bar_o = bar_g1 + 3;   // the chunk's P U is done: its output rows may be read
+  uint64_t* bar_g2 = bar_g1 + 4;  // G2a done: the state may be updated
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::kTmemSlot);
 
   if (tid == 0) {
-    mbar_init(bar_mma, 1);
-    mbar_init(bar_qw, 1);
-    mbar_init(bar_pk, 1);
-    mbar_init(bar_o, 1);
+    for (int i = 0; i < 5; ++i) mbar_init(bar_g1 + i, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -988,7 +1000,7 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
   const uint32_t lane_off = static_cast<uint32_t>(lq * 32) << 16;
 
   auto item_of = [&](int c) -> const uint8_t* { return p.items + (static_cast<size_t>(c) * H + h) * kItemBytes; };
-  // loads issued / waited per barrier (thread 0 issues; the counts tell the teardown
+  // loads issued / waited per barrier (the issuer issues; the counts tell the teardown
   // what may still be in flight)
   int qw_issued = 0, pk_issued = 0;
   auto load_qw = [&](int c) {
@@ -1006,14 +1018,14 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
     bulk_load(pt, it + kItemGamma, 512u, bar_pk);
     ++pk_issued;
   };
-  if (tid == 0 && c_begin < c_end) {
+  if (issuer && c_begin < c_end) {
     load_qw(c_begin);
     load_pk(c_begin, 0);
     if (c_begin + 1 < c_end) bulk_prefetch_l2(item_of(c_begin + 1), kItemBytes);
   }
 
   // ---- the state slice: TMEM D2 (lane c = key row c) and the S^T operand ---------------
-  {
+  if (!issuer_warp) {
     const float* h0 = a.h0 ? a.h0 + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0 : nullptr;
 #pragma unroll
     for (int j = 0; j < kPart; j += 8) {
@@ -1044,31 +1056,29 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
       ut[4 * e] = x.x; ut[4 * e + 1] = x.y; ut[4 * e + 2] = x.z; ut[4 * e + 3] = x.w;
     }
   };
-  if (lq < 2 && c_begin < c_end) load_ut(c_begin);
+  if (!issuer_warp && lq < 2 && c_begin < c_end) load_ut(c_begin);
 
   const __nv_bfloat16* gateg = static_cast<const __nv_bfloat16*>(a.gate);
   TOut* outg = static_cast<TOut*>(a.out);
   const int64_t tok_stride = static_cast<int64_t>(H) * kD;
   // output rows of a finished chunk: rows 64..127 of its D1 buffer (* sigmoid(gate))
   auto out_rows = [&](uint32_t d1, int64_t tt0, int tlen) {
-    if (lq >= 2) {
-      const int r = row - 64;
+    const int r = row - 64;
 #pragma unroll
-      for (int j = 0; j < kPart; j += 8) {
-        const int c = cp * kPart + j;
-        float o[8];
-        tmem_ld8(d1 + lane_off + c, o);
-        tmem_ld_wait();
-        if (r < tlen) {
-          const size_t off = static_cast<size_t>(tt0 + r) * tok_stride + static_cast<size_t>(h) * kD + col0 + c;
-          if (gateg) {
-            const uint4 g0 = *reinterpret_cast<const uint4*>(gateg + off);
-            const __nv_bfloat16* gb0 = reinterpret_cast<const __nv_bfloat16*>(&g0);
+    for (int j = 0; j < kPart; j += 8) {
+      const int c = cp * kPart + j;
+      float o[8];
+      tmem_ld8(d1 + lane_off + c, o);
+      tmem_ld_wait();
+      if (r < tlen) {
+        const size_t off = static_cast<size_t>(tt0 + r) * tok_stride + static_cast<size_t>(h) * kD + col0 + c;
+        if (gateg) {
+          const uint4 g0 = *reinterpret_cast<const uint4*>(gateg + off);
+          const __nv_bfloat16* gb0 = reinterpret_cast<const __nv_bfloat16*>(&g0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] *= 1.f / (1.f + __expf(-bf2f(gb0[i])));
-          }
-          store8(outg + off, o);
+          for (int i = 0; i < 8; ++i) o[i] *= 1.f / (1.f + __expf(-bf2f(gb0[i])));
         }
+        store8(outg + off, o);
       }
     }
   };
@@ -1080,14 +1090,17 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
 
   constexpr uint32_t kIdV = idesc_tf32(128, DV, false, false);
   bool lost = false, failed = false;
-  uint32_t mma_phase = 0;
-  auto wait_mma = [&]() {
-    if (!lost && !mbar_wait(bar_mma, mma_phase, a.status)) lost = true;
-    mma_phase ^= 1u;
-    tc_fence_after_sync();
+  // completions seen per barrier (each thread counts those it waits for)
+  uint32_t g1_phase = 0, g2_phase = 0, o_phase = 0;
+  int qw_waited = 0, pk_waited = 0;
+  auto wait_bar = [&](uint64_t* bar, uint32_t& phase) {
+    if (!lost && !mbar_wait(bar, phase, a.status)) lost = true;
+    phase ^= 1u;
   };
-  int qw_waited = 0, pk_waited = 0;  // (thread 0: QW; every thread: PK)
-  uint32_t o_phase = 0;               // output-row warps: completions of bar_o seen
+  auto wait_loads = [&](uint64_t* bar, int& waited) {
+    if (!lost && !mbar_wait(bar, static_cast<uint32_t>(waited & 1), a.status)) lost = true;
+    ++waited;
+  };
 
   int64_t prev_t0 = -1;
   int prev_len = 0;
@@ -1110,26 +1123,28 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
       // -- the exact token walk: k | q in QW, log_alpha in KHT, beta in this chunk's PT slot
       //    (P's bytes), v staged from the item into the other PT slot; the state slice moves
       //    TMEM -> registers -> TMEM and the S^T operand
-      if (prev_t0 >= 0 && lq >= 2) {  // the previous chunk's output rows first
-        if (!lost && !mbar_wait(bar_o, o_phase, a.status)) lost = true;
-        o_phase ^= 1u;
+      if (!issuer_warp && prev_t0 >= 0 && lq >= 2) {  // the previous chunk's output rows first
+        wait_bar(bar_o, o_phase);
         tc_fence_after_sync();
         out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);
       }
       prev_t0 = -1;
-      if (tid == 0 && !lost && !mbar_wait(bar_qw, static_cast<uint32_t>(qw_waited & 1), a.status)) lost = true;
-      if (tid == 0) ++qw_waited;
-      if (!lost && !mbar_wait(bar_pk, static_cast<uint32_t>(pk_waited & 1), a.status)) lost = true;
-      ++pk_waited;
+      if (issuer) {
+        wait_loads(bar_qw, qw_waited);
+        wait_loads(bar_pk, pk_waited);
+      }
       tc_fence_before_sync();
-      failed = cta_any(lost);
+      failed = cta_any(lost);  // the raw rows have landed (or a wait gave up)
       tc_fence_after_sync();
+      // the epilogue warps count the PK phase the issuer waited for (their next wait names
+      // the right parity)
+      if (!issuer_warp) ++pk_waited;
       if (failed) break;
-      {
+      if (!issuer_warp) {
         // the chunk's v slice (DV columns) into the other PT slot, row-major, for the walk
         const float* vsrc = reinterpret_cast<const float*>(item_of(c) + kItemU) + col0;
         float* sv = reinterpret_cast<float*>(sm + SM::kPT + ((i + 1) & 1) * 32768);
-        for (int idx = tid; idx < 64 * (DV / 4); idx += kRecThreads) {
+        for (int idx = tid; idx < 64 * (DV / 4); idx += kRecEpiThreads) {
           const int t = idx / (DV / 4), c4 = 4 * (idx % (DV / 4));
           *reinterpret_cast<float4*>(sv + t * DV + c4) = __ldg(reinterpret_cast<const float4*>(vsrc + t * kD + c4));
         }
@@ -1148,82 +1163,81 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
         wa.scale = 1.f;
         wa.len = len;
         walk_chunk<DV, TOut>(wa);
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
-      __syncthreads();  // QW, KHT and the PT slot are read: the next chunk's tiles may land
-      if (tid == 0 && c + 1 < c_end) {
+      tc_fence_before_sync();
+      failed = cta_any(lost);  // QW, KHT and the PT slots are read: the next chunk's tiles may land
+      tc_fence_after_sync();
+      if (issuer && c + 1 < c_end) {
         load_qw(c + 1);
         load_pk(c + 1, (i + 1) & 1);
         if (c + 2 < c_end) bulk_prefetch_l2(item_of(c + 2), kItemBytes);
       }
-      if (lq < 2 && c + 1 < c_end) load_ut(c + 1);
-      tc_fence_before_sync();
-      failed = cta_any(lost);
-      tc_fence_after_sync();
+      if (!issuer_warp && lq < 2 && c + 1 < c_end) load_ut(c + 1);
       raw = raw_next;
       continue;
     }
 
-    // -- group 1: D1 = [-W S; Qt S] --------------------------------------------------------
-    if (tid == 0) {
-      if (!lost && !mbar_wait(bar_qw, static_cast<uint32_t>(qw_waited & 1), a.status)) lost = true;
-      ++qw_waited;
-      tc_fence_after_sync();
-      const uint64_t a0 = kdesc0(sb + SM::kQW), b0 = kdesc0(sb + SM::kST);
+    if (issuer_warp) {
+      // ================================ the MMA issuer ====================================
+      if (issuer) {
+        wait_loads(bar_qw, qw_waited);
+        tc_fence_after_sync();
+        const uint64_t a0 = kdesc0(sb + SM::kQW), b0 = kdesc0(sb + SM::kST);
 #pragma unroll
-      for (int kk = 0; kk < 16; ++kk) umma_tf32(d1, a0 + kstep(kk, 128), b0 + kstep(kk, DV), kIdV, kk > 0);
-      umma_commit(bar_mma);
-    }
-    if (prev_t0 >= 0 && lq >= 2) {  // the previous chunk's output rows, while the MMAs run
-      if (!lost && !mbar_wait(bar_o, o_phase, a.status)) lost = true;
-      o_phase ^= 1u;
-      tc_fence_after_sync();
-      out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);
-    }
-    wait_mma();
-
-    // -- U = U~ + D1[0:64] -> U^T operand; next chunk's [-W; Qt] on its way ------------------
-    if (tid == 0 && c + 1 < c_end) {
-      load_qw(c + 1);
-      if (c + 2 < c_end) bulk_prefetch_l2(item_of(c + 2), kItemBytes);
-    }
-    if (lq < 2) {
-#pragma unroll
-      for (int j = 0; j < kPart; j += 8) {
-        const int cc = cp * kPart + j;
-        float ws[8];
-        tmem_ld8(d1 + lane_off + cc, ws);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 8; ++e) st_tf32(sm + SM::kUT, f32_offset(cc + e, row, DV), ut[j + e] + ws[e]);
+        for (int kk = 0; kk < 16; ++kk) umma_tf32(d1, a0 + kstep(kk, 128), b0 + kstep(kk, DV), kIdV, kk > 0);
+        umma_commit(bar_g1);
+        wait_bar(bar_g1, g1_phase);  // QW has been read: the next chunk's [-W; Qt] on its way
+        if (c + 1 < c_end) {
+          load_qw(c + 1);
+          if (c + 2 < c_end) bulk_prefetch_l2(item_of(c + 2), kItemBytes);
+        }
       }
-      if (c + 1 < c_end) load_ut(c + 1);
-    }
-    if (!lost && !mbar_wait(bar_pk, static_cast<uint32_t>(pk_waited & 1), a.status)) lost = true;
-    ++pk_waited;
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
-
-    // -- group 2: D2 += Kh^T U (the state chain waits for this commit only), then
-    //    D1 += [.; P] U -> O = Qt S + P U in rows 64..127 (read a chunk later) ----------------
-    if (tid == 0) {
+      group_sync(kRecBarU, kRecThreads);  // U^T is written
+      if (issuer) {
+        wait_loads(bar_pk, pk_waited);
+        tc_fence_after_sync();
+        const uint64_t ka = kdesc0(sb + SM::kKHT), ub = kdesc0(sb + SM::kUT);
+        const uint64_t pa = kdesc0(sb + SM::kPT + (i & 1) * 32768);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) umma_tf32(tmem + kD2, ka + kstep(kk, 128), ub + kstep(kk, DV), kIdV, 1u);
+        umma_commit(bar_g2);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) umma_tf32(d1, pa + kstep(kk, 128), ub + kstep(kk, DV), kIdV, 1u);
+        umma_commit(bar_o);
+        // Kh^T and the other PT slot (last read by the P U of the previous chunk, which the
+        // G2a commit covers) are free: the next chunk's P, Kh^T, e^g_last on their way
+        wait_bar(bar_g2, g2_phase);
+        if (c + 1 < c_end) load_pk(c + 1, (i + 1) & 1);
+      }
+    } else {
+      // ================================ the epilogue warps ================================
+      if (prev_t0 >= 0 && lq >= 2) {  // the previous chunk's output rows, while G1 runs
+        wait_bar(bar_o, o_phase);
+        tc_fence_after_sync();
+        out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);
+      }
+      if (lq < 2) {  // U = U~ + D1[0:64] -> U^T operand
+        wait_bar(bar_g1, g1_phase);
+        tc_fence_after_sync();
+#pragma unroll
+        for (int j = 0; j < kPart; j += 8) {
+          const int cc = cp * kPart + j;
+          float ws[8];
+          tmem_ld8(d1 + lane_off + cc, ws);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) st_tf32(sm + SM::kUT, f32_offset(cc + e, row, DV), ut[j + e] + ws[e]);
+        }
+        if (c + 1 < c_end) load_ut(c + 1);
+        fence_proxy_async_smem();
+      }
+      tc_fence_before_sync();
+      group_sync(kRecBarU, kRecThreads);  // U^T is written
+      // S <- e^g_last D2 (TMEM and S^T), once G2a is done and this chunk's e^g_last has landed
+      wait_loads(bar_pk, pk_waited);
+      wait_bar(bar_g2, g2_phase);
       tc_fence_after_sync();
-      const uint64_t ka = kdesc0(sb + SM::kKHT), ub = kdesc0(sb + SM::kUT);
-      const uint64_t pa = kdesc0(sb + SM::kPT + (i & 1) * 32768);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) umma_tf32(tmem + kD2, ka + kstep(kk, 128), ub + kstep(kk, DV), kIdV, 1u);
-      umma_commit(bar_mma);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) umma_tf32(d1, pa + kstep(kk, 128), ub + kstep(kk, DV), kIdV, 1u);
-      umma_commit(bar_o);
-    }
-    wait_mma();
-
-    // -- S <- e^g_last D2 (TMEM and S^T); next chunk's P, Kh^T, e^g_last on their way (the
-    //    other PT buffer: its last reader, the P U of chunk i-1, finished before group 1) --
-    if (tid == 0 && c + 1 < c_end) load_pk(c + 1, (i + 1) & 1);
-    {
       const float gm = reinterpret_cast<const float*>(sm + SM::kPT + (i & 1) * 32768)[row];
 #pragma unroll
       for (int j = 0; j < kPart; j += 8) {
@@ -1239,25 +1253,24 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
         tmem_st8(tmem + lane_off + kD2 + cc, x);
       }
       tmem_st_wait();
+      fence_proxy_async_smem();
     }
-    fence_proxy_async_smem();
     tc_fence_before_sync();
-    failed = cta_any(lost);
+    failed = cta_any(lost);  // the state is written (S^T and TMEM): the next chunk's G1 may go
     tc_fence_after_sync();
     prev_t0 = t0;
     prev_len = len;
     b ^= 1;
     raw = raw_next;
   }
-  if (!failed && prev_t0 >= 0 && lq >= 2) {
-    if (!lost && !mbar_wait(bar_o, o_phase, a.status)) lost = true;
-    o_phase ^= 1u;
+  if (!failed && !issuer_warp && prev_t0 >= 0 && lq >= 2) {
+    wait_bar(bar_o, o_phase);
     tc_fence_after_sync();
     out_rows(tmem + kD1 + (b ^ 1) * DV, prev_t0, prev_len);
   }
 
   // ---- final state ---------------------------------------------------------------------------
-  if (!failed && a.ht) {
+  if (!failed && !issuer_warp && a.ht) {
     float* ht = a.ht + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0;
 #pragma unroll
     for (int j = 0; j < kPart; j += 8) {
@@ -1272,9 +1285,9 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
 
   // ---- teardown: after a lost wait, let the tensor pipe and the bulk loads drain (bounded)
   //      before the TMEM and the shared memory go back --------------------------------------
-  if (failed && tid == 0) {
-    umma_commit(bar_mma);
-    mbar_wait(bar_mma, mma_phase, a.status);
+  if (failed && issuer) {
+    umma_commit(bar_o);
+    mbar_wait(bar_o, o_phase, a.status);
     for (; qw_waited < qw_issued; ++qw_waited) mbar_wait(bar_qw, static_cast<uint32_t>(qw_waited & 1), a.status);
     for (; pk_waited < pk_issued; ++pk_waited) mbar_wait(bar_pk, static_cast<uint32_t>(pk_waited & 1), a.status);
   }
@@ -1285,7 +1298,6 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
     tmem_dealloc(tmem, kCols);
   }
 }
-
 template <int DV, typename TOut>
 __global__ void __launch_bounds__(kRecThreads, 1) kda_recur_kernel(const PrefillArgs a, const SplitPlan p) {
   if (__ldg(p.any_raw))

@@ -252,8 +252,12 @@ struct WalkArgs {
   int len;                     // tokens of the chunk (<= 64)
 };
 
-// Walks tokens 0..len-1 of one chunk through the recurrence. Every thread of the CTA
-// calls it (it synchronises the CTA); on return the TMEM state slice (and sST, if
+// Named barrier of the 512 threads that walk (a CTA may hold more warps, which do not).
+constexpr uint32_t kWalkBar = 2;
+__device__ __forceinline__ void walk_sync() { group_sync(kWalkBar, 512); }
+
+// Walks tokens 0..len-1 of one chunk through the recurrence. Threads 0..511 of the CTA
+// call it (they synchronise on kWalkBar); on return the TMEM state slice (and sST, if
 // given) hold the state after the chunk and out (x sigmoid(gate)) holds its rows. Kept
 // out of line: it is the rare path, and inlining it would weigh on the register
 // allocation of the kernels' tensor-core loops.
@@ -286,7 +290,7 @@ __device__ __noinline__ void walk_chunk(const WalkArgs& wa) {
     for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
     if (lane == 0) sKQ[t] = x;
   }
-  __syncthreads();
+  walk_sync();
   TOut* out = static_cast<TOut*>(wa.out);
   for (int t = 0; t < wa.len; ++t) {
     const float al = __expf(wa.sLA[t * 128 + r]), kr = sK[t * 128 + r], qr = sQ[t * 128 + r];
@@ -303,7 +307,7 @@ __device__ __noinline__ void walk_chunk(const WalkArgs& wa) {
       const float x = warp_reduce_scatter16(p);
       if (!(lane & 1)) red[g * 256 + (cp * 4 + lq) * 16 + (lane >> 1)] = x;
     }
-    __syncthreads();  // (the other buffer takes the next token: one barrier per token)
+    walk_sync();  // (the other buffer takes the next token: one barrier per token)
     const float bt = wa.sBeta[t], kq = sKQ[t];
     const float* vr = wa.sV + t * DV + cp * KP;
 #pragma unroll
@@ -350,7 +354,7 @@ __device__ __noinline__ void walk_chunk(const WalkArgs& wa) {
     tmem_st8(wa.tmem_state + cp * KP + j, x);
   }
   tmem_st_wait();
-  __syncthreads();  // the scratch and the chunk's inputs are free again
+  walk_sync();  // the scratch and the chunk's inputs are free again
 }
 
 // ---- TMA descriptor encoding through the driver entry point ----------------------------
