@@ -500,8 +500,9 @@ def run_gpu(args):
         ci = device_prefill_inputs(Tc, H, D, 1370006, device, state_N=1)
         cargs = [ci[k] for k in ("q", "k", "v", "log_alpha", "beta")]
         seg_of = lambda x, i: x[i * T1:(i + 1) * T1].contiguous()
-        last = [seg_of(x, segs - 1) for x in cargs]
-        maps = [cpm.segment_map(*[seg_of(x, i) for x in cargs], N=1) for i in range(segs)]
+        segs_in = [[seg_of(x, i) for x in cargs] for i in range(segs)]
+        maps = [kda.segment_maps(*p, N=1) for p in segs_in]
+        last = segs_in[segs - 1]
 
         def timed(fn, n=5):
             for _ in range(2):
@@ -515,22 +516,36 @@ def run_gpu(args):
             torch.cuda.synchronize(device)
             return e0.elapsed_time(e1) / n
 
-        S_last = cpm.start_state(maps, segs - 1, ci["initial_state"])
-        t_map = timed(lambda: cpm.segment_map(*last, N=1))
-        t_fold = timed(lambda: cpm.start_state(maps, segs - 1, ci["initial_state"]))
-        t_final = timed(lambda: kda.chunk_fwd(*last, S_last, None, N=1))
+        MB = torch.stack([torch.stack([m[0], m[1]]) for m in maps])  # the all-gather's layout
+        S_last = torch.empty_like(ci["initial_state"])
+        fold = lambda: lib.kda_state_fold(MB.data_ptr(), segs - 1, ci["initial_state"].data_ptr(),
+                                          S_last.data_ptr(), H, D, stream.cuda_stream)
+        kda._check(fold())
+        mws = maps[segs - 1][2].workspace
+        M_l, B_l = torch.empty_like(maps[0][0]), torch.empty_like(maps[0][1])
+        o_l = torch.empty(T1, H, D, dtype=torch.bfloat16, device=device)
+        f_l = torch.empty(1, H, D, D, dtype=torch.float32, device=device)
+        t_map = timed(lambda: lib.kda_segment_maps(last[0].data_ptr(), last[1].data_ptr(), last[2].data_ptr(),
+                                                   kda.KDA_DT_BF16, last[3].data_ptr(), last[4].data_ptr(), None,
+                                                   T1, 1, H, D, D, M_l.data_ptr(), B_l.data_ptr(), mws.data_ptr(),
+                                                   mws.numel(), stream.cuda_stream))
+        t_fold = timed(fold)
+        t_final = timed(lambda: lib.kda_segment_prefill(mws.data_ptr(), mws.numel(), kda.KDA_DT_BF16,
+                                                        S_last.data_ptr(), None, T1, 1, H, D, D, o_l.data_ptr(),
+                                                        f_l.data_ptr(), stream.cuda_stream))
         t_emul = timed(lambda: cpm.context_parallel_emulate(*cargs, ci["initial_state"], N=1, segments=segs), 3)
         t_plain = timed(lambda: kda.chunk_fwd(*cargs, ci["initial_state"], None, N=1), 3)
-        # timed calls x kernels: maps 5 x 2 prefills x 3, fold 5 x 3 affine, segment prefill 5 x 3,
-        # emulation 3 x (4 maps x 6 + 4 prefills x 3 + 6 affine), plain prefill 3 x 3
-        launches += 5 * 6 + 5 * 3 + 5 * 3 + 3 * (4 * 6 + 4 * 3 + 6) + 3 * 3
+        # timed calls x kernels: maps 7 x 3, fold 7 x 1, segment prefill 7 x 1,
+        # emulation 5 x (4 maps x 3 + 3 folds + 4 prefills x 1), plain prefill 5 x 3
+        launches += 7 * 3 + 7 + 7 + 5 * (4 * 3 + 3 + 4) + 5 * 3
         cpar = {"workload": f"context-parallel prefill of one {Tc}-token sequence (H={H} d={D}) in {segs} segments; "
-                            "pieces timed on one GPU with CUDA events (the exchange is not part of it)",
-                "segment_map_ms": t_map, "fold_ms": t_fold, "segment_prefill_ms": t_final,
+                            "pieces timed on one GPU with CUDA events (the exchange is not part of it); the last "
+                            "rank's path: segment maps, fold of the earlier maps, segment prefill",
+                "segment_maps_ms": t_map, "fold_ms": t_fold, "segment_prefill_ms": t_final,
                 "per_rank_path_ms": t_map + t_fold + t_final,
                 "emulated_on_one_gpu_ms": t_emul, "plain_prefill_ms": t_plain,
                 "exchange_bytes_per_rank": 2 * H * D * D * 4}
-        del ci, cargs, maps, last
+        del ci, cargs, maps, last, segs_in, MB
 
     # ---------------- full mixer (conv4 + L2 + KDA + gate), B=2 x T=32768 ----------------
     mix = None

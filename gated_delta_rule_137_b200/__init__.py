@@ -62,6 +62,11 @@ _SIGNATURES = {
     "kda_workspace_status": (_i32, [_vp, _vp, _u32p]),
     "kda_mixer_fwd_noalloc_status": (_i32, [_vp, _u32p]),
     "kda_selftest_wait_timeout": (_i32, [_vp, _sz, ctypes.c_uint32, _vp]),
+    "kda_state_fold": (_i32, [_vp, _i32, _vp, _vp, _i64, _i32, _vp]),
+    "kda_segment_maps_workspace": (_sz, [_i64, _i32, _i32, _i32, _i32]),
+    "kda_segment_maps": (_i32, [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _vp, _vp,
+                                _vp, _sz, _vp]),
+    "kda_segment_prefill": (_i32, [_vp, _sz, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "kda_mixer_fwd_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
                                      _vp, _vp, _vp]),
     "kda_mixer_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
@@ -397,3 +402,70 @@ def selftest_wait_timeout(workspace, budget_us: int, stream=None) -> None:
     lib = load_library()
     _check(lib.kda_selftest_wait_timeout(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                          budget_us, _stream(stream)))
+
+
+class SegmentMaps:
+    """What kda_segment_maps leaves for kda_segment_prefill: the workspace holding the
+    segment's per-chunk operands, and the sizes and dtype they were made with."""
+
+    def __init__(self, workspace, cu_seqlens, total_T: int, N: int, H: int, dtype_code: int, device):
+        self.workspace, self.cu_seqlens = workspace, cu_seqlens
+        self.total_T, self.N, self.H, self.dtype_code, self.device = total_T, N, H, dtype_code, device
+
+
+def segment_maps(q, k, v, log_alpha, beta, cu_seqlens=None, *, N: Optional[int] = None, workspace=None,
+                 stream=None, check_status: bool = False):
+    """(M, B, handle) of a segment (kda_segment_maps): S_end = M S_start + B for each of its
+    sequences; `handle` feeds segment_prefill."""
+    torch = _torch()
+    lib = load_library()
+    total_T, H, dk = q.shape
+    dv = v.shape[-1]
+    if N is None:
+        if cu_seqlens is None:
+            raise ValueError("N is needed when cu_seqlens is not given")
+        N = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    M, B = torch.empty((N, H, dk, dv), **f32), torch.empty((N, H, dk, dv), **f32)
+    need = int(lib.kda_segment_maps_workspace(total_T, N, H, dk, dv))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib.kda_segment_maps(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(log_alpha), _ptr(beta), _ptr(cu_seqlens),
+                                total_T, N, H, dk, dv, _ptr(M), _ptr(B), _ptr(workspace), workspace.numel(),
+                                _stream(stream)))
+    if check_status:
+        workspace_status(workspace, stream)
+    return M, B, SegmentMaps(workspace, cu_seqlens, total_T, N, H, dt, q.device)
+
+
+def segment_prefill(handle: SegmentMaps, initial_state=None, *, out=None, final_state=None,
+                    output_final_state: bool = True, stream=None, check_status: bool = False):
+    """The segment of `handle` prefilled from `initial_state` (kda_segment_prefill)."""
+    torch = _torch()
+    lib = load_library()
+    h = handle
+    if out is None:
+        dtype = torch.float32 if h.dtype_code == KDA_DT_F32 else torch.bfloat16
+        out = torch.empty((h.total_T, h.H, 128), dtype=dtype, device=h.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((h.N, h.H, 128, 128), dtype=torch.float32, device=h.device)
+    _check(lib.kda_segment_prefill(_ptr(h.workspace), h.workspace.numel(), h.dtype_code, _ptr(initial_state),
+                                   _ptr(h.cu_seqlens), h.total_T, h.N, h.H, 128, 128, _ptr(out), _ptr(final_state),
+                                   _stream(stream)))
+    if check_status:
+        workspace_status(h.workspace, stream)
+    return out, final_state
+
+
+def state_fold(MB, maps: int, S0=None, *, out=None, stream=None):
+    """S <- M_j S + B_j for j < maps (kda_state_fold); MB [>= maps, 2, ..., 128, 128] fp32
+    (M then B of each map), S0 like one M or None (zero)."""
+    torch = _torch()
+    lib = load_library()
+    d = MB.shape[-1]
+    count = MB[0, 0].numel() // (d * d)
+    if out is None:
+        out = torch.empty(MB.shape[2:], dtype=torch.float32, device=MB.device)
+    _check(lib.kda_state_fold(_ptr(MB), maps, _ptr(S0), _ptr(out), count, d, _stream(stream)))
+    return out

@@ -321,6 +321,25 @@ kda_status kda_state_affine(const float* M, const float* S, const float* B, floa
   if (e != cudaSuccess) return cuda_fail(e, "state affine kernel launch");
   return ok();
 }
+kda_status kda_state_fold(const float* MB, int maps, const float* S0, float* out, int64_t count, int d,
+                          kda_stream_t stream_) {
+  if (count < 0 || maps < 0) return fail(KDA_ERR_INVALID_ARG, "count=%lld and maps=%d must be >= 0",
+                                         static_cast<long long>(count), maps);
+  if (d != kda::kD) return fail(KDA_ERR_UNSUPPORTED, "kda_state_fold is built for d = 128 (got %d)", d);
+  if (count > (int64_t{1} << 31) - 1) return fail(KDA_ERR_INVALID_ARG, "count too large");
+  if (count == 0) return ok();
+  if (!out || (maps > 0 && !MB)) return fail(KDA_ERR_INVALID_ARG, "MB and out must be non-NULL");
+  const void* ptrs[] = {MB, S0, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "MB, S0 and out must be 16-byte aligned");
+  const size_t n = static_cast<size_t>(count) * d * d * sizeof(float);
+  if (maps > 0 && ranges_overlap(out, n, MB, 2 * static_cast<size_t>(maps) * n))
+    return fail(KDA_ERR_INVALID_ARG, "out must not overlap the maps");
+  if (S0 && S0 != out && ranges_overlap(out, n, S0, n)) return fail(KDA_ERR_INVALID_ARG, "out partially overlaps S0");
+  cudaError_t e = kda::launch_state_fold(MB, maps, S0, out, count, reinterpret_cast<cudaStream_t>(stream_));
+  if (e != cudaSuccess) return cuda_fail(e, "state fold kernel launch");
+  return ok();
+}
 size_t kda_mixer_fwd_workspace(int64_t total_T, int N, int H, int dk, int dv) {
   if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
   if (dk != kda::kD || dv != kda::kD) return 0;
@@ -515,6 +534,104 @@ kda_status kda_workspace_status(void* workspace, kda_stream_t stream_, uint32_t*
 }
 
 }  // extern "C"
+
+namespace {
+kda_status check_segment(const void* q, const void* k, const void* v, kda_dtype dt, const float* log_alpha,
+                         const float* beta, const int32_t* cu_seqlens, int64_t total_T, int N, int H, int dk, int dv) {
+  kda_status st = check_common(total_T, N, H, dk, dv);
+  if (st != KDA_OK) return st;
+  if (dk != kda::kD || dv != kda::kD)
+    return fail(KDA_ERR_UNSUPPORTED, "the segment calls are built for dk = dv = 128 (got %d, %d)", dk, dv);
+  if (dt != KDA_DT_F32 && dt != KDA_DT_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "qkv_dtype=%d is neither KDA_DT_F32 nor KDA_DT_BF16", static_cast<int>(dt));
+  if (N < 1 || total_T < 1) return fail(KDA_ERR_INVALID_ARG, "a segment needs N >= 1 and total_T >= 1");
+  if (!cu_seqlens && total_T % N != 0)
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is NULL but total_T=%lld is not a multiple of N=%d",
+                static_cast<long long>(total_T), N);
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+  const void* ptrs[] = {q, k, v, log_alpha, beta};
+  const char* names[] = {"q", "k", "v", "log_alpha", "beta"};
+  for (int i = 0; i < 5; ++i) {
+    if (!ptrs[i]) return fail(KDA_ERR_INVALID_ARG, "%s must be non-NULL", names[i]);
+    if (!aligned16(ptrs[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  return KDA_OK;
+}
+}  // namespace
+
+extern "C" size_t kda_segment_maps_workspace(int64_t total_T, int N, int H, int dk, int dv) {
+  if (check_common(total_T, N, H, dk, dv) != KDA_OK || dk != kda::kD || dv != kda::kD) return 0;
+  const size_t s = kda::split_workspace_bytes(total_T, N, H, /*any_chains=*/true);
+  return s ? kda::kStatusBytes + s : 0;
+}
+
+extern "C" kda_status kda_segment_maps(const void* q, const void* k, const void* v, kda_dtype qkv_dtype,
+                                       const float* log_alpha, const float* beta, const int32_t* cu_seqlens,
+                                       int64_t total_T, int N, int H, int dk, int dv, float* M, float* B,
+                                       void* workspace, size_t workspace_bytes, kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  kda_status st = check_segment(q, k, v, qkv_dtype, log_alpha, beta, cu_seqlens, total_T, N, H, dk, dv);
+  if (st != KDA_OK) return st;
+  if (!M || !B || !aligned16(M) || !aligned16(B))
+    return fail(KDA_ERR_INVALID_ARG, "M and B must be non-NULL and 16-byte aligned");
+  const size_t n_st = static_cast<size_t>(N) * H * kda::kD * kda::kD * sizeof(float);
+  if (ranges_overlap(M, n_st, B, n_st)) return fail(KDA_ERR_INVALID_ARG, "M and B overlap");
+  const size_t need = kda_segment_maps_workspace(total_T, N, H, dk, dv);
+  if (need == 0) return fail(KDA_ERR_UNSUPPORTED, "the items of this segment would pass 32 GiB");
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed (16-byte aligned)",
+                workspace ? workspace_bytes : 0, need);
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  kda::PrefillArgs a{};
+  a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.cu = cu_seqlens;
+  a.status = status; a.total_T = total_T; a.N = N; a.H = H;
+  a.in_f32 = a.out_f32 = (qkv_dtype == KDA_DT_F32);
+  a.split_ws = ws + kda::kStatusBytes;
+  a.map_M = M; a.map_B = B;
+  e = kda::launch_prefill_split(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "segment map kernels launch");
+  return ok();
+}
+
+extern "C" kda_status kda_segment_prefill(void* workspace, size_t workspace_bytes, kda_dtype qkv_dtype,
+                                          const float* initial_state, const int32_t* cu_seqlens, int64_t total_T,
+                                          int N, int H, int dk, int dv, void* out, float* final_state,
+                                          kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  kda_status st = check_common(total_T, N, H, dk, dv);
+  if (st != KDA_OK) return st;
+  if (dk != kda::kD || dv != kda::kD)
+    return fail(KDA_ERR_UNSUPPORTED, "the segment calls are built for dk = dv = 128 (got %d, %d)", dk, dv);
+  if (qkv_dtype != KDA_DT_F32 && qkv_dtype != KDA_DT_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "qkv_dtype=%d is neither KDA_DT_F32 nor KDA_DT_BF16", static_cast<int>(qkv_dtype));
+  if (N < 1 || total_T < 1) return fail(KDA_ERR_INVALID_ARG, "a segment needs N >= 1 and total_T >= 1");
+  if (!out || !aligned16(out)) return fail(KDA_ERR_INVALID_ARG, "out must be non-NULL and 16-byte aligned");
+  const void* opt[] = {initial_state, final_state};
+  for (const void* x : opt)
+    if (x && !aligned16(x)) return fail(KDA_ERR_INVALID_ARG, "initial_state and final_state must be 16-byte aligned");
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+  const size_t n_st = static_cast<size_t>(N) * H * kda::kD * kda::kD * sizeof(float);
+  if (final_state && initial_state && final_state != initial_state &&
+      ranges_overlap(final_state, n_st, initial_state, n_st))
+    return fail(KDA_ERR_INVALID_ARG, "final_state partially overlaps initial_state");
+  const size_t need = kda_segment_maps_workspace(total_T, N, H, dk, dv);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(KDA_ERR_WORKSPACE, "the workspace of the segment's kda_segment_maps call is needed (%zu bytes)", need);
+  char* ws = static_cast<char*>(workspace);
+  kda::PrefillArgs a{};
+  a.cu = cu_seqlens; a.status = reinterpret_cast<uint32_t*>(ws); a.total_T = total_T; a.N = N; a.H = H;
+  a.h0 = initial_state; a.out = out; a.ht = final_state;
+  a.in_f32 = a.out_f32 = (qkv_dtype == KDA_DT_F32);
+  a.split_ws = ws + kda::kStatusBytes;
+  cudaError_t e = kda::launch_recur_only(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "segment prefill kernel launch");
+  return ok();
+}
 
 namespace {
 // One thread waits on an mbarrier that nothing arrives at, with the library's bounded

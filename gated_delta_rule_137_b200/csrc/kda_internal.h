@@ -46,6 +46,10 @@ struct PrefillArgs {
   const void* a_pre;      // bf16 [total_T, H, 128] or null: the decay gate's pre-activation, with
   const float* a_scale;   // fp32 [H]: log_alpha = -a_scale[h] * softplus(a_pre) (log_alpha null);
                           // two-pass full mixer only
+  float* map_M;           // segment maps (two-pass only): when set, the recurrence writes no
+  float* map_B;           // outputs; half of its value-column slices run from the identity with zero
+                          // values (their final states are M [N, H, 128, 128]), the other half from
+                          // zero with the real values (B); out, ht and h0 are not used
 };
 
 // ---- two-pass prefill (kda_split.cu) ---------------------------------------------------
@@ -76,6 +80,9 @@ inline size_t split_workspace_bytes(int64_t total_T, int N, int H, bool any_chai
   return split_plan_bytes(N) + items;
 }
 cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream);
+// The recurrence alone over the plan and items a previous launch_prefill_split left in
+// a.split_ws (same sequences): outputs and final states from a new initial state.
+cudaError_t launch_recur_only(const PrefillArgs& a, cudaStream_t stream);
 // cu_seqlens (or N equal lengths) -> chunk_start[N + 1]: the first 64-token chunk of each
 // sequence, [N] = total; -1 there and the status flag on bad cu_seqlens.
 cudaError_t launch_plan(const int32_t* cu, int64_t total_T, int N, int32_t* chunk_start, uint32_t* status,
@@ -108,6 +115,9 @@ cudaError_t launch_mixer_decode_commit(const float* state_ckpt, const void* conv
 // out[i] = M[i] S[i] + B[i] for `count` 128 x 128 fp32 matrices (S, B may be null: zero).
 cudaError_t launch_state_affine(const float* M, const float* S, const float* B, float* out, int64_t count,
                                 cudaStream_t stream);
+// S <- M_j S + B_j for j = 0 .. maps-1 (MB: [maps][2][count][128][128]; S0 null: zero).
+cudaError_t launch_state_fold(const float* MB, int maps, const float* S0, float* out, int64_t count,
+                              cudaStream_t stream);
 
 // Tensor-core chunked prefill on d = 128 operands (bf16 or fp32 q/k/v/out).
 cudaError_t launch_prefill_d128(const PrefillArgs& a, cudaStream_t stream);

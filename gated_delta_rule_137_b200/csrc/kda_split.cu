@@ -955,8 +955,13 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
   const int lq = warp & 3;
   const int cp = warp >> 2;
   const int row = lq * 32 + lane;
-  const int slice = blockIdx.x % kSlices;
-  const int nh = blockIdx.x / kSlices;
+  // segment maps: slices [0, kSlices) run from the identity with zero values (M), slices
+  // [kSlices, 2 kSlices) from zero with the real values (B); no outputs
+  const bool maps = a.map_M != nullptr;
+  const int nslices = maps ? 2 * kSlices : kSlices;
+  const bool map_m = maps && static_cast<int>(blockIdx.x % nslices) < kSlices;
+  const int slice = (blockIdx.x % nslices) % kSlices;
+  const int nh = blockIdx.x / nslices;
   const int H = a.H;
   const int h = nh % H;
   const int n = nh / H;
@@ -1026,12 +1031,16 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
 
   // ---- the state slice: TMEM D2 (lane c = key row c) and the S^T operand ---------------
   if (!issuer_warp) {
-    const float* h0 = a.h0 ? a.h0 + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0 : nullptr;
+    const float* h0 =
+        a.h0 && !maps ? a.h0 + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0 : nullptr;
 #pragma unroll
     for (int j = 0; j < kPart; j += 8) {
       const int c = cp * kPart + j;
       float x[8];
-      if (h0) {
+      if (map_m) {  // the identity (key row = value column)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = (row == col0 + c + e) ? 1.f : 0.f;
+      } else if (h0) {
         const float4 u = *reinterpret_cast<const float4*>(h0 + c);
         const float4 w = *reinterpret_cast<const float4*>(h0 + c + 4);
         x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
@@ -1046,9 +1055,13 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
     tmem_st_wait();
   }
 
-  // U~ of the next chunk for this thread (rows 0..63: row, columns col0 + cp*kPart ..)
+  // U~ of the next chunk for this thread (rows 0..63: row, columns col0 + cp*kPart ..);
+  // zero for the identity slices of the segment maps (zero values)
   float ut[kPart];
+#pragma unroll
+  for (int e = 0; e < kPart; ++e) ut[e] = 0.f;
   auto load_ut = [&](int c) {
+    if (map_m) return;
     const uint8_t* src = item_of(c) + kItemU;
 #pragma unroll
     for (int e = 0; e < kPart / 4; ++e) {
@@ -1063,6 +1076,7 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
   const int64_t tok_stride = static_cast<int64_t>(H) * kD;
   // output rows of a finished chunk: rows 64..127 of its D1 buffer (* sigmoid(gate))
   auto out_rows = [&](uint32_t d1, int64_t tt0, int tlen) {
+    if (maps) return;
     const int r = row - 64;
 #pragma unroll
     for (int j = 0; j < kPart; j += 8) {
@@ -1146,7 +1160,8 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
         float* sv = reinterpret_cast<float*>(sm + SM::kPT + ((i + 1) & 1) * 32768);
         for (int idx = tid; idx < 64 * (DV / 4); idx += kRecEpiThreads) {
           const int t = idx / (DV / 4), c4 = 4 * (idx % (DV / 4));
-          *reinterpret_cast<float4*>(sv + t * DV + c4) = __ldg(reinterpret_cast<const float4*>(vsrc + t * kD + c4));
+          *reinterpret_cast<float4*>(sv + t * DV + c4) =
+              map_m ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(reinterpret_cast<const float4*>(vsrc + t * kD + c4));
         }
         WalkArgs wa;
         wa.sK = reinterpret_cast<const float*>(sm + SM::kQW);
@@ -1156,7 +1171,7 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
         wa.sV = sv;
         wa.scr = reinterpret_cast<float*>(sm + SM::kUT);
         wa.sST = reinterpret_cast<float*>(sm + SM::kST);
-        wa.out = outg + static_cast<size_t>(t0) * tok_stride + static_cast<size_t>(h) * kD + col0;
+        wa.out = maps ? nullptr : outg + static_cast<size_t>(t0) * tok_stride + static_cast<size_t>(h) * kD + col0;
         wa.gate = gateg ? gateg + static_cast<size_t>(t0) * tok_stride + static_cast<size_t>(h) * kD + col0 : nullptr;
         wa.out_stride = tok_stride;
         wa.tmem_state = tmem + lane_off + kD2;
@@ -1270,8 +1285,9 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
   }
 
   // ---- final state ---------------------------------------------------------------------------
-  if (!failed && !issuer_warp && a.ht) {
-    float* ht = a.ht + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0;
+  float* ht_base = maps ? (map_m ? a.map_M : a.map_B) : a.ht;
+  if (!failed && !issuer_warp && ht_base) {
+    float* ht = ht_base + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0;
 #pragma unroll
     for (int j = 0; j < kPart; j += 8) {
       const int c = cp * kPart + j;
@@ -1336,7 +1352,7 @@ cudaError_t launch_recur_dv(const PrefillArgs& a, const SplitPlan& p, cudaStream
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RecSmem<DV>::kAlloc);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  const unsigned grid = static_cast<unsigned>(a.N) * static_cast<unsigned>(a.H) * (kD / DV);
+  const unsigned grid = static_cast<unsigned>(a.N) * static_cast<unsigned>(a.H) * (kD / DV) * (a.map_M ? 2u : 1u);
   kern<<<grid, kRecThreads, RecSmem<DV>::kAlloc, stream>>>(a, p);
   return cudaGetLastError();
 }
@@ -1346,7 +1362,8 @@ cudaError_t launch_recur(const PrefillArgs& a, const SplitPlan& p, cudaStream_t 
   // value-column slices per chain: as many as a single wave of CTAs over the 148 SMs
   // allows (one CTA per SM); beyond 74 chains (only the gate-from-pre-activation mixer
   // takes the two passes there) 64-column slices in several waves
-  const int64_t chains = static_cast<int64_t>(a.N) * a.H;
+  // (the segment maps run twice the slices: both halves of a single wave where they fit)
+  const int64_t chains = static_cast<int64_t>(a.N) * a.H * (a.map_M ? 2 : 1);
   if (4 * chains <= 148) return launch_recur_dv<32, TOut>(a, p, stream);
   return launch_recur_dv<64, TOut>(a, p, stream);  // more than 74 chains: several waves
 }
@@ -1357,6 +1374,13 @@ cudaError_t launch_plan(const int32_t* cu, int64_t total_T, int N, int32_t* chun
                         cudaStream_t stream) {
   kda_plan_kernel<<<1, 1024, 0, stream>>>(cu, total_T, N, chunk_start, status);
   return cudaGetLastError();
+}
+
+cudaError_t launch_recur_only(const PrefillArgs& a, cudaStream_t stream) {
+  uint8_t* ws = static_cast<uint8_t*>(a.split_ws);
+  SplitPlan p{reinterpret_cast<const int32_t*>(ws), reinterpret_cast<int32_t*>(ws) + a.N + 1,
+              ws + split_plan_bytes(a.N)};
+  return a.out_f32 ? launch_recur<float>(a, p, stream) : launch_recur<__nv_bfloat16>(a, p, stream);
 }
 
 cudaError_t launch_prefill_split(const PrefillArgs& a, cudaStream_t stream) {

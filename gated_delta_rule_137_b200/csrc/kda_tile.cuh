@@ -244,7 +244,7 @@ struct WalkArgs {
   const float* sV;             // shared [64][DV]: v, the CTA's value columns
   float* scr;                  // shared, WalkScratch<DV / 4>::kFloats floats
   float* sST;                  // shared S^T operand tile to refresh (f32_offset(col, row, DV)), or null
-  void* out;                   // global: out[t0][h][col0]; rows out_stride elements apart
+  void* out;                   // global: out[t0][h][col0]; rows out_stride elements apart (null: none)
   const __nv_bfloat16* gate;   // global: gate[t0][h][col0] (same strides), or null
   int64_t out_stride;
   uint32_t tmem_state;         // TMEM address of the state slice's column 0 for this thread's lanes
@@ -333,7 +333,7 @@ __device__ __noinline__ void walk_chunk(const WalkArgs& wa) {
         o[j] = fmaf(u, kq, b[j]);
         s[g * 8 + j] = fmaf(kr, u, s[g * 8 + j]);
       }
-      if (lq == 0 && lane == 0) {  // one thread per column part writes the row
+      if (out && lq == 0 && lane == 0) {  // one thread per column part writes the row
         const size_t off = static_cast<size_t>(t) * wa.out_stride + cp * KP + g * 8;
         if (wa.gate) {
 #pragma unroll

@@ -119,7 +119,7 @@ KDA_API size_t kda_chunk_fwd_workspace(int64_t total_T, int N, int H, int dk, in
  *   log_alpha  device fp32 [total_T, H, dk]: natural log of the per-channel
  *              decay, <= 0 (finite). Any decay is supported. A 64-token chunk
  *              (aligned to the sequence start) whose decay summed over its tokens
- *              stays within 80 nats in every key channel takes the tensor-core form,
+ *              stays within 20 nats in every key channel takes the tensor-core form,
  *              which multiplies k e^g by k e^-g; any other chunk is walked token by
  *              token with the recurrence itself (exact for any decay, slower).
  *   beta       device fp32 [total_T, H], the write strength (sigmoid output).
@@ -240,6 +240,51 @@ KDA_API kda_status kda_mixer_decode_commit(const float* state_ckpt, const void* 
  */
 KDA_API kda_status kda_state_affine(const float* M, const float* S, const float* B, float* out, int64_t count,
                             int d, kda_stream_t stream);
+
+/*
+ * Segment maps, for prefilling one long sequence on several devices at once (context
+ * parallelism). The state after a stretch of tokens is affine in the state before it
+ * (the KDA section cited at the top: each token multiplies the state on the left by
+ * (I - beta k k^T) Diag(alpha) and adds beta k v^T), so a segment acts on the state as
+ * S_end = M S_start + B: M is the segment's final state from the identity with zero
+ * values, B its final state from zero. kda_segment_maps computes both from one pass over
+ * the segment's chunks and keeps that pass's per-chunk operands in `workspace`;
+ * kda_segment_prefill then runs the segment from any start state on those operands (once
+ * the start state is known, e.g. after the ranks have exchanged their maps and folded the
+ * earlier segments' maps with kda_state_affine). Together they cost about one prefill and
+ * a half instead of three.
+ *
+ *   q, k, v, qkv_dtype, log_alpha, beta, cu_seqlens, total_T, N, H: as for kda_chunk_fwd
+ *              (dk = dv = 128; total_T >= 1)
+ *   M, B       device fp32 [N, H, 128, 128], written
+ *   workspace  device, >= kda_segment_maps_workspace(...) bytes, 16-byte aligned; keep it
+ *              untouched between the two calls (its status word holds the flags of both)
+ * kda_segment_prefill writes out ([total_T, H, 128], qkv_dtype) and final_state (fp32
+ * [N, H, 128, 128] or NULL) from initial_state (fp32 [N, H, 128, 128] or NULL: zero), for
+ * the same segment (same sizes and cu_seqlens as the maps call). Status words and errors
+ * as for kda_chunk_fwd.
+ */
+KDA_API size_t kda_segment_maps_workspace(int64_t total_T, int N, int H, int dk, int dv);
+KDA_API kda_status kda_segment_maps(const void* q, const void* k, const void* v, kda_dtype qkv_dtype,
+                                    const float* log_alpha, const float* beta, const int32_t* cu_seqlens,
+                                    int64_t total_T, int N, int H, int dk, int dv, float* M, float* B,
+                                    void* workspace, size_t workspace_bytes, kda_stream_t stream);
+KDA_API kda_status kda_segment_prefill(void* workspace, size_t workspace_bytes, kda_dtype qkv_dtype,
+                                       const float* initial_state, const int32_t* cu_seqlens, int64_t total_T,
+                                       int N, int H, int dk, int dv, void* out, float* final_state,
+                                       kda_stream_t stream);
+
+/*
+ * A chain of affine maps in one call: S <- M_j S + B_j for j = 0 .. maps-1, starting from
+ * S0 (NULL: zero); out receives the result. The start state of segment r of a context-
+ * parallel prefill is the fold of the maps of segments 0 .. r-1 (see kda_segment_maps).
+ *   MB   device fp32 [maps, 2, count, d, d]: M then B of each map (the layout of the
+ *        ranks' all-gathered maps)
+ *   S0   device fp32 [count, d, d] or NULL;  out device fp32 [count, d, d] (may be S0)
+ * d must be 128; pointers 16-byte aligned; fp32 arithmetic.
+ */
+KDA_API kda_status kda_state_fold(const float* MB, int maps, const float* S0, float* out, int64_t count, int d,
+                                  kda_stream_t stream);
 
 /* Workspace for kda_mixer_fwd (bytes, multiple of 256; 0 for rejected sizes): the
  * status word plus the two-pass prefill's scratch, sized as for kda_chunk_fwd (the

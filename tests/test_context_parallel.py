@@ -110,8 +110,9 @@ def test_emulation_on_one_device_matches_the_recurrence():
 
 @pytest.mark.gpu
 def test_context_parallel_emulation_with_the_kernels():
-    """4 segments of a 1024-token sequence (H = 4, d = 128, bf16) through kda_chunk_fwd and
-    kda_state_affine on one GPU, against the oracle's whole-sequence recurrence."""
+    """4 segments of a 1024-token sequence (H = 4, d = 128, bf16) through kda_segment_maps,
+    kda_state_fold and kda_segment_prefill on one GPU, against the oracle's whole-sequence
+    recurrence."""
     import torch
     from gated_delta_rule_137_b200 import build
     build.build()
@@ -146,3 +147,63 @@ def test_state_affine_kernel_against_matmul():
     kda.state_affine(M, S, out, out=out)  # in place over B
     torch.cuda.synchronize()
     assert (out.double() - ref).abs().max().item() / ref.abs().max().item() < 1e-5
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("maps", [0, 1, 3])
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_state_fold_kernel_against_matmul(maps, with_s0):
+    """kda_state_fold: S <- M_j S + B_j for j < maps, the maps laid out [maps + 1, 2, N, H, d, d]
+    (one more than are folded, as a rank below the last sees them), against the chain of
+    fp64 products; in place over S0 too."""
+    import torch
+    from gated_delta_rule_137_b200 import build
+    build.build()
+    import gated_delta_rule_137_b200 as kda
+    g = torch.Generator(device="cuda").manual_seed(137203 + maps)
+    MB = torch.randn(maps + 1, 2, 2, 3, 128, 128, generator=g, device="cuda") / 8
+    S0 = torch.randn(2, 3, 128, 128, generator=g, device="cuda") if with_s0 else None
+    want = S0.double() if with_s0 else torch.zeros(2, 3, 128, 128, dtype=torch.float64, device="cuda")
+    for j in range(maps):
+        want = MB[j, 0].double() @ want + MB[j, 1].double()
+    out = kda.state_fold(MB, maps, S0)
+    torch.cuda.synchronize()
+    scale = max(want.abs().max().item(), 1.0)
+    assert (out.double() - want).abs().max().item() / scale < 1e-5
+    if with_s0:
+        kda.state_fold(MB, maps, S0, out=S0)
+        torch.cuda.synchronize()
+        assert (S0.double() - want).abs().max().item() / scale < 1e-5
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("lens,H,strong", [([200, 64], 4, False), ([130, 7], 4, True), ([70] * 20, 4, False)])
+def test_segment_maps_and_prefill_against_the_oracle(lens, H, strong):
+    """kda_segment_maps: M = final state from the identity with zero values, B = final state
+    from zero, from one pass over the chunks; kda_segment_prefill from a start state on what
+    it left. Ragged sequences, strong decay on the odd chunks (walked), and 80 chains
+    (several waves of the doubled slices)."""
+    import torch
+    from gated_delta_rule_137_b200 import build
+    build.build()
+    import gated_delta_rule_137_b200 as kda
+    from tests.helpers import assert_prefill_close, to_device, to_host
+    w = I.make_prefill(lens, H, 128, 128, seed=I.SEED_BASE + 52 + len(lens))
+    la = w.log_alpha.copy()
+    if strong:
+        for n in range(w.N):
+            s, e = int(w.cu_seqlens[n]), int(w.cu_seqlens[n + 1])
+            la[s:e][((np.arange(e - s) // 64) % 2) == 1] *= 128.0
+    cu = to_device(w.cu_seqlens, "i32")
+    M, B, handle = kda.segment_maps(to_device(w.q, "bf16"), to_device(w.k, "bf16"), to_device(w.v, "bf16"),
+                                    to_device(la, "f32"), to_device(w.beta, "f32"), cu, check_status=True)
+    out, fin = kda.segment_prefill(handle, to_device(w.initial_state, "f32"), check_status=True)
+    torch.cuda.synchronize()
+    eye = np.broadcast_to(np.eye(128), (w.N, H, 128, 128))
+    _, rM = O.kda_recurrence(w.q, w.k, np.zeros_like(w.v), la, w.beta, eye, w.cu_seqlens)
+    _, rB = O.kda_recurrence(w.q, w.k, w.v, la, w.beta, None, w.cu_seqlens)
+    ro, rf = O.kda_recurrence(w.q, w.k, w.v, la, w.beta, w.initial_state, w.cu_seqlens)
+    assert_prefill_close(to_host(M), rM, "segment map M")
+    assert_prefill_close(to_host(B), rB, "segment map B")
+    assert_prefill_close(to_host(out), ro, "segment prefill out", stored_bf16=True)
+    assert_prefill_close(to_host(fin), rf, "segment prefill final state")
