@@ -59,6 +59,8 @@ _SIGNATURES = {
     "kda_mixer_fwd_workspace": (_sz, [_i64, _i32, _i32, _i32, _i32]),
     "kda_mixer_fwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
                              _vp, _vp, _vp, _sz, _vp]),
+    "kda_mixer_fwd_pooled": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
+                                    _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp]),
     "kda_workspace_status": (_i32, [_vp, _vp, _u32p]),
     "kda_mixer_fwd_noalloc_status": (_i32, [_vp, _u32p]),
     "kda_selftest_wait_timeout": (_i32, [_vp, _sz, ctypes.c_uint32, _vp]),
@@ -222,6 +224,34 @@ def mixer_fwd(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate=None, initial_s
     if check_status:
         workspace_status(workspace, stream)
     return out, final_state
+
+
+def mixer_fwd_pooled(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool, conv_pool,
+                     state_indices=None, initial_state=None, cu_seqlens=None, *, N: Optional[int] = None, out=None,
+                     workspace=None, stream=None, check_status: bool = False):
+    """Full mixer prefill handing its sequences to the serving decode (kda_mixer_fwd_pooled):
+    final states into state_pool[slot] fp32 [P, H, 128, 128], the last three raw q, k, v rows
+    into conv_pool[slot] bf16 [P, H, 3, 3, 128]. Returns out."""
+    torch = _torch()
+    lib = load_library()
+    total_T, H, dk = q_raw.shape
+    dv = v_raw.shape[-1]
+    if N is None:
+        if cu_seqlens is None:
+            raise ValueError("N is needed when cu_seqlens is not given")
+        N = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((total_T, H, dv), dtype=torch.bfloat16, device=q_raw.device)
+    need = int(lib.kda_mixer_fwd_workspace(total_T, N, H, dk, dv))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q_raw.device)
+    _check(lib.kda_mixer_fwd_pooled(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w), _ptr(log_alpha), _ptr(beta),
+                                    _ptr(gate), _ptr(initial_state), _ptr(cu_seqlens), total_T, N, H, dk, dv,
+                                    _ptr(out), _ptr(state_pool), _ptr(conv_pool), _ptr(state_indices),
+                                    state_pool.shape[0], _ptr(workspace), workspace.numel(), _stream(stream)))
+    if check_status:
+        workspace_status(workspace, stream)
+    return out
 
 
 def mixer_decode_step(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, state_pool, conv_pool,

@@ -408,6 +408,59 @@ kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   return ok();
 }
 
+kda_status kda_mixer_fwd_pooled(const void* q_raw, const void* k_raw, const void* v_raw, const float* conv_w,
+                                const float* log_alpha, const float* beta, const void* gate,
+                                const float* initial_state, const int32_t* cu_seqlens, int64_t total_T, int N, int H,
+                                int dk, int dv, void* out, float* state_pool, void* conv_pool,
+                                const int32_t* state_indices, int pool_size, void* workspace, size_t workspace_bytes,
+                                kda_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  kda_status st = check_mixer(q_raw, k_raw, v_raw, conv_w, log_alpha, beta, gate, initial_state, cu_seqlens,
+                              total_T, N, H, dk, dv, out, nullptr);
+  if (st != KDA_OK) return st;
+  if (pool_size < 1) return fail(KDA_ERR_INVALID_ARG, "pool_size=%d must be >= 1", pool_size);
+  if (!state_indices && N > pool_size)
+    return fail(KDA_ERR_INVALID_ARG, "state_indices is NULL but N=%d exceeds pool_size=%d", N, pool_size);
+  if (!state_pool || !conv_pool) return fail(KDA_ERR_INVALID_ARG, "state_pool and conv_pool must be non-NULL");
+  if (!aligned16(state_pool) || !aligned16(conv_pool))
+    return fail(KDA_ERR_INVALID_ARG, "state_pool and conv_pool must be 16-byte aligned");
+  if (state_indices && (reinterpret_cast<uintptr_t>(state_indices) & 3u))
+    return fail(KDA_ERR_INVALID_ARG, "state_indices is not 4-byte aligned");
+  const size_t n_state = static_cast<size_t>(pool_size) * H * dk * dv * sizeof(float);
+  const size_t n_conv = static_cast<size_t>(pool_size) * H * 9 * dk * 2;
+  const size_t n_out = static_cast<size_t>(total_T) * H * dv * 2;
+  const size_t n_h0 = static_cast<size_t>(N) * H * dk * dv * sizeof(float);
+  if (ranges_overlap(state_pool, n_state, conv_pool, n_conv) || ranges_overlap(out, n_out, state_pool, n_state) ||
+      ranges_overlap(out, n_out, conv_pool, n_conv) ||
+      (initial_state && ranges_overlap(initial_state, n_h0, state_pool, n_state)))
+    return fail(KDA_ERR_INVALID_ARG, "out, initial_state, state_pool and conv_pool must not overlap");
+  if (N == 0) return ok();
+  if (workspace && !aligned16(workspace)) return fail(KDA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  const size_t need = kda_mixer_fwd_workspace(total_T, N, H, dk, dv);
+  if (!workspace || workspace_bytes < need)
+    return fail(KDA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? workspace_bytes : 0, need);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  kda::PrefillArgs a{};
+  a.q = q_raw; a.k = k_raw; a.v = v_raw; a.log_alpha = log_alpha; a.beta = beta; a.h0 = initial_state;
+  a.cu = cu_seqlens; a.gate = gate; a.conv_w = conv_w; a.out = out; a.ht = state_pool; a.status = status;
+  a.total_T = total_T; a.N = N; a.H = H;
+  a.slots = state_indices;  // NULL: slot n, and the pool holds at least N states
+  a.pool_size = pool_size;
+  a.in_f32 = false;
+  a.out_f32 = false;
+  if (kda::split_workspace_bytes(total_T, N, H) > 0) a.split_ws = static_cast<char*>(workspace) + kda::kStatusBytes;
+  if (total_T > 0) {
+    e = kda::launch_prefill_d128(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+  }
+  e = kda::launch_pool_store(q_raw, k_raw, v_raw, cu_seqlens, total_T, N, H, state_indices, pool_size, conv_pool,
+                             total_T == 0, initial_state, state_pool, status, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "pool store kernel launch");
+  return ok();
+}
+
 size_t kda_mixer_fwd_gate_workspace(int64_t total_T, int N, int H, int dk, int dv) {
   if (check_common(total_T, N, H, dk, dv) != KDA_OK) return 0;
   if (dk != kda::kD || dv != kda::kD) return 0;

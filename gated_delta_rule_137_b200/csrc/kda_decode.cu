@@ -394,6 +394,63 @@ cudaError_t launch_mixer_decode_commit(const float* state_ckpt, const void* conv
   return cudaGetLastError();
 }
 
+namespace {
+// After a pooled mixer prefill: one CTA of 128 threads per (sequence, head), thread c =
+// channel c. Writes the sequence's last three raw q, k, v rows (oldest first, zeros before
+// its start) into its conv_pool slot, the layout the decode step reads; with copy_states
+// (a call with no tokens), the slot's state becomes h0[n] or zero.
+__global__ void __launch_bounds__(128) pool_store_kernel(const __nv_bfloat16* __restrict__ q,
+                                                         const __nv_bfloat16* __restrict__ k,
+                                                         const __nv_bfloat16* __restrict__ v, const int32_t* cu,
+                                                         int64_t total_T, int N, int H, const int32_t* slots,
+                                                         int pool_size, __nv_bfloat16* conv_pool, bool copy_states,
+                                                         const float* h0, float* state_pool, uint32_t* status) {
+  const int n = blockIdx.x / H, h = blockIdx.x % H, c = threadIdx.x;
+  int64_t bos, eos;
+  if (cu) {
+    bos = __ldg(cu + n);
+    eos = __ldg(cu + n + 1);
+  } else {
+    const int64_t len = total_T / N;
+    bos = n * len;
+    eos = bos + len;
+  }
+  if (bos < 0 || eos < bos || eos > total_T) return;  // bad cu_seqlens: the prefill's plan flags them
+  const int slot = slots ? __ldg(slots + n) : n;
+  if (slot < 0 || slot >= pool_size) {
+    if (c == 0 && status) atomicOr(status, kFlagBadIndex);
+    return;
+  }
+  const __nv_bfloat16* src[3] = {q, k, v};
+  __nv_bfloat16* dst = conv_pool + (static_cast<size_t>(slot) * H + h) * 9 * kD + c;
+#pragma unroll
+  for (int w = 0; w < 3; ++w)
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      const int64_t t = eos - 3 + r;
+      dst[(w * 3 + r) * kD] = t >= bos ? src[w][(static_cast<size_t>(t) * H + h) * kD + c] : __float2bfloat16(0.f);
+    }
+  if (copy_states) {
+    float4* S = reinterpret_cast<float4*>(state_pool + (static_cast<size_t>(slot) * H + h) * kD * kD);
+    const float4* S0 = h0 ? reinterpret_cast<const float4*>(h0 + (static_cast<size_t>(n) * H + h) * kD * kD) : nullptr;
+    for (int i = c; i < kD * kD / 4; i += 128) S[i] = S0 ? S0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+}  // namespace
+
+cudaError_t launch_pool_store(const void* q_raw, const void* k_raw, const void* v_raw, const int32_t* cu,
+                              int64_t total_T, int N, int H, const int32_t* slots, int pool_size, void* conv_pool,
+                              bool copy_states, const float* h0, float* state_pool, uint32_t* status,
+                              cudaStream_t stream) {
+  const unsigned grid = static_cast<unsigned>(N) * static_cast<unsigned>(H);
+  if (grid == 0) return cudaSuccess;
+  pool_store_kernel<<<grid, 128, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(k_raw),
+      static_cast<const __nv_bfloat16*>(v_raw), cu, total_T, N, H, slots, pool_size,
+      static_cast<__nv_bfloat16*>(conv_pool), copy_states, h0, state_pool, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, bool bf16, const float* log_alpha,
                                const float* beta, float* state, int N, int H, int dk, int dv, void* out,
                                cudaStream_t stream) {

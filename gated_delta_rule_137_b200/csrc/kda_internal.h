@@ -50,7 +50,22 @@ struct PrefillArgs {
   float* map_B;           // outputs; half of its value-column slices run from the identity with zero
                           // values (their final states are M [N, H, 128, 128]), the other half from
                           // zero with the real values (B); out, ht and h0 are not used
+  const int32_t* slots;   // int32 [N] or null: sequence n's final state goes to ht slot slots[n]
+  int pool_size;          // (ht then holds pool_size states); a slot outside [0, pool_size) is
+                          // flagged (kFlagBadIndex) and that state is not written
 };
+
+#ifdef __CUDACC__
+// The index of sequence n's final state in a.ht: n, or its pool slot; -1 (nothing is
+// written) for a slot outside the pool, which the thread with `flag` reports.
+__device__ __forceinline__ int64_t final_state_index(const PrefillArgs& a, int n, bool flag) {
+  if (!a.slots) return n;
+  const int s = __ldg(a.slots + n);
+  if (s >= 0 && s < a.pool_size) return s;
+  if (flag && a.status) atomicOr(a.status, kFlagBadIndex);
+  return -1;
+}
+#endif
 
 // ---- two-pass prefill (kda_split.cu) ---------------------------------------------------
 // Pass 1 writes one item of kItemBytes per (chunk, head) — the state-independent part
@@ -116,6 +131,13 @@ cudaError_t launch_mixer_decode_commit(const float* state_ckpt, const void* conv
 cudaError_t launch_state_affine(const float* M, const float* S, const float* B, float* out, int64_t count,
                                 cudaStream_t stream);
 // S <- M_j S + B_j for j = 0 .. maps-1 (MB: [maps][2][count][128][128]; S0 null: zero).
+// The serving hand-off after a pooled mixer prefill: each sequence's last three raw q, k,
+// v rows (zeros before its start) into conv_pool[slot] ([pool, H, 3, 3, 128] bf16); with
+// copy_states, also state_pool[slot] <- h0[n] (or zero), for calls with no tokens.
+cudaError_t launch_pool_store(const void* q_raw, const void* k_raw, const void* v_raw, const int32_t* cu,
+                              int64_t total_T, int N, int H, const int32_t* slots, int pool_size, void* conv_pool,
+                              bool copy_states, const float* h0, float* state_pool, uint32_t* status,
+                              cudaStream_t stream);
 cudaError_t launch_state_fold(const float* MB, int maps, const float* S0, float* out, int64_t count,
                               cudaStream_t stream);
 

@@ -655,9 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- final state: e^{g_last} of the last chunk times D2 --------------------------------
-  if (!failed && a.ht) {
+  const int64_t hn = a.ht ? final_state_index(a, n, tid == 0) : -1;
+  if (!failed && hn >= 0) {
     const float gm = sGamma[gslot * 128 + row];
-    float* ht = a.ht + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0;
+    float* ht = a.ht + ((static_cast<size_t>(hn) * H + h) * kD + row) * kD + col0;
 #pragma unroll
     for (int j = 0; j < kPart; j += 8) {
       const int c = cp * kPart + j;
@@ -723,7 +724,7 @@ cudaError_t launch_types(const PrefillArgs& a, cudaStream_t stream) {
 cudaError_t launch_prefill_d128(const PrefillArgs& a, cudaStream_t stream) {
   if (a.N == 0) return cudaSuccess;
   if (a.total_T == 0) {
-    if (!a.ht) return cudaSuccess;
+    if (!a.ht || a.slots) return cudaSuccess;  // pooled states: launch_pool_store copies them
     const size_t n4 = static_cast<size_t>(a.N) * a.H * kD * kD / 4;
     copy_states_kernel<<<static_cast<unsigned>((n4 + 255) / 256 < 4096 ? (n4 + 255) / 256 : 4096), 256, 0, stream>>>(
         a.h0, a.ht, n4);

@@ -243,7 +243,7 @@ __device__ __noinline__ void raw_rows_front(const RawRowsFront r) {
         float x[4];
         ld4_in(static_cast<const __nv_bfloat16*>(r.a_pre) + static_cast<size_t>(r.t0 + t) * ts + hc, x);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) l[e] = -sc * (fmaxf(x[e], 0.f) + log1pf(__expf(-fabsf(x[e]))));
+        for (int e = 0; e < 4; ++e) l[e] = -sc * softplus_fast(x[e]);
       } else {
         ld4_in(r.log_alpha + static_cast<size_t>(r.t0 + t) * ts + hc, l);
       }
@@ -435,13 +435,13 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
           const bool in = r0 + i < len;
           const size_t o = static_cast<size_t>(t0 + (in ? r0 + i : 0)) * tok_stride + static_cast<size_t>(h) * kD + c0;
           if constexpr (kPre) {
-            // log alpha = -scale * softplus(x), softplus(x) = max(x, 0) + log1p(e^-|x|)
+            // log alpha = -scale * softplus(x)
             const float sc = __ldg(a.a_scale + h);
             float x[4];
             ld4_in(static_cast<const __nv_bfloat16*>(a.a_pre) + o, x);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              la[s][i][e] = in ? -sc * (fmaxf(x[e], 0.f) + log1pf(__expf(-fabsf(x[e])))) : 0.f;
+              la[s][i][e] = in ? -sc * softplus_fast(x[e]) : 0.f;
           } else {
             const float4 l4 = __ldg(reinterpret_cast<const float4*>(a.log_alpha + o));
             la[s][i][0] = in ? l4.x : 0.f; la[s][i][1] = in ? l4.y : 0.f;
@@ -1286,8 +1286,9 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
 
   // ---- final state ---------------------------------------------------------------------------
   float* ht_base = maps ? (map_m ? a.map_M : a.map_B) : a.ht;
-  if (!failed && !issuer_warp && ht_base) {
-    float* ht = ht_base + ((static_cast<size_t>(n) * H + h) * kD + row) * kD + col0;
+  const int64_t hn = ht_base && !maps ? final_state_index(a, n, threadIdx.x == 0) : n;
+  if (!failed && !issuer_warp && ht_base && hn >= 0) {
+    float* ht = ht_base + ((static_cast<size_t>(hn) * H + h) * kD + row) * kD + col0;
 #pragma unroll
     for (int j = 0; j < kPart; j += 8) {
       const int c = cp * kPart + j;

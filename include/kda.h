@@ -314,6 +314,32 @@ KDA_API kda_status kda_mixer_fwd(const void* q_raw, const void* k_raw, const voi
                          void* workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * Full mixer prefill that hands its sequences over to the serving decode
+ * (kda_mixer_decode_step / kda_mixer_decode_tokens): the same computation as
+ * kda_mixer_fwd, but each sequence's final state goes into its slot of state_pool, and
+ * its last three raw q, k, v rows (oldest first, zeros where the prompt is shorter) into
+ * the same slot of conv_pool, the layout the decode step reads. Each sequence starts
+ * with a zero conv history (a new prompt) and from initial_state[n] (or zero).
+ *   state_pool    device fp32 [pool_size, H, d, d]; slots no sequence names are untouched
+ *   conv_pool     device bf16 [pool_size, H, 3, 3, d]
+ *   state_indices device int32 [N]: the slot of each sequence, or NULL for slot n (then
+ *                 pool_size >= N). Slots must be distinct within a call. A slot outside
+ *                 [0, pool_size) sets KDA_DEVFLAG_BAD_INDEX; that sequence's out rows are
+ *                 still written, its pools are not.
+ *   the other arguments and the workspace (kda_mixer_fwd_workspace): as for kda_mixer_fwd.
+ * initial_state, state_pool, conv_pool and out must not overlap. Requires dk = dv = d = 128.
+ * (The article's deployment runs prefill and decode on one cache of states; the pooled
+ * layout and this hand-off are the library's own.)
+ */
+KDA_API kda_status kda_mixer_fwd_pooled(const void* q_raw, const void* k_raw, const void* v_raw,
+                                        const float* conv_w, const float* log_alpha, const float* beta,
+                                        const void* gate, const float* initial_state, const int32_t* cu_seqlens,
+                                        int64_t total_T, int N, int H, int dk, int dv, void* out,
+                                        float* state_pool, void* conv_pool, const int32_t* state_indices,
+                                        int pool_size, void* workspace, size_t workspace_bytes,
+                                        kda_stream_t stream);
+
+/*
  * Full mixer prefill with the decay gate made from its pre-activation (the article's
  * KDA panel names a softplus for the gate; the form read here is one positive scale
  * per head): log_alpha = -a_scale[h] * softplus(a_pre), computed in fp32 as the

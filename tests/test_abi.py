@@ -240,3 +240,33 @@ def test_chunk_bwd_rejects_overlapping_outputs(lib):
     assert call(dla=la + 16 * (tok // 8)) == kda.KDA_ERR_INVALID_ARG  # partly inside log_alpha
     assert call(dk=dq) == kda.KDA_ERR_INVALID_ARG                 # two outputs on each other
     assert call(dbeta=dv + 256) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_mixer_pooled_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, w=FAKE, la=FAKE, b=FAKE, g=None, h0=None, cu=None, T=128, N=2, H=2, dk=128,
+                 dv=128, out=FAKE * 2, sp=FAKE * 256, cp=FAKE * 1024, idx=None, pool=8, ws=FAKE * 3, wsb=1 << 24)
+        a.update(kw)
+        return lib.kda_mixer_fwd_pooled(a["q"], a["k"], a["v"], a["w"], a["la"], a["b"], a["g"], a["h0"], a["cu"],
+                                        a["T"], a["N"], a["H"], a["dk"], a["dv"], a["out"], a["sp"], a["cp"],
+                                        a["idx"], a["pool"], a["ws"], a["wsb"], None)
+    assert call(dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
+    assert call(pool=0) == kda.KDA_ERR_INVALID_ARG
+    assert call(pool=1) == kda.KDA_ERR_INVALID_ARG              # no indices: slot n needs n < pool_size
+    assert call(sp=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(cp=FAKE * 1024 + 8) == kda.KDA_ERR_INVALID_ARG  # misaligned history pool
+    assert call(idx=FAKE + 2) == kda.KDA_ERR_INVALID_ARG        # misaligned indices
+    assert call(out=FAKE * 256) == kda.KDA_ERR_INVALID_ARG      # out overlaps the state pool
+    assert call(h0=FAKE * 256) == kda.KDA_ERR_INVALID_ARG       # the start states inside the pool
+    assert call(wsb=100) == kda.KDA_ERR_WORKSPACE
+    assert call(N=0, T=0) == kda.KDA_OK                         # nothing to do
+
+
+def test_state_fold_rejects_bad_arguments(lib):
+    assert lib.kda_state_fold(FAKE, 2, None, FAKE * 64, 2, 64, None) == kda.KDA_ERR_UNSUPPORTED
+    assert lib.kda_state_fold(FAKE, -1, None, FAKE * 64, 2, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_state_fold(None, 2, None, FAKE * 64, 2, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_state_fold(FAKE, 2, None, FAKE * 64 + 4, 2, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_state_fold(FAKE, 2, None, FAKE * 2, 2, 128, None) == kda.KDA_ERR_INVALID_ARG  # out in the maps
+    assert lib.kda_state_fold(FAKE, 2, FAKE * 64 + 16, FAKE * 64, 2, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_state_fold(None, 0, None, None, 0, 128, None) == kda.KDA_OK  # nothing to do

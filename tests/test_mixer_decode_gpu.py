@@ -8,7 +8,7 @@ import pytest
 
 from gated_delta_rule_137_b200 import inputs as I
 from oracle import kda_oracle as O
-from tests.helpers import assert_decode_out_close, assert_decode_state_close, to_device, to_host
+from tests.helpers import assert_decode_out_close, assert_decode_state_close, assert_prefill_close, to_device, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -172,3 +172,98 @@ def test_mixer_decode_one_token_call_is_the_decode_step(kda):
         outs.append((to_host(o), to_host(sp)))
     np.testing.assert_array_equal(outs[0][0], outs[1][0])
     np.testing.assert_array_equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("lens,H", [([130, 2, 64, 0], 4),   # 16 chains: the two-pass prefill
+                                    ([70] * 19 + [1], 4)])  # 80 chains: the single-pass prefill
+def test_pooled_prefill_hands_over_to_the_decode_step(kda, lens, H):
+    """kda_mixer_fwd_pooled over each sequence's first T tokens into permuted slots of
+    larger pools, then kda_mixer_decode_step on token T + 1, against oracle.kda_mixer over
+    all T + 1 tokens: the prefill's out rows, the pooled states and conv histories after
+    the prefill (histories bit-exact: copies of bf16 inputs, zeros before a short prompt),
+    the decode's out row and the state after it. Slots no sequence names stay untouched.
+    The decode's results sit on a prefill-computed state, so they are held to the prefill's
+    bar."""
+    import torch
+    N, d = len(lens), 128
+    w = I.make_prefill([L + 1 for L in lens], H, d, d, seed=I.SEED_BASE + 43 + N, normalise_qk=False, mixer=True)
+    cu = w.cu_seqlens
+    first = np.concatenate([np.arange(cu[n], cu[n + 1] - 1) for n in range(N)]).astype(np.int64)
+    last = cu[1:] - 1
+    pcu = np.zeros(N + 1, dtype=np.int32)
+    pcu[1:] = np.cumsum(lens)
+    pool = N + 5
+    rng = np.random.default_rng(I.SEED_BASE + 44)
+    slots = rng.permutation(pool)[:N].astype(np.int32)
+    sp0 = rng.standard_normal((pool, H, d, d)).astype(np.float32)
+    cp0 = I.bf16_round(rng.standard_normal((pool, H, 3, 3, d)).astype(np.float32))
+    sp, cp = to_device(sp0, "f32"), to_device(cp0, "bf16")
+    idx = to_device(slots, "i32")
+    cw = to_device(w.conv_w, "f32")
+    sel = lambda x, rows, dt: to_device(x[rows], dt)
+    out = kda.mixer_fwd_pooled(sel(w.q, first, "bf16"), sel(w.k, first, "bf16"), sel(w.v, first, "bf16"), cw,
+                               sel(w.log_alpha, first, "f32"), sel(w.beta, first, "f32"), sel(w.gate, first, "bf16"),
+                               sp, cp, idx, to_device(w.initial_state, "f32"), to_device(pcu, "i32"), N=N,
+                               check_status=True)
+    torch.cuda.synchronize()
+    sp_pre, cp_pre = to_host(sp), cp.view(torch.int16).cpu().numpy().view(np.uint16).copy()
+    status = torch.zeros(64, dtype=torch.int32, device="cuda")
+    dout = kda.mixer_decode_step(sel(w.q, last, "bf16"), sel(w.k, last, "bf16"), sel(w.v, last, "bf16"), cw,
+                                 sel(w.log_alpha, last, "f32"), sel(w.beta, last, "f32"), sel(w.gate, last, "bf16"),
+                                 sp, cp, idx, status=status)
+    torch.cuda.synchronize()
+    assert int(to_host(status)[0]) == 0
+
+    pre = [w.q[first], w.k[first], w.v[first], w.conv_w, w.log_alpha[first], w.beta[first], w.gate[first], pcu]
+    ro_pre, rf_pre = O.kda_mixer(*pre, initial_state=w.initial_state)
+    ro, rf = O.kda_mixer(w.q, w.k, w.v, w.conv_w, w.log_alpha, w.beta, w.gate, cu, initial_state=w.initial_state)
+    assert_prefill_close(to_host(out), ro_pre, "pooled prefill out", stored_bf16=True)
+    assert_prefill_close(sp_pre[slots], rf_pre, "pooled prefill state")
+    assert_prefill_close(to_host(dout), ro[last], "decode out after the prefill", stored_bf16=True)
+    assert_prefill_close(to_host(sp)[slots], rf, "state after prefill + decode")
+
+    def history(rows_of):  # the last three raw rows of each sequence, oldest first, zeros before it
+        h = np.zeros((N, H, 3, 3, d))
+        for n in range(N):
+            rows = rows_of(n)
+            for r in range(3):
+                t = len(rows) - 3 + r
+                if t >= 0:
+                    for i, x in enumerate((w.q, w.k, w.v)):
+                        h[n, :, i, r] = x[rows[t]]
+        return h
+
+    np.testing.assert_array_equal(cp_pre[slots], I.bf16_bits(history(lambda n: np.arange(cu[n], cu[n + 1] - 1))))
+    got_h = cp.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got_h[slots], I.bf16_bits(history(lambda n: np.arange(cu[n], cu[n + 1]))))
+    unused = np.setdiff1d(np.arange(pool), slots)
+    np.testing.assert_array_equal(to_host(sp)[unused], sp0[unused])
+    np.testing.assert_array_equal(got_h[unused], I.bf16_bits(cp0[unused]))
+
+
+def test_pooled_prefill_flags_a_slot_outside_the_pool(kda):
+    """A slot outside [0, pool_size) is reported and that sequence's pools are left alone;
+    the other sequences are handed over as usual and every out row is written."""
+    import torch
+    lens, H, d = [40, 90], 2, 128
+    w = I.make_prefill(lens, H, d, d, seed=I.SEED_BASE + 45, normalise_qk=False, mixer=True)
+    pool = 3
+    sp0 = np.zeros((pool, H, d, d), np.float32)
+    cp0 = np.zeros((pool, H, 3, 3, d), np.float32)
+    sp, cp = to_device(sp0, "f32"), to_device(cp0, "bf16")
+    ws = torch.empty(kda.load_library().kda_mixer_fwd_workspace(w.total_T, 2, H, d, d), dtype=torch.uint8,
+                     device="cuda")
+    out = kda.mixer_fwd_pooled(to_device(w.q, "bf16"), to_device(w.k, "bf16"), to_device(w.v, "bf16"),
+                               to_device(w.conv_w, "f32"), to_device(w.log_alpha, "f32"), to_device(w.beta, "f32"),
+                               to_device(w.gate, "bf16"), sp, cp, to_device(np.array([7, 1], np.int32), "i32"),
+                               to_device(w.initial_state, "f32"), to_device(w.cu_seqlens, "i32"), N=2, workspace=ws)
+    torch.cuda.synchronize()
+    with pytest.raises(kda.KdaError) as err:
+        kda.workspace_status(ws)
+    assert int(str(err.value).split("0x")[-1][:8], 16) == kda.DEVFLAG_BAD_INDEX
+    ro, rf = O.kda_mixer(w.q, w.k, w.v, w.conv_w, w.log_alpha, w.beta, w.gate, w.cu_seqlens,
+                         initial_state=w.initial_state)
+    assert_prefill_close(to_host(out), ro, "out", stored_bf16=True)
+    assert_prefill_close(to_host(sp)[1], rf[1], "state of the valid slot")
+    np.testing.assert_array_equal(to_host(sp)[[0, 2]], 0.0)
+    np.testing.assert_array_equal(to_host(cp)[[0, 2]], 0.0)
