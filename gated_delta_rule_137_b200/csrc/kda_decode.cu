@@ -338,6 +338,283 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2) mixer_decode_kernel(cons
   }
 }
 
+// K = 2..4 tokens of one (sequence, head) with a single pass over the state (512 threads:
+// 16 warps of 8 state rows, so that the 2K column sums fit in registers): the K-token
+// block of the recurrence in the WY form the chunked prefill uses (chunk size K), with
+// every product on the CUDA cores. Per key channel r, with tokens j = 0..K-1,
+//   c_j = alpha_0 ... alpha_j,   D(i, j) = alpha_{i+1} ... alpha_j   (D(j, j) = 1),
+//   S'_j = Diag(c_j) S_0 + sum_{i<j} Diag(D(i, j)) k_i u_i^T   (the state before token j
+//          is read, after its decay),
+//   a_j = S'_j^T k_j = S_0^T (c_j k_j) + sum_{i<j} G_ji u_i,   G_ji = sum_r k_j k_i D(i, j),
+//   u_j = beta_j (v_j - a_j),
+//   o_j = S_j^T q_j = S_0^T (c_j q_j) + sum_{i<=j} Q_ji u_i,   Q_ji = sum_r q_j k_i D(i, j),
+//   S_j = Diag(c_j) S_0 + sum_{i<=j} Diag(D(i, j)) k_i u_i^T.
+// One pass over S_0 gives the 2K column sums S_0^T (c_j k_j), S_0^T (c_j q_j); the K x K
+// terms come from the token vectors alone, so the tokens' dependency runs through
+// K x 4 numbers per thread instead of the state. The conv, L2 norm and gate are those of
+// mixer_decode_kernel; the state after every token is written only with checkpoints.
+constexpr int kBlockWarps = 16;  // 512 threads, 8 state rows per warp
+constexpr int kBlockRows = kMixD / kBlockWarps;
+template <int KB>
+struct BlockSmem {
+  static constexpr int kC1 = (2 * KB + 3) & ~3;  // per key row: c_j k_j, c_j q_j (padded)
+  static constexpr int kC2 = (KB + 1 + 3) & ~3;  // per key row: c_{K-1}, D(j, K-1) k_j
+  static constexpr int kCk = KB * (KB + 1);      // per key row and token j: c_j, D(i, j) k_i (i <= j)
+  static constexpr int kPairs = KB * KB;         // G_ji (i < j) and Q_ji (i <= j)
+  float v[KB][kMixD];
+  float ss[KB][2][4];
+  float pair[kPairs][4];
+  float pairT[kPairs];
+  alignas(16) float c1[kMixD][kC1];
+  alignas(16) float c2[kMixD][kC2];
+  float ck[kMixD][kCk];
+  float4 red[2 * KB][kBlockWarps][32];
+  float4 sum[2 * KB][32];
+};
+
+// G_ji (i < j) at index j * K + i, Q_ji (i <= j) at index i * K + j (the upper triangle)
+template <int KB>
+__host__ __device__ constexpr int g_index(int j, int i) { return j * KB + i; }
+template <int KB>
+__host__ __device__ constexpr int q_index(int j, int i) { return i * KB + j; }
+
+template <int KB>
+__global__ void __launch_bounds__(kBlockWarps * 32, 1) mixer_decode_block_kernel(const MixerDecodeArgs a) {
+  using SM = BlockSmem<KB>;
+  extern __shared__ __align__(16) uint8_t block_smem_raw[];
+  SM& sm = *reinterpret_cast<SM*>(block_smem_raw);
+  const int nh = blockIdx.x;  // n * H + h
+  const int H = a.H;
+  const int n = nh / H, h = nh % H;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int col = lane * 4;
+  const int slot = a.state_indices ? a.state_indices[n] : n;
+  if (slot < 0 || slot >= a.pool_size) {  // the whole CTA takes this branch
+    if (threadIdx.x == 0 && a.status) atomicOr(a.status, kFlagBadIndex);
+    return;
+  }
+  float* S = a.state_pool + (static_cast<size_t>(slot) * H + h) * kMixD * kMixD;
+  __nv_bfloat16* hist = a.conv_pool + (static_cast<size_t>(slot) * H + h) * (3 * 3 * kMixD);
+
+  // ---- the K tokens' conv (q, k: threads 0..127; v: 128..255), L2 sums, decays --------
+  const int i = threadIdx.x, c = i & (kMixD - 1);
+  const int t0 = i < kMixD ? 0 : 2;
+  const int nt = i < kMixD ? 2 : (i < 2 * kMixD ? 1 : 0);  // threads 256.. join at the state pass
+  float y[2][KB];
+  const float* cwp = a.conv_w + (static_cast<size_t>(t0) * H + h) * kMixD * 4 + c * 4;
+  const __nv_bfloat16* raw0 = i < kMixD ? a.q_raw : a.v_raw;
+  // raw row m of this thread's tensor u: the three of the history, then the K tokens' (read
+  // again for the history written at the end, so that they need no registers meanwhile)
+  auto raw_row = [&](int u, int m) -> __nv_bfloat16 {
+    if (m < 3) return hist[((t0 + u) * 3 + m) * kMixD + c];
+    const __nv_bfloat16* src = u == 0 ? raw0 : a.k_raw;
+    return src[((static_cast<size_t>(n) * KB + (m - 3)) * H + h) * kMixD + c];
+  };
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    if (u >= nt) break;
+    float xr[3 + KB];
+#pragma unroll
+    for (int m = 0; m < 3 + KB; ++m) xr[m] = __bfloat162float(raw_row(u, m));
+    const float4 cw = __ldg(reinterpret_cast<const float4*>(cwp + static_cast<size_t>(u) * H * kMixD * 4));
+#pragma unroll
+    for (int j = 0; j < KB; ++j)
+      y[u][j] = fmaf(cw.x, xr[j], fmaf(cw.y, xr[j + 1], fmaf(cw.z, xr[j + 2], cw.w * xr[j + 3])));
+  }
+  float al[KB];
+  if (i < kMixD) {
+#pragma unroll
+    for (int j = 0; j < KB; ++j) {
+      al[j] = expf(a.log_alpha[((static_cast<size_t>(n) * KB + j) * H + h) * kMixD + c]);
+      const float sq = warp_sum(y[0][j] * y[0][j]), sk = warp_sum(y[1][j] * y[1][j]);
+      if (lane == 0) {
+        sm.ss[j][0][warp] = sq;
+        sm.ss[j][1][warp] = sk;
+      }
+    }
+  } else if (i < 2 * kMixD) {
+#pragma unroll
+    for (int j = 0; j < KB; ++j) sm.v[j][c] = y[0][j];
+  }
+  float bt[KB];
+#pragma unroll
+  for (int j = 0; j < KB; ++j) bt[j] = a.beta[(static_cast<size_t>(n) * KB + j) * H + h];
+  __syncthreads();
+
+  // ---- per key channel: the coefficient rows and the K x K terms (threads 0..127) --------
+  if (i < kMixD) {
+    float q[KB], k[KB], cc[KB];
+#pragma unroll
+    for (int j = 0; j < KB; ++j) {
+      q[j] = y[0][j] * rsqrtf(sm.ss[j][0][0] + sm.ss[j][0][1] + sm.ss[j][0][2] + sm.ss[j][0][3] + 1e-6f);
+      k[j] = y[1][j] * rsqrtf(sm.ss[j][1][0] + sm.ss[j][1][1] + sm.ss[j][1][2] + sm.ss[j][1][3] + 1e-6f);
+      cc[j] = j == 0 ? al[0] : cc[j - 1] * al[j];
+      sm.c1[c][j] = cc[j] * k[j];
+      sm.c1[c][KB + j] = cc[j] * q[j];
+    }
+    sm.c2[c][0] = cc[KB - 1];
+#pragma unroll
+    for (int j = 0; j < KB; ++j) {
+      // D(i, j) for i = j, j-1, .., 0: the decays after token i up to token j
+      float d = 1.f;
+      sm.ck[c][j * (KB + 1)] = cc[j];
+#pragma unroll
+      for (int ii = j; ii >= 0; --ii) {
+        sm.ck[c][j * (KB + 1) + 1 + ii] = d * k[ii];
+        const float qp = warp_sum(q[j] * k[ii] * d);
+        if (lane == 0) sm.pair[q_index<KB>(j, ii)][warp] = qp;
+        if (ii < j) {
+          const float gp = warp_sum(k[j] * k[ii] * d);
+          if (lane == 0) sm.pair[g_index<KB>(j, ii)][warp] = gp;
+        }
+        if (ii > 0) d *= al[ii];
+      }
+      if (j == KB - 1) {
+        float e = 1.f;
+#pragma unroll
+        for (int ii = KB - 1; ii >= 0; --ii) {
+          sm.c2[c][1 + ii] = e * k[ii];
+          if (ii > 0) e *= al[ii];
+        }
+      }
+    }
+  }
+  // the state slice of this warp (loaded once the token vectors are done with their
+  // registers; the other resident CTAs keep HBM busy meanwhile)
+  float4 s[kBlockRows];
+#pragma unroll
+  for (int r = 0; r < kBlockRows; ++r)
+    s[r] = __ldcs(reinterpret_cast<const float4*>(S + static_cast<size_t>(warp * kBlockRows + r) * kMixD + col));
+  __syncthreads();
+  if (threadIdx.x < SM::kPairs)
+    sm.pairT[threadIdx.x] = sm.pair[threadIdx.x][0] + sm.pair[threadIdx.x][1] + sm.pair[threadIdx.x][2] +
+                            sm.pair[threadIdx.x][3];
+
+  // ---- one pass over S_0: the 2K column sums --------------------------------------------
+  float4 acc[2 * KB];
+#pragma unroll
+  for (int v = 0; v < 2 * KB; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int r = 0; r < kBlockRows; ++r) {
+    const float* cr = sm.c1[warp * kBlockRows + r];
+#pragma unroll
+    for (int v = 0; v < 2 * KB; ++v) {
+      const float w = cr[v];
+      acc[v].x = fmaf(w, s[r].x, acc[v].x); acc[v].y = fmaf(w, s[r].y, acc[v].y);
+      acc[v].z = fmaf(w, s[r].z, acc[v].z); acc[v].w = fmaf(w, s[r].w, acc[v].w);
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < 2 * KB; ++v) sm.red[v][warp][lane] = acc[v];
+  __syncthreads();
+  for (int v = warp; v < 2 * KB; v += kBlockWarps) {
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kBlockWarps; ++w) {
+      const float4 x = sm.red[v][w][lane];
+      t.x += x.x; t.y += x.y; t.z += x.z; t.w += x.w;
+    }
+    sm.sum[v][lane] = t;
+  }
+  __syncthreads();
+
+  // ---- the K tokens' u and o for this lane's four value columns ---------------------------
+  float4 uu[KB];
+#pragma unroll
+  for (int j = 0; j < KB; ++j) {
+    float4 t = sm.sum[j][lane];  // S_0^T (c_j k_j)
+#pragma unroll
+    for (int ii = 0; ii < j; ++ii) {
+      const float g = sm.pairT[g_index<KB>(j, ii)];
+      t.x = fmaf(g, uu[ii].x, t.x); t.y = fmaf(g, uu[ii].y, t.y);
+      t.z = fmaf(g, uu[ii].z, t.z); t.w = fmaf(g, uu[ii].w, t.w);
+    }
+    const float4 vv = *reinterpret_cast<const float4*>(&sm.v[j][col]);
+    uu[j] = make_float4(bt[j] * (vv.x - t.x), bt[j] * (vv.y - t.y), bt[j] * (vv.z - t.z), bt[j] * (vv.w - t.w));
+  }
+  if (warp < KB) {  // warp j writes token j's output row
+    const int j = warp;
+    float4 o = sm.sum[KB + j][lane];  // S_0^T (c_j q_j)
+#pragma unroll
+    for (int ii = 0; ii < KB; ++ii) {
+      if (ii > j) break;
+      const float qv = sm.pairT[q_index<KB>(j, ii)];
+      o.x = fmaf(qv, uu[ii].x, o.x); o.y = fmaf(qv, uu[ii].y, o.y);
+      o.z = fmaf(qv, uu[ii].z, o.z); o.w = fmaf(qv, uu[ii].w, o.w);
+    }
+    float ov[4] = {o.x, o.y, o.z, o.w};
+    const size_t oo = ((static_cast<size_t>(n) * KB + j) * H + h) * kMixD + col;
+    if (a.gate) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ov[e] *= 1.f / (1.f + expf(-__bfloat162float(a.gate[oo + e])));
+    }
+    store4<__nv_bfloat16>(a.out + oo, make_float4(ov[0], ov[1], ov[2], ov[3]));
+  }
+
+  // ---- the states after the tokens: every one with checkpoints, else the last -------------
+  if (a.state_ckpt) {
+#pragma unroll
+    for (int j = 0; j < KB; ++j) {
+      float* C = a.state_ckpt + ((static_cast<size_t>(n) * KB + j) * H + h) * kMixD * kMixD;
+#pragma unroll
+      for (int r = 0; r < kBlockRows; ++r) {
+        const int row = warp * kBlockRows + r;
+        const float* ck = sm.ck[row] + j * (KB + 1);
+        float4 x = make_float4(ck[0] * s[r].x, ck[0] * s[r].y, ck[0] * s[r].z, ck[0] * s[r].w);
+#pragma unroll
+        for (int ii = 0; ii <= j; ++ii) {
+          const float w = ck[1 + ii];
+          x.x = fmaf(w, uu[ii].x, x.x); x.y = fmaf(w, uu[ii].y, x.y);
+          x.z = fmaf(w, uu[ii].z, x.z); x.w = fmaf(w, uu[ii].w, x.w);
+        }
+        __stcs(reinterpret_cast<float4*>(C + static_cast<size_t>(row) * kMixD + col), x);
+      }
+      __nv_bfloat16* hc = a.conv_ckpt + ((static_cast<size_t>(n) * KB + j) * H + h) * (3 * 3 * kMixD) + c;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (u >= nt) break;
+#pragma unroll
+        for (int m = 0; m < 3; ++m) hc[((t0 + u) * 3 + m) * kMixD] = raw_row(u, j + 1 + m);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < kBlockRows; ++r) {
+      const int row = warp * kBlockRows + r;
+      const float* c2 = sm.c2[row];
+      float4 x = make_float4(c2[0] * s[r].x, c2[0] * s[r].y, c2[0] * s[r].z, c2[0] * s[r].w);
+#pragma unroll
+      for (int ii = 0; ii < KB; ++ii) {
+        const float w = c2[1 + ii];
+        x.x = fmaf(w, uu[ii].x, x.x); x.y = fmaf(w, uu[ii].y, x.y);
+        x.z = fmaf(w, uu[ii].z, x.z); x.w = fmaf(w, uu[ii].w, x.w);
+      }
+      __stcs(reinterpret_cast<float4*>(S + static_cast<size_t>(row) * kMixD + col), x);
+    }
+    // the last three raw rows (read before any is written: for K < 3 some come from the history)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u >= nt) break;
+      __nv_bfloat16 last[3];
+#pragma unroll
+      for (int m = 0; m < 3; ++m) last[m] = raw_row(u, KB + m);
+#pragma unroll
+      for (int m = 0; m < 3; ++m) hist[((t0 + u) * 3 + m) * kMixD + c] = last[m];
+    }
+  }
+}
+
+template <int KB>
+cudaError_t launch_block(const MixerDecodeArgs& a, unsigned grid, cudaStream_t stream) {
+  constexpr int kSmem = static_cast<int>(sizeof(BlockSmem<KB>));
+  static cudaError_t attr = cudaFuncSetAttribute(mixer_decode_block_kernel<KB>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (attr != cudaSuccess) return attr;
+  mixer_decode_block_kernel<KB><<<grid, kBlockWarps * 32, kSmem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 // Commit after speculative decoding: slot <- the checkpoint after token accepted[n] - 1
 // (accepted[n] = 0 keeps the slot as it is). One CTA per (n, h) copies 64 KiB of state
 // and the 2.25 KiB history.
@@ -376,6 +653,11 @@ cudaError_t launch_mixer_decode(const void* q_raw, const void* k_raw, const void
                     static_cast<const __nv_bfloat16*>(gate), state_pool, static_cast<__nv_bfloat16*>(conv_pool),
                     state_indices, state_ckpt, static_cast<__nv_bfloat16*>(conv_ckpt),
                     static_cast<__nv_bfloat16*>(out), status, pool_size, K, H};
+  // K = 2..4: the block form (one pass over the state); longer runs of tokens step through
+  // them one at a time
+  if (K == 2) return launch_block<2>(a, grid, stream);
+  if (K == 3) return launch_block<3>(a, grid, stream);
+  if (K == 4) return launch_block<4>(a, grid, stream);
   if (K == 1 && !state_ckpt)
     mixer_decode_kernel<true><<<grid, kDecodeWarps * 32, 0, stream>>>(a);
   else

@@ -194,8 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t tok_stride = static_cast<int64_t>(H) * kD;  // elements between tokens
 
   constexpr uint32_t kIdAP = idesc_tf32(128, 64, false, false);
-  constexpr uint32_t kIdW = idesc_tf32(128, 128, false, false);
-  constexpr uint32_t kIdV = idesc_tf32(128, DV, false, false);
+  // the B operands Kt, V, S and U are MN-major, and so is Kh^T as the A of Kh^T U
+  constexpr uint32_t kIdW = idesc_tf32(128, 128, false, true);
+  constexpr uint32_t kIdV = idesc_tf32(128, DV, false, true);
+  constexpr uint32_t kIdVmn = idesc_tf32(128, DV, true, true);
 
   uint32_t mma_phase = 0, tma_phase = 0;
   bool failed = false;
@@ -378,36 +380,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<float4*>(sLAr + r * kD + c0) = in ? la4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       } else {
-        float kt[4][4], kh[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float qt[4];
+          float kt[4], kh[4], qt[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float g = pre[e] + la[i][e];
             const float eg = __expf(g), eng = __expf(-g);
-            kt[i][e] = kv[i][e] * eg;
-            kh[i][e] = to_tf32(kv[i][e] * eng);
+            kt[e] = kv[i][e] * eg;
+            kh[e] = to_tf32(kv[i][e] * eng);
             qt[e] = qv[i][e] * eg;
           }
           const int r = r0 + i;
-          st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[i][0], kt[i][1], kt[i][2], kt[i][3]);    // Kt [tok][ch]
-          st4_tf32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);          // Qt [tok][ch]
-          st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);     // Kh [tok][ch]
-        }
-        // channel-major copies: channel c0+e, tokens r0..r0+3; lanes rotate e so that one
-        // store instruction touches different swizzle rows
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int e = (j + lane) & 3;
-          float x[4], y[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            x[i] = e == 0 ? kt[i][0] : e == 1 ? kt[i][1] : e == 2 ? kt[i][2] : kt[i][3];
-            y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
-          }
-          st4_f32(sm + SM::kKTT, f32_offset(c0 + e, r0, 128), x[0], x[1], x[2], x[3]);    // Kt^T [ch][tok]
-          st4_f32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);    // Kh^T [ch][tok]
+          st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[0], kt[1], kt[2], kt[3]);           // Kt [tok][ch]
+          st4_tf32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);     // Qt [tok][ch]
+          st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[0], kh[1], kh[2], kh[3]);            // Kh [tok][ch]
+          // the same rows as lines of the MN-major operands: Kt of T Kt, Kh (Kh^T) of Kh^T U
+          st4_f32(sm + SM::kKTT, mn_offset(r, c0, 64), kt[0], kt[1], kt[2], kt[3]);
+          st4_f32(sm + SM::kKHT, mn_offset(r, c0, 64), kh[0], kh[1], kh[2], kh[3]);
         }
       }  // factorised form
     }
@@ -442,8 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           float* vr = reinterpret_cast<float*>(sm + SM::kVT);
 #pragma unroll
           for (int e = 0; e < 4; ++e) vr[(t4 + e) * DV + j] = x[e];
-        } else {
-          st4_tf32(sm + SM::kVT, f32_offset(j, t4, DV), x[0], x[1], x[2], x[3]);
+        } else {  // lines of the MN-major B operand of T V (a warp writes 32 columns of a token)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) st_tf32(sm + SM::kVT, mn_offset(t4 + e, j, kChunk), x[e]);
         }
       }
     }
@@ -536,13 +527,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -- 7. D0 = [W; -] = [T; P] Kt   and   D3 = [U~; -] = [T; P] V -------------------------
     if (tid == 0) {
       tc_fence_after_sync();
-      const uint64_t a0 = kdesc0(sb + SM::kTP), b0 = kdesc0(sb + SM::kKTT), v0 = kdesc0(sb + SM::kVT);
+      const uint64_t a0 = kdesc0(sb + SM::kTP);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_tf32(tmem + TM::kD0, a0 + kstep(kk, 128), b0 + kstep(kk, 128), kIdW, kk > 0);
+        umma_tf32(tmem + TM::kD0, a0 + kstep(kk, 128), mndesc(sb + SM::kKTT, kChunk, kk), kIdW, kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_tf32(tmem + TM::kD3, a0 + kstep(kk, 128), v0 + kstep(kk, DV), kIdV, kk > 0);
+        umma_tf32(tmem + TM::kD3, a0 + kstep(kk, 128), mndesc(sb + SM::kVT, kChunk, kk), kIdV, kk > 0);
       umma_commit(bar_mma);
     }
     wait_mma();
@@ -570,10 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld8(tmem + lane_off + TM::kD2 + c, x);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x[e] *= gm;
-          *reinterpret_cast<float*>(sm + SM::kST + f32_offset(c + e, row, DV)) = x[e];
-        }
+        for (int e = 0; e < 8; ++e) x[e] *= gm;
+        st8_line(sm + SM::kST, row, c, kD, x, false);  // row `row` of the MN-major S operand
         tmem_st8(tmem + lane_off + TM::kD2 + c, x);
       }
       tmem_st_wait();
@@ -585,10 +574,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -- 9. D1 = [-W S; Qt S] ----------------------------------------------------------------
     if (tid == 0) {
       tc_fence_after_sync();
-      const uint64_t a0 = kdesc0(sb + SM::kKQ), b0 = kdesc0(sb + SM::kST);
+      const uint64_t a0 = kdesc0(sb + SM::kKQ);
 #pragma unroll
       for (int kk = 0; kk < 16; ++kk)
-        umma_tf32(tmem + TM::kD1, a0 + kstep(kk, 128), b0 + kstep(kk, DV), kIdV, kk > 0);
+        umma_tf32(tmem + TM::kD1, a0 + kstep(kk, 128), mndesc(sb + SM::kST, kD, kk), kIdV, kk > 0);
       umma_commit(bar_mma);
     }
     if (t0 + kChunk < eos) {  // next chunk's gate inputs, in flight during the MMAs
@@ -606,8 +595,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld8(tmem + lane_off + TM::kD3 + c, ut);
         tmem_ld8(tmem + lane_off + TM::kD1 + c, ws);
         tmem_ld_wait();
+        float u[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) st_tf32(sm + SM::kVT, f32_offset(c + e, row, DV), ut[e] + ws[e]);
+        for (int e = 0; e < 8; ++e) u[e] = ut[e] + ws[e];
+        st8_line(sm + SM::kVT, row, c, kChunk, u, true);  // row `row` of the MN-major U operand
       }
     }
     fence_proxy_async_smem();
@@ -617,13 +608,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -- 11. D2 = S + Kh^T U ;  D1 += [T; P] U  ->  O = Qt S + P U in rows 64..127 ------------
     if (tid == 0) {
       tc_fence_after_sync();
-      const uint64_t a0 = kdesc0(sb + SM::kKHT), b0 = kdesc0(sb + SM::kVT), t0d = kdesc0(sb + SM::kTP);
+      const uint64_t t0d = kdesc0(sb + SM::kTP);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_tf32(tmem + TM::kD2, a0 + kstep(kk, 128), b0 + kstep(kk, DV), kIdV, 1u);
+        umma_tf32(tmem + TM::kD2, mndesc(sb + SM::kKHT, kChunk, kk), mndesc(sb + SM::kVT, kChunk, kk), kIdVmn, 1u);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_tf32(tmem + TM::kD1, t0d + kstep(kk, 128), b0 + kstep(kk, DV), kIdV, 1u);
+        umma_tf32(tmem + TM::kD1, t0d + kstep(kk, 128), mndesc(sb + SM::kVT, kChunk, kk), kIdV, 1u);
       umma_commit(bar_mma);
     }
     wait_mma();

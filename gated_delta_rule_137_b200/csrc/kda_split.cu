@@ -578,31 +578,23 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
                 qv[i][e] = rin[i] ? unpack(qraw[i], e) : 0.f;
               }
           }
-          float kh[4][4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            float kt[4], qt[4];
+            float kt[4], qt[4], kh[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float g = pre[s][e] + la[s][i][e];
               const float eg = __expf(g), eng = __expf(-g);
               kt[e] = kv[i][e] * eg;
-              kh[i][e] = to_tf32(kv[i][e] * eng);
+              kh[e] = to_tf32(kv[i][e] * eng);
               qt[e] = to_tf32(qv[i][e] * eg);
             }
             const int r = r0 + i;
-            st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[0], kt[1], kt[2], kt[3]);          // Kt [tok][ch]
-            st4_f32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);     // Qt [tok][ch]
-            st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[i][0], kh[i][1], kh[i][2], kh[i][3]);  // Kh [tok][ch]
-          }
-          // Kh^T (staged for the item): channel c0+e, tokens r0..r0+3
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int e = (j + lane) & 3;
-            float y[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) y[i] = e == 0 ? kh[i][0] : e == 1 ? kh[i][1] : e == 2 ? kh[i][2] : kh[i][3];
-            st4_f32(sm + SM::kKHT, f32_offset(c0 + e, r0, 128), y[0], y[1], y[2], y[3]);
+            st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[0], kt[1], kt[2], kt[3]);       // Kt [tok][ch]
+            st4_f32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);  // Qt [tok][ch]
+            st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[0], kh[1], kh[2], kh[3]);        // Kh [tok][ch]
+            // the same rows for the item: Kh as the MN-major A operand (Kh^T) of the state update
+            st4_f32(sm + SM::kKHT, mn_offset(r, c0, 64), kh[0], kh[1], kh[2], kh[3]);
           }
         }
       }  // factorised form
@@ -635,19 +627,90 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         }
       }
 
-      // -- Kt^T, once the back group's previous W / U~ MMA and its staging have let go of KTT --
+      // the V rows this thread turns into operand lines below (4-token x 4-column blocks, all
+      // their rows in flight at once; they were warmed into L2): for plain bf16 inputs they
+      // are loaded before waiting for VT; with the conv's extra rows (or fp32 inputs) after
+      // it, where fewer registers are live
+      constexpr int kW = sizeof(TIn);  // 32-bit words per 4 elements
+      constexpr bool kEarlyV = !kConv && kW == 2;
+      uint32_t vraw[2][kGRows][kW];
+      auto load_v = [&] {
+        const TIn* vh = vg + static_cast<size_t>(h) * kD;
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int blk = ftid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+#pragma unroll
+          for (int m = 0; m < kGRows; ++m) {
+            const int rr = t4 - kHist + m;
+            const bool in = rr < len && t0 + rr >= bos;
+            const TIn* src = vh + static_cast<size_t>(in ? t0 + rr : t0) * tok_stride + j4;
+            if constexpr (kW == 2) {
+              const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
+              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
+            } else {
+              const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
+              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
+              vraw[bb][m][2] = in ? x.z : 0u; vraw[bb][m][3] = in ? x.w : 0u;
+            }
+          }
+        }
+      };
+      if (kEarlyV && !strong) load_v();
+
+      // -- Kt and V, once the back group's previous W / U~ MMA and its staging have let go of
+      //    KTT and VT --------------------------------------------------------------------------
       if (k > 0) {
         if (ftid == 0 && !lost && !mbar_wait(bars + kBWFree, ph_wfree, a.status)) lost = true;
         ph_wfree ^= 1u;
         fsync();
       }
-      for (int i = ftid; i < (strong ? 0 : kD * 16); i += kGroupThreads) {  // Kt (rows 0..63 of KQ) -> Kt^T
-        const int c = i % kD, r4 = (i / kD) * 4;
-        const float* kq = reinterpret_cast<const float*>(sm + SM::kKQ);
-        st4_f32(sm + SM::kKTT, f32_offset(c, r4, 128), kq[f32_offset(r4, c, 128) >> 2],
-                kq[f32_offset(r4 + 1, c, 128) >> 2], kq[f32_offset(r4 + 2, c, 128) >> 2],
-                kq[f32_offset(r4 + 3, c, 128) >> 2]);
+      for (int i = ftid; i < (strong ? 0 : kChunk * 32); i += kGroupThreads) {
+        // Kt (rows 0..63 of KQ) -> the MN-major B operand of T Kt, 4 channels at a time
+        const int r = i >> 5, c = 4 * (i & 31);
+        *reinterpret_cast<float4*>(sm + SM::kKTT + mn_offset(r, c, 64)) =
+            *reinterpret_cast<const float4*>(sm + SM::kKQ + f32_offset(r, c, 128));
       }
+      // V rows (tf32; conv for the mixer) as the MN-major B operand of T V: each thread takes
+      // 4-token x 4-column blocks (their rows loaded above)
+      if (!strong) {
+        if constexpr (!kEarlyV) load_v();
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int blk = ftid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+          auto elem = [&](int jr, int m) -> float {  // column j4 + jr of loaded row m
+            if constexpr (kW == 2) {
+              const uint32_t x = vraw[bb][m][jr >> 1];
+              return __uint_as_float((jr & 1) ? (x & 0xFFFF0000u) : (x << 16));
+            } else {
+              return __uint_as_float(vraw[bb][m][jr]);
+            }
+          };
+          float4 wv[kConv ? 4 : 1];  // conv taps of columns j4 .. j4 + 3
+          if constexpr (kConv) {
+#pragma unroll
+            for (int jr = 0; jr < 4; ++jr)
+              wv[jr] = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((2 * H + h) * kD + j4 + jr) * 4));
+          }
+          // V rows t4 .. t4 + 3 as whole lines of the MN-major B operand of T V
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float y[4];
+#pragma unroll
+            for (int jr = 0; jr < 4; ++jr) {
+              if constexpr (kConv) {
+                const float4 w4 = wv[jr];
+                const float yc = fmaf(w4.x, elem(jr, e), fmaf(w4.y, elem(jr, e + 1),
+                                                              fmaf(w4.z, elem(jr, e + 2), w4.w * elem(jr, e + 3))));
+                y[jr] = (t4 + e < len) ? yc : 0.f;
+              } else {
+                y[jr] = elem(jr, e);
+              }
+            }
+            st4_tf32(sm + SM::kVT, mn_offset(t4 + e, j4, 64), y[0], y[1], y[2], y[3]);
+          }
+        }
+      }
+
       fence_proxy_async_smem();
       fsync();
       if (ftid == 0) mbar_arrive(bars + kBVtFull);
@@ -665,9 +728,8 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
     float* sY = sA + 64 * kLd;                            // [32][kLd]
     uint32_t ph_apfull = 0, ph_vtfull = 0, ph_wu = 0;
     auto bsync = [] { group_sync(kBarBack, kGroupThreads); };
-    constexpr uint32_t kIdN128 = idesc_tf32(128, 128, false, false);
+    constexpr uint32_t kIdN128Bmn = idesc_tf32(128, 128, false, true);  // B (Kt, V) MN-major
 
-    const TIn* __restrict__ vg = static_cast<const TIn*>(a.v);
     for (int k = 0; k < n_mine; ++k) {
       const int64_t it = blockIdx.x + static_cast<int64_t>(k) * gridDim.x;
       const ItemPos ip = item_pos(it, a, p);
@@ -754,78 +816,17 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       tc_fence_before_sync();
       bsync();
 
-      // -- V^T (tf32; conv for the mixer): each thread takes 4-token x 4-column blocks, all
-      //    of whose rows are loaded before any is used (the rows were warmed into L2) ----------
-      {
-        constexpr int kW = sizeof(TIn);  // 32-bit words per 4 elements
-        const TIn* vh = vg + static_cast<size_t>(ip.h) * kD;
-        uint32_t vraw[2][kGRows][kW];
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
-#pragma unroll
-          for (int m = 0; m < kGRows; ++m) {
-            const int rr = t4 - kHist + m;
-            const bool in = rr < ip.len && ip.t0 + rr >= ip.bos;
-            const TIn* src = vh + static_cast<size_t>(in ? ip.t0 + rr : ip.t0) * tok_stride + j4;
-            if constexpr (kW == 2) {
-              const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
-              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
-            } else {
-              const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
-              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
-              vraw[bb][m][2] = in ? x.z : 0u; vraw[bb][m][3] = in ? x.w : 0u;
-            }
-          }
-        }
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const int jr = (jj + lane) & 3;  // lanes rotate the column so a store spreads over swizzle rows
-            auto elem = [&](int m) -> float {  // selects, not indexing: the array stays in registers
-              if constexpr (kW == 2) {
-                const uint32_t x = (jr >> 1) ? vraw[bb][m][1] : vraw[bb][m][0];
-                return __uint_as_float((jr & 1) ? (x & 0xFFFF0000u) : (x << 16));
-              } else {
-                const uint32_t lo = (jr & 1) ? vraw[bb][m][1] : vraw[bb][m][0];
-                const uint32_t hi = (jr & 1) ? vraw[bb][m][3] : vraw[bb][m][2];
-                return __uint_as_float((jr >> 1) ? hi : lo);
-              }
-            };
-            float x[4];
-            if constexpr (kConv) {
-              const float4 w4 =
-                  __ldg(reinterpret_cast<const float4*>(a.conv_w + ((2 * H + ip.h) * kD + j4 + jr) * 4));
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float y = fmaf(w4.x, elem(e), fmaf(w4.y, elem(e + 1), fmaf(w4.z, elem(e + 2), w4.w * elem(e + 3))));
-                x[e] = (t4 + e < ip.len) ? y : 0.f;
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) x[e] = elem(e);
-            }
-            st4_tf32(sm + SM::kVT, f32_offset(j4 + jr, t4, 128), x[0], x[1], x[2], x[3]);
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      bsync();
-
-      // -- D[W; -] = T Kt, D[U~; -] = T V, once the front group has written Kt^T ------------
+      // -- D[W; -] = T Kt, D[U~; -] = T V, once the front group has written Kt and V ---------
       if (btid == 0) {
         if (!lost && !mbar_wait(bars + kBVtFull, ph_vtfull, a.status)) lost = true;
         ph_vtfull ^= 1u;
         tc_fence_after_sync();
-        const uint64_t kt0 = kdesc0(sb + SM::kKTT), v0 = kdesc0(sb + SM::kVT);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_tf32_ta(tmem + kTmW, tmem + kTmT + kk * 8, kt0 + kstep(kk, 128), kIdN128, kk > 0);
+          umma_tf32_ta(tmem + kTmW, tmem + kTmT + kk * 8, mndesc(sb + SM::kKTT, 64, kk), kIdN128Bmn, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_tf32_ta(tmem + kTmU, tmem + kTmT + kk * 8, v0 + kstep(kk, 128), kIdN128, kk > 0);
+          umma_tf32_ta(tmem + kTmU, tmem + kTmT + kk * 8, mndesc(sb + SM::kVT, 64, kk), kIdN128Bmn, kk > 0);
         umma_commit(bars + kBWuDone);
       }
       if (btid == 0 && !lost && !mbar_wait(bars + kBWuDone, ph_wu, a.status)) lost = true;
@@ -1102,7 +1103,9 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
   __syncthreads();
   tc_fence_after_sync();
 
+  // B (S^T, U^T) is K-major; A is [-W; Qt] and P (K-major) or Kh^T (MN-major: Kh's rows)
   constexpr uint32_t kIdV = idesc_tf32(128, DV, false, false);
+  constexpr uint32_t kIdVmn = idesc_tf32(128, DV, true, false);
   bool lost = false, failed = false;
   // completions seen per barrier (each thread counts those it waits for)
   uint32_t g1_phase = 0, g2_phase = 0, o_phase = 0;
@@ -1212,10 +1215,10 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
       if (issuer) {
         wait_loads(bar_pk, pk_waited);
         tc_fence_after_sync();
-        const uint64_t ka = kdesc0(sb + SM::kKHT), ub = kdesc0(sb + SM::kUT);
-        const uint64_t pa = kdesc0(sb + SM::kPT + (i & 1) * 32768);
+        const uint64_t pa = kdesc0(sb + SM::kPT + (i & 1) * 32768), ub = kdesc0(sb + SM::kUT);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) umma_tf32(tmem + kD2, ka + kstep(kk, 128), ub + kstep(kk, DV), kIdV, 1u);
+        for (int kk = 0; kk < 8; ++kk)
+          umma_tf32(tmem + kD2, mndesc(sb + SM::kKHT, kChunk, kk), ub + kstep(kk, DV), kIdVmn, 1u);
         umma_commit(bar_g2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) umma_tf32(d1, pa + kstep(kk, 128), ub + kstep(kk, DV), kIdV, 1u);
@@ -1241,6 +1244,7 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
           float ws[8];
           tmem_ld8(d1 + lane_off + cc, ws);
           tmem_ld_wait();
+          // U row `row` as a line of the MN-major B operand of group 2
 #pragma unroll
           for (int e = 0; e < 8; ++e) st_tf32(sm + SM::kUT, f32_offset(cc + e, row, DV), ut[j + e] + ws[e]);
         }
@@ -1261,10 +1265,9 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
         tmem_ld8(tmem + lane_off + kD2 + cc, x);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x[e] *= gm;
-          *reinterpret_cast<float*>(sm + SM::kST + f32_offset(cc + e, row, DV)) = x[e];
-        }
+        for (int e = 0; e < 8; ++e) x[e] *= gm;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) *reinterpret_cast<float*>(sm + SM::kST + f32_offset(cc + e, row, DV)) = x[e];
         tmem_st8(tmem + lane_off + kD2 + cc, x);
       }
       tmem_st_wait();

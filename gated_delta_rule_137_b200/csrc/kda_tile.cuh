@@ -42,6 +42,27 @@ __host__ __device__ constexpr uint64_t kstep(int kk, uint32_t rows) {
 // from it moves by less than 1e-6 nats per token).
 __device__ __forceinline__ float softplus_fast(float x) { return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x))); }
 
+// MN-major fp32 operand tile of `krows` K lines (mn_offset): descriptor of K step kk
+// (8 lines, 1024 B, per tf32 instruction).
+__device__ __forceinline__ uint64_t mndesc(uint32_t base, uint32_t krows, int kk) {
+  return sdesc(base + static_cast<uint32_t>(kk) * 1024u, krows * 128u, 512u, kSwz128A32);
+}
+
+// Eight consecutive elements (mn .. mn + 7, mn a multiple of 8) of line k of an MN-major
+// tile, as two 16-byte stores (tf32-rounded if `tf32`). When the 32 lanes of a warp write
+// 32 consecutive lines at the same mn, rows with bit 2 set store their upper half first,
+// so that each quarter-warp's 16-byte stores land on 8 different bank groups.
+__device__ __forceinline__ void st8_line(uint8_t* tile, uint32_t k, uint32_t mn, uint32_t krows, const float (&x)[8],
+                                         bool tf32) {
+  const bool swap = (k >> 2) & 1u;
+  float y[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) y[e] = tf32 ? to_tf32(x[e]) : x[e];
+  const float4 lo = make_float4(y[0], y[1], y[2], y[3]), hi = make_float4(y[4], y[5], y[6], y[7]);
+  *reinterpret_cast<float4*>(tile + mn_offset(k, mn + (swap ? 4u : 0u), krows)) = swap ? hi : lo;
+  *reinterpret_cast<float4*>(tile + mn_offset(k, mn + (swap ? 0u : 4u), krows)) = swap ? lo : hi;
+}
+
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // read-only loads of an input element as fp32

@@ -282,13 +282,14 @@ __device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint
 // descriptors
 // ---------------------------------------------------------------------------------
 // Swizzle modes of the shared-memory matrix descriptor (bits 61..63).
-constexpr uint32_t kSwzNone = 0, kSwz128 = 2, kSwz64 = 4, kSwz32 = 6;
+// kSwz128A32: 128B swizzle with 32-byte atoms, the layout an MN-major tf32 operand takes.
+constexpr uint32_t kSwzNone = 0, kSwz128A32 = 1, kSwz128 = 2, kSwz64 = 4, kSwz32 = 6;
 
 // Shared-memory matrix descriptor. Byte offsets; the operand tile must start on
 // the swizzle atom's alignment (1024 B for 128B swizzle, 512 B for 64B).
 //   K-major swizzled:  SBO = stride between 8-row groups, LBO unused (1).
-//   MN-major swizzled: LBO = stride between swizzle atoms along M/N,
-//                      SBO = stride between 8-row groups along K.
+//   MN-major (kSwz128A32): LBO = stride between 32-element blocks along M/N,
+//                      SBO = stride between 4-row groups along K (512 B).
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint32_t swz) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
@@ -335,6 +336,15 @@ __device__ __forceinline__ float to_tf32(float x) {
 // the bytes are the same.
 __device__ __forceinline__ uint32_t f32_offset(uint32_t row, uint32_t col, uint32_t rows) {
   return (col >> 5) * rows * 128u + row * 128u + ((((col & 31u) >> 2) ^ (row & 7u)) << 4) + (col & 3u) * 4u;
+}
+
+// Byte offset of fp32 element (k, mn) of an MN-major tf32 operand tile: one 128-B line
+// per K index holding 32 consecutive M/N elements, the 32-byte quarters of a line
+// swizzled with (k mod 4), 32-element M/N blocks `krows` lines apart. Rows of a matrix
+// whose columns are M/N (V as the B operand of T V, Kt of T Kt, S of [-W; Qt] S) are
+// written here as whole lines, with no transpose.
+__device__ __forceinline__ uint32_t mn_offset(uint32_t k, uint32_t mn, uint32_t krows) {
+  return (mn >> 5) * krows * 128u + k * 128u + ((((mn & 31u) >> 3) ^ (k & 3u)) << 5) + (mn & 7u) * 4u;
 }
 
 // Byte offset of element (row, col) of a K-major tile stored with 128-byte

@@ -93,9 +93,10 @@ def _tok(x):
     return np.ascontiguousarray(np.swapaxes(x, 0, 1))
 
 
-def test_mixer_decode_tokens_without_checkpoints_matches_k_steps(kda):
+@pytest.mark.parametrize("K", [2, 3, 4, 6])  # 2..4: the one-pass block form; 6: token by token
+def test_mixer_decode_tokens_without_checkpoints_matches_k_steps(kda, K):
     import torch
-    w = I.make_mixer_decode(10, 4, 128, 4, 16, seed=I.SEED_BASE + 43)
+    w = I.make_mixer_decode(10, 4, 128, K, 16, seed=I.SEED_BASE + 43 + K)
     sp, cp = to_device(w.state_pool, "f32"), to_device(w.conv_pool, "bf16")
     out = kda.mixer_decode_tokens(to_device(_tok(w.q), "bf16"), to_device(_tok(w.k), "bf16"),
                                   to_device(_tok(w.v), "bf16"), to_device(w.conv_w, "f32"),
@@ -110,10 +111,11 @@ def test_mixer_decode_tokens_without_checkpoints_matches_k_steps(kda):
     np.testing.assert_array_equal(cp.view(torch.int16).cpu().numpy().view(np.uint16)[idx], I.bf16_bits(rh[:, -1]))
 
 
-def test_mixer_decode_tokens_checkpoints_and_commit(kda):
+@pytest.mark.parametrize("K", [3, 4, 5])
+def test_mixer_decode_tokens_checkpoints_and_commit(kda, K):
     import torch
-    w = I.make_mixer_decode(6, 2, 128, 4, 9, seed=I.SEED_BASE + 44)
-    N, K, H = 6, 4, 2
+    w = I.make_mixer_decode(6, 2, 128, K, 9, seed=I.SEED_BASE + 44 + K)
+    N, H = 6, 2
     sp, cp = to_device(w.state_pool, "f32"), to_device(w.conv_pool, "bf16")
     idx = to_device(w.indices, "i32")
     sck = torch.full((N, K, H, 128, 128), float("nan"), device="cuda")
@@ -135,7 +137,7 @@ def test_mixer_decode_tokens_checkpoints_and_commit(kda):
     ck_bits = cck.view(torch.int16).cpu().numpy().view(np.uint16)
     np.testing.assert_array_equal(ck_bits, I.bf16_bits(rh))
     # commit: sequence n keeps accepted[n] tokens
-    accepted = np.array([0, 1, 4, 2, 3, 1], dtype=np.int32)
+    accepted = np.array([0, 1, K, 2, 3, 1], dtype=np.int32)
     kda.mixer_decode_commit(sck, cck, to_device(accepted, "i32"), sp, cp, idx, status=status)
     torch.cuda.synchronize()
     assert int(to_host(status)[0]) == 0
