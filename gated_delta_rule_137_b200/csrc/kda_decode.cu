@@ -338,8 +338,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2) mixer_decode_kernel(cons
   }
 }
 
-// K = 2..4 tokens of one (sequence, head) with a single pass over the state (512 threads:
-// 16 warps of 8 state rows, so that the 2K column sums fit in registers): the K-token
+// K = 2..4 tokens of one (sequence, head) with a single pass over the state (256 threads,
+// 8 warps of 16 state rows, two CTAs per SM): the K-token
 // block of the recurrence in the WY form the chunked prefill uses (chunk size K), with
 // every product on the CUDA cores. Per key channel r, with tokens j = 0..K-1,
 //   c_j = alpha_0 ... alpha_j,   D(i, j) = alpha_{i+1} ... alpha_j   (D(j, j) = 1),
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 2) mixer_decode_kernel(cons
 // terms come from the token vectors alone, so the tokens' dependency runs through
 // K x 4 numbers per thread instead of the state. The conv, L2 norm and gate are those of
 // mixer_decode_kernel; the state after every token is written only with checkpoints.
-constexpr int kBlockWarps = 16;  // 512 threads, 8 state rows per warp
+constexpr int kBlockWarps = 8;  // 256 threads, 16 state rows per warp, two CTAs per SM
 constexpr int kBlockRows = kMixD / kBlockWarps;
 template <int KB>
 struct BlockSmem {
@@ -379,7 +379,7 @@ template <int KB>
 __host__ __device__ constexpr int q_index(int j, int i) { return i * KB + j; }
 
 template <int KB>
-__global__ void __launch_bounds__(kBlockWarps * 32, 1) mixer_decode_block_kernel(const MixerDecodeArgs a) {
+__global__ void __launch_bounds__(kBlockWarps * 32, 2) mixer_decode_block_kernel(const MixerDecodeArgs a) {
   using SM = BlockSmem<KB>;
   extern __shared__ __align__(16) uint8_t block_smem_raw[];
   SM& sm = *reinterpret_cast<SM*>(block_smem_raw);
@@ -491,22 +491,26 @@ __global__ void __launch_bounds__(kBlockWarps * 32, 1) mixer_decode_block_kernel
     sm.pairT[threadIdx.x] = sm.pair[threadIdx.x][0] + sm.pair[threadIdx.x][1] + sm.pair[threadIdx.x][2] +
                             sm.pair[threadIdx.x][3];
 
-  // ---- one pass over S_0: the 2K column sums --------------------------------------------
-  float4 acc[2 * KB];
+  // ---- one pass over S_0 (held in registers): the 2K column sums, K at a time so that
+  //      the accumulators fit beside the state -----------------------------------------
 #pragma unroll
-  for (int v = 0; v < 2 * KB; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int half = 0; half < 2; ++half) {
+    float4 acc[KB];
 #pragma unroll
-  for (int r = 0; r < kBlockRows; ++r) {
-    const float* cr = sm.c1[warp * kBlockRows + r];
+    for (int v = 0; v < KB; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int v = 0; v < 2 * KB; ++v) {
-      const float w = cr[v];
-      acc[v].x = fmaf(w, s[r].x, acc[v].x); acc[v].y = fmaf(w, s[r].y, acc[v].y);
-      acc[v].z = fmaf(w, s[r].z, acc[v].z); acc[v].w = fmaf(w, s[r].w, acc[v].w);
+    for (int r = 0; r < kBlockRows; ++r) {
+      const float* cr = sm.c1[warp * kBlockRows + r] + half * KB;
+#pragma unroll
+      for (int v = 0; v < KB; ++v) {
+        const float w = cr[v];
+        acc[v].x = fmaf(w, s[r].x, acc[v].x); acc[v].y = fmaf(w, s[r].y, acc[v].y);
+        acc[v].z = fmaf(w, s[r].z, acc[v].z); acc[v].w = fmaf(w, s[r].w, acc[v].w);
+      }
     }
-  }
 #pragma unroll
-  for (int v = 0; v < 2 * KB; ++v) sm.red[v][warp][lane] = acc[v];
+    for (int v = 0; v < KB; ++v) sm.red[half * KB + v][warp][lane] = acc[v];
+  }
   __syncthreads();
   for (int v = warp; v < 2 * KB; v += kBlockWarps) {
     float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
