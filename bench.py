@@ -791,6 +791,40 @@ def run_profile_case(args):
                       "bytes_per_call": prefill_bytes(n * T, n)}), flush=True)
 
 
+def run_profile_tokens(args):
+    """The serving decode with K = 4 draft tokens per call (N = 256 sequences x 32 heads,
+    no checkpoints, the block form), W + K calls, then one line with the CUDA-event time
+    per call; for kernel captures."""
+    import torch
+    import gated_delta_rule_137_b200 as kda
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(device)
+    kda.load_library()
+    Nd, Kt = 256, 4
+    g = torch.Generator(device=device).manual_seed(1370005)
+    sp = 0.02 * torch.randn(Nd, H, D, D, generator=g, device=device)
+    cp = torch.randn(Nd, H, 3, 3, D, generator=g, device=device).bfloat16()
+    idx = torch.randperm(Nd, generator=g, device=device).to(torch.int32)
+    cw = (0.5 * torch.randn(3, H * D, 4, generator=g, device=device)).contiguous()
+    t = dict(q=torch.randn(Nd, Kt, H, D, generator=g, device=device).bfloat16(),
+             k=torch.randn(Nd, Kt, H, D, generator=g, device=device).bfloat16(),
+             v=torch.randn(Nd, Kt, H, D, generator=g, device=device).bfloat16(),
+             g=torch.randn(Nd, Kt, H, D, generator=g, device=device).bfloat16(),
+             la=(-torch.nn.functional.softplus(torch.randn(Nd, Kt, H, D, generator=g, device=device)) / 16).contiguous(),
+             b=torch.sigmoid(torch.randn(Nd, Kt, H, generator=g, device=device)).contiguous())
+    out = torch.empty(Nd, Kt, H, D, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def call(i):
+        kda.mixer_decode_tokens(t["q"], t["k"], t["v"], cw, t["la"], t["b"], t["g"], sp, cp, idx, out=out,
+                                stream=stream)
+
+    per, tot = time_region(call, args.steps, args.warmup, stream, device)
+    print(json.dumps({"case": f"serving decode, {Kt} tokens per call, N={Nd} H={H} d={D}",
+                      "us_per_call": tot / args.steps * 1e3,
+                      "bytes_per_call": mixer_decode_tokens_bytes(Nd, Kt)}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -802,6 +836,8 @@ def main(argv=None):
     ap.add_argument("--cpu-heads", type=int, default=32)
     ap.add_argument("--profile-case", action="store_true",
                     help="only a mid-size single-pass prefill (8 x 4096 tokens, 32 heads), for kernel captures")
+    ap.add_argument("--profile-tokens", action="store_true",
+                    help="only the 4-token serving decode (256 sequences, 32 heads), for kernel captures")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per headline call to report instead of profiles/traffic.json")
     args = ap.parse_args(argv)
@@ -811,6 +847,8 @@ def main(argv=None):
         run_reference(args)
     elif args.profile_case:
         run_profile_case(args)
+    elif args.profile_tokens:
+        run_profile_tokens(args)
     else:
         run_gpu(args)
 
