@@ -194,10 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t tok_stride = static_cast<int64_t>(H) * kD;  // elements between tokens
 
   constexpr uint32_t kIdAP = idesc_tf32(128, 64, false, false);
-  // the B operands Kt, V, S and U are MN-major, and so is Kh^T as the A of Kh^T U
   constexpr uint32_t kIdW = idesc_tf32(128, 128, false, true);
-  constexpr uint32_t kIdV = idesc_tf32(128, DV, false, true);
-  constexpr uint32_t kIdVmn = idesc_tf32(128, DV, true, true);
+  constexpr uint32_t kIdVb = idesc_tf32(128, DV, false, true);   // B = V (MN-major)
+  constexpr uint32_t kIdV = idesc_tf32(128, DV, false, false);   // B = S^T, U^T (K-major)
+  constexpr uint32_t kIdVmn = idesc_tf32(128, DV, true, false);  // A = Kh^T (MN-major)
 
   uint32_t mma_phase = 0, tma_phase = 0;
   bool failed = false;
@@ -533,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_tf32(tmem + TM::kD0, a0 + kstep(kk, 128), mndesc(sb + SM::kKTT, kChunk, kk), kIdW, kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_tf32(tmem + TM::kD3, a0 + kstep(kk, 128), mndesc(sb + SM::kVT, kChunk, kk), kIdV, kk > 0);
+        umma_tf32(tmem + TM::kD3, a0 + kstep(kk, 128), mndesc(sb + SM::kVT, kChunk, kk), kIdVb, kk > 0);
       umma_commit(bar_mma);
     }
     wait_mma();
@@ -562,7 +562,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] *= gm;
-        st8_line(sm + SM::kST, row, c, kD, x, false);  // row `row` of the MN-major S operand
+#pragma unroll
+        for (int e = 0; e < 8; ++e) *reinterpret_cast<float*>(sm + SM::kST + f32_offset(c + e, row, DV)) = x[e];
         tmem_st8(tmem + lane_off + TM::kD2 + c, x);
       }
       tmem_st_wait();
@@ -577,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t a0 = kdesc0(sb + SM::kKQ);
 #pragma unroll
       for (int kk = 0; kk < 16; ++kk)
-        umma_tf32(tmem + TM::kD1, a0 + kstep(kk, 128), mndesc(sb + SM::kST, kD, kk), kIdV, kk > 0);
+        umma_tf32(tmem + TM::kD1, a0 + kstep(kk, 128), kdesc0(sb + SM::kST) + kstep(kk, DV), kIdV, kk > 0);
       umma_commit(bar_mma);
     }
     if (t0 + kChunk < eos) {  // next chunk's gate inputs, in flight during the MMAs
@@ -595,10 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld8(tmem + lane_off + TM::kD3 + c, ut);
         tmem_ld8(tmem + lane_off + TM::kD1 + c, ws);
         tmem_ld_wait();
-        float u[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) u[e] = ut[e] + ws[e];
-        st8_line(sm + SM::kVT, row, c, kChunk, u, true);  // row `row` of the MN-major U operand
+        for (int e = 0; e < 8; ++e) st_tf32(sm + SM::kVT, f32_offset(c + e, row, DV), ut[e] + ws[e]);
       }
     }
     fence_proxy_async_smem();
@@ -611,10 +610,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t t0d = kdesc0(sb + SM::kTP);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_tf32(tmem + TM::kD2, mndesc(sb + SM::kKHT, kChunk, kk), mndesc(sb + SM::kVT, kChunk, kk), kIdVmn, 1u);
+        umma_tf32(tmem + TM::kD2, mndesc(sb + SM::kKHT, kChunk, kk), kdesc0(sb + SM::kVT) + kstep(kk, DV), kIdVmn, 1u);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        umma_tf32(tmem + TM::kD1, t0d + kstep(kk, 128), mndesc(sb + SM::kVT, kChunk, kk), kIdV, 1u);
+        umma_tf32(tmem + TM::kD1, t0d + kstep(kk, 128), kdesc0(sb + SM::kVT) + kstep(kk, DV), kIdV, 1u);
       umma_commit(bar_mma);
     }
     wait_mma();

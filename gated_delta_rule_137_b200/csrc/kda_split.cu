@@ -319,6 +319,9 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
   using SM = IntraSmem;
   constexpr int kHist = kConv ? 3 : 0;    // tokens of history the conv needs
   constexpr int kGRows = 4 + kHist;       // q/k rows a thread loads per 4-token group
+  // which group builds the V rows: the front one, except for the mixer, whose gate pass
+  // (conv and L2 norm of q and k) already makes the front group the longer one
+  constexpr bool kVFront = !kConv;
 
   const int H = a.H;
   const int total_chunks = __ldg(p.chunk_start + a.N);
@@ -672,7 +675,7 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       }
       // V rows (tf32; conv for the mixer) as the MN-major B operand of T V: each thread takes
       // 4-token x 4-column blocks (their rows loaded above)
-      if (!strong) {
+      if (kVFront && !strong) {
         if constexpr (!kEarlyV) load_v();
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
@@ -814,6 +817,70 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         tmem_st_wait();
       }
       tc_fence_before_sync();
+      bsync();
+
+      // -- the V rows with their conv (the mixer) as lines of the MN-major B operand of T V:
+      //    each thread takes 4-token x 4-column blocks, all of whose rows are loaded before
+      //    any is used (the rows were warmed into L2) ------------------------------------------
+      if constexpr (!kVFront) {
+        constexpr int kW = sizeof(TIn);  // 32-bit words per 4 elements
+        const TIn* vh = static_cast<const TIn*>(a.v) + static_cast<size_t>(ip.h) * kD;
+        uint32_t vraw[2][kGRows][kW];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+#pragma unroll
+          for (int m = 0; m < kGRows; ++m) {
+            const int rr = t4 - kHist + m;
+            const bool in = rr < ip.len && ip.t0 + rr >= ip.bos;
+            const TIn* src = vh + static_cast<size_t>(in ? ip.t0 + rr : ip.t0) * tok_stride + j4;
+            if constexpr (kW == 2) {
+              const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
+              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
+            } else {
+              const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
+              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
+              vraw[bb][m][2] = in ? x.z : 0u; vraw[bb][m][3] = in ? x.w : 0u;
+            }
+          }
+        }
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+          auto elem = [&](int jr, int m) -> float {  // column j4 + jr of loaded row m
+            if constexpr (kW == 2) {
+              const uint32_t x = vraw[bb][m][jr >> 1];
+              return __uint_as_float((jr & 1) ? (x & 0xFFFF0000u) : (x << 16));
+            } else {
+              return __uint_as_float(vraw[bb][m][jr]);
+            }
+          };
+          float4 wv[kConv ? 4 : 1];  // conv taps of columns j4 .. j4 + 3
+          if constexpr (kConv) {
+#pragma unroll
+            for (int jr = 0; jr < 4; ++jr)
+              wv[jr] = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((2 * H + ip.h) * kD + j4 + jr) * 4));
+          }
+          // V rows t4 .. t4 + 3 as whole lines of the MN-major B operand of T V
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float y[4];
+#pragma unroll
+            for (int jr = 0; jr < 4; ++jr) {
+              if constexpr (kConv) {
+                const float4 w4 = wv[jr];
+                const float yc = fmaf(w4.x, elem(jr, e), fmaf(w4.y, elem(jr, e + 1),
+                                                              fmaf(w4.z, elem(jr, e + 2), w4.w * elem(jr, e + 3))));
+                y[jr] = (t4 + e < ip.len) ? yc : 0.f;
+              } else {
+                y[jr] = elem(jr, e);
+              }
+            }
+            st4_tf32(sm + SM::kVT, mn_offset(t4 + e, j4, 64), y[0], y[1], y[2], y[3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
       bsync();
 
       // -- D[W; -] = T Kt, D[U~; -] = T V, once the front group has written Kt and V ---------
