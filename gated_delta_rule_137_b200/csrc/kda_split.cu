@@ -800,6 +800,30 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       if (btid == 0) mbar_arrive(bars + kBApFree);
 
       // -- X = (I + A)^-1; T = X Diag(beta) into TMEM rows 0..63 (the W / U~ MMA's A) ---------
+      // the mixer's V rows (with the conv's history rows) in flight during the inverse
+      constexpr int kWb = sizeof(TIn);  // 32-bit words per 4 elements
+      uint32_t vraw[2][kGRows][kWb];
+      if constexpr (!kVFront) {
+        const TIn* vh = static_cast<const TIn*>(a.v) + static_cast<size_t>(ip.h) * kD;
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+#pragma unroll
+          for (int m = 0; m < kGRows; ++m) {
+            const int rr = t4 - kHist + m;
+            const bool in = rr < ip.len && ip.t0 + rr >= ip.bos;
+            const TIn* src = vh + static_cast<size_t>(in ? ip.t0 + rr : ip.t0) * tok_stride + j4;
+            if constexpr (kWb == 2) {
+              const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
+              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
+            } else {
+              const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
+              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
+              vraw[bb][m][2] = in ? x.z : 0u; vraw[bb][m][3] = in ? x.w : 0u;
+            }
+          }
+        }
+      }
       invert_unit_lower_64(sA, sY, bw, bsync);
       if (lq < 2) {
         const int r = row;
@@ -823,32 +847,11 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       //    each thread takes 4-token x 4-column blocks, all of whose rows are loaded before
       //    any is used (the rows were warmed into L2) ------------------------------------------
       if constexpr (!kVFront) {
-        constexpr int kW = sizeof(TIn);  // 32-bit words per 4 elements
-        const TIn* vh = static_cast<const TIn*>(a.v) + static_cast<size_t>(ip.h) * kD;
-        uint32_t vraw[2][kGRows][kW];
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
-#pragma unroll
-          for (int m = 0; m < kGRows; ++m) {
-            const int rr = t4 - kHist + m;
-            const bool in = rr < ip.len && ip.t0 + rr >= ip.bos;
-            const TIn* src = vh + static_cast<size_t>(in ? ip.t0 + rr : ip.t0) * tok_stride + j4;
-            if constexpr (kW == 2) {
-              const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
-              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
-            } else {
-              const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
-              vraw[bb][m][0] = in ? x.x : 0u; vraw[bb][m][1] = in ? x.y : 0u;
-              vraw[bb][m][2] = in ? x.z : 0u; vraw[bb][m][3] = in ? x.w : 0u;
-            }
-          }
-        }
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
           const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
           auto elem = [&](int jr, int m) -> float {  // column j4 + jr of loaded row m
-            if constexpr (kW == 2) {
+            if constexpr (kWb == 2) {
               const uint32_t x = vraw[bb][m][jr >> 1];
               return __uint_as_float((jr & 1) ? (x & 0xFFFF0000u) : (x << 16));
             } else {

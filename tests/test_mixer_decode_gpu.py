@@ -176,8 +176,9 @@ def test_mixer_decode_one_token_call_is_the_decode_step(kda):
     np.testing.assert_array_equal(outs[0][1], outs[1][1])
 
 
-@pytest.mark.parametrize("lens,H", [([130, 2, 64, 0], 4),   # 16 chains: the two-pass prefill
-                                    ([70] * 19 + [1], 4)])  # 80 chains: the single-pass prefill
+@pytest.mark.parametrize("lens,H", [([130, 2, 64, 0], 4),        # 16 chains: the two-pass prefill
+                                    ([70] * 19 + [1], 4),       # 80 chains: the single-pass prefill
+                                    ([0] + [66] * 18 + [3], 4)])  # single-pass, an empty prompt first
 def test_pooled_prefill_hands_over_to_the_decode_step(kda, lens, H):
     """kda_mixer_fwd_pooled over each sequence's first T tokens into permuted slots of
     larger pools, then kda_mixer_decode_step on token T + 1, against oracle.kda_mixer over
@@ -269,3 +270,29 @@ def test_pooled_prefill_flags_a_slot_outside_the_pool(kda):
     assert_prefill_close(to_host(sp)[1], rf[1], "state of the valid slot")
     np.testing.assert_array_equal(to_host(sp)[[0, 2]], 0.0)
     np.testing.assert_array_equal(to_host(cp)[[0, 2]], 0.0)
+
+
+def test_pooled_prefill_of_empty_prompts_starts_the_slots(kda):
+    """total_T = 0: nothing to prefill; each named slot gets the sequence's initial state (or
+    zero) and an all-zero conv history, the other slots are untouched."""
+    import torch
+    N, H, d, pool = 3, 2, 128, 5
+    rng = np.random.default_rng(I.SEED_BASE + 46)
+    sp0 = rng.standard_normal((pool, H, d, d)).astype(np.float32)
+    cp0 = I.bf16_round(rng.standard_normal((pool, H, 3, 3, d)).astype(np.float32))
+    s0 = (0.02 * rng.standard_normal((N, H, d, d))).astype(np.float32)
+    slots = np.array([4, 0, 2], dtype=np.int32)
+    empty = lambda dt: to_device(np.zeros((0, H, d), np.float32), dt)
+    for init in (s0, None):
+        sp, cp = to_device(sp0, "f32"), to_device(cp0, "bf16")
+        kda.mixer_fwd_pooled(empty("bf16"), empty("bf16"), empty("bf16"), to_device(np.ones((3, H * d, 4), np.float32), "f32"),
+                             empty("f32"), to_device(np.zeros((0, H), np.float32), "f32"), None, sp, cp,
+                             to_device(slots, "i32"), None if init is None else to_device(init, "f32"),
+                             to_device(np.zeros(N + 1, np.int32), "i32"), N=N, check_status=True)
+        torch.cuda.synchronize()
+        got_s, got_h = to_host(sp), to_host(cp)
+        want = np.zeros((N, H, d, d), np.float32) if init is None else init
+        np.testing.assert_array_equal(got_s[slots], want)
+        np.testing.assert_array_equal(got_h[slots], 0.0)
+        np.testing.assert_array_equal(got_s[[1, 3]], sp0[[1, 3]])
+        np.testing.assert_array_equal(got_h[[1, 3]], to_host(to_device(cp0, "bf16"))[[1, 3]])
