@@ -12,10 +12,11 @@
 //   U  = U~ - W S,   O = Qt S + P U,   S' = Diag(e^g_last) (S + Kh^T U)
 // (the last line folds the usual K*e^(g_last-g) factor into Kh and a row scale).
 //
-// Mapping onto one CTA of 128 threads (thread i <-> TMEM lane i):
-//   * the CTA owns one (sequence, head) chain and a slice of DV value columns;
-//     the fp32 state slice S [128 x DV] lives in registers (thread c = key row c)
-//     and is copied to shared memory as an MMA operand once per chunk;
+// Mapping onto one CTA of 512 threads (warp w reads TMEM lanes 32 (w % 4) .. and value
+// column part w / 4):
+//   * the CTA owns one (sequence, head) chain and a slice of DV value columns; the fp32
+//     state slice S [128 x DV] lives in TMEM (lane c = key row c) and is copied to
+//     shared memory as an MMA operand once per chunk;
 //   * every GEMM is tcgen05.mma kind::tf32 (fp32 operands in shared memory read
 //     with a 10-bit mantissa, fp32 accumulate in TMEM), M = 128, with 64-row
 //     operands stacked in pairs:
@@ -25,16 +26,17 @@
 //       [-W; Qt] S        -> D1 = [-W S; Qt S]       (M128 NDV  K128)
 //       Kh^T U            -> D2                      (M128 NDV  K64)
 //       [T; P] U  (+= D1) -> D1 = [-; Qt S + P U]    (M128 NDV  K64)
-//     ("-" rows are by-products that are never read). Every operand is stored
-//     K-major (the K index contiguous within 128-byte swizzled rows), so Kt and Kh
-//     are written twice, token-major and channel-major, and V, S, U transposed.
-//     bf16 operands would cost about 2% of RMS in the worst output element on top
-//     of the bf16 store; tf32 keeps the operand error well below the store's own
-//     rounding;
+//     ("-" rows are by-products that are never read). Kt, Kh and V are written once
+//     more as whole lines of MN-major tiles (128B swizzle with 32-byte atoms), the B
+//     operands Kt and V and the A operand Kh^T, so nothing is transposed on the CUDA
+//     cores for them; S^T and U^T are written K-major by the epilogues (MN-major lines
+//     measured slower there). bf16 operands would cost about 2% of RMS in the worst
+//     output element on top of the bf16 store; tf32 keeps the operand error well below
+//     the store's own rounding;
 //   * the 64x64 unit-lower-triangular inverse is done in fp32 on CUDA cores:
 //     16x16 diagonal blocks by substitution, then two levels of block doubling
 //     X21 = -X22 (A21 X11);
-//   * V arrives by TMA (no multicast) and is widened/transposed to fp32 in shared
+//   * V arrives by TMA (no multicast) and is widened to fp32 operand lines in shared
 //     memory; q, k, log_alpha, beta are read with coalesced read-only loads by the
 //     thread that owns each key channel.
 // Decay range: the factorised products need e^{-g} finite, so a chunk whose decay summed
@@ -53,14 +55,14 @@ namespace kda {
 namespace {
 
 constexpr int kThreads = 512;  // 16 warps; warp w reads TMEM lanes 32*(w%4).. and column part w/4
-// ---- shared memory plan (bytes from a 1024-aligned base); fp32 K-major tiles -------
+// ---- shared memory plan (bytes from a 1024-aligned base); fp32 operand tiles ------
 //  region   size        holds (in chunk order)
 //  KQ       64 KB       [Kt; Qt] (128 tok-rows x 128 ch)  ->  [-W; Qt]
 //  KH       32 KB       Kh (64 tok-rows x 128 ch)  ->  solve scratch  ->  S^T (with KTT)
-//  KTT      32 KB       Kt^T (128 ch-rows x 64 tok)  ->  S^T (second half)
-//  KHT      32 KB       Kh^T (128 ch-rows x 64 tok)
+//  KTT      32 KB       Kt as MN-major lines (64 tok x 128 ch)  ->  S^T (second half)
+//  KHT      32 KB       Kh as MN-major lines (64 tok x 128 ch)
 //  TP       32 KB       bf16 V from TMA  ->  [T; P] (128 rows x 64 tok)
-//  VT       DV*256 B    V^T (DV rows x 64 tok)  ->  U^T
+//  VT       DV*256 B    V as MN-major lines (64 tok x DV)  ->  U^T
 template <int DV>
 struct Smem {
   static constexpr int kKQ = 0;
@@ -402,11 +404,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }  // factorised form
     }
 
-    // -- 3. V landed: widen/transpose to V^T fp32 (rows past the sequence end -> 0) -------
+    // -- 3. V landed: widen to fp32 operand lines (rows past the sequence end -> 0) --------
     {
       if (!lost && !mbar_wait(bar_tma, tma_phase, a.status)) lost = true;
       tma_phase ^= 1u;
-      __syncthreads();  // every thread is done with the decay totals (they share V^T's space)
+      __syncthreads();  // every thread is done with the decay totals (they share V's space)
       const TIn* st = reinterpret_cast<const TIn*>(sm + SM::kStage);  // row m = token t0 - kHist + m
       for (int i = tid; i < DV * 16; i += kThreads) {
         const int j = i % DV, t4 = (i / DV) * 4;
@@ -587,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     wait_mma();
 
-    // -- 10. U = U~ - W S -> U^T operand (over V^T) ---------------------------------------------
+    // -- 10. U = U~ - W S -> U^T operand (over V) -----------------------------------------------
     if (lq < 2) {
 #pragma unroll
       for (int j = 0; j < kPart; j += 8) {

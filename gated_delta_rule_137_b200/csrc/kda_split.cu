@@ -12,15 +12,16 @@
 // independent across chunks. So the work is split:
 //
 //   plan  (kda_plan_kernel): cu_seqlens -> first global chunk index of each sequence;
-//   pass 1 (kda_intra_kernel): one CTA per (chunk, head), every chunk of the batch at
-//     once. Computes the state-free part and writes one item per (chunk, head):
-//       [-W; Qt]  128 x 128 fp32 tile   (A operand of D1 = [-W; Qt] S)
-//       P         rows 64..127 of a 128 x 64 tile (A operand of D1 += [.; P] U)
-//       Kh^T      128 x 64 tile         (A operand of D2 += Kh^T U)
-//       U~        64 x 128 fp32 (same swizzled layout, read back row by row)
+//   pass 1 (kda_intra_kernel): persistent CTAs walk every (chunk, head) of the batch.
+//     Computes the state-free part and writes one item per (chunk, head):
+//       [-W; Qt]  128 x 128 fp32 tile   (A operand of D1 = [-W; Qt] S, K-major)
+//       P         rows 64..127 of a 128 x 64 tile (A operand of D1 += [.; P] U, K-major)
+//       Kh        64 token lines of 128 channels: the MN-major A operand Kh^T of
+//                 D2 += Kh^T U (128B swizzle with 32-byte atoms)
+//       U~        64 x 128 fp32 (64-row swizzled layout, read back row by row)
 //       e^g_last  128 fp32
-//     The three tiles are written in the exact 128B-swizzled K-major layout the MMAs
-//     read, so pass 2 moves them into shared memory with plain bulk copies;
+//     The three tiles are written in the exact layouts the MMAs read, so pass 2 moves
+//     them into shared memory with plain bulk copies;
 //   pass 2 (kda_recur_kernel): one CTA per (sequence, head, slice of DV value columns)
 //     walks its chunks in order with the fp32 state slice in TMEM. Per chunk:
 //       group 1:  D1 = [-W; Qt] S                         (M128 NDV K128)
@@ -47,7 +48,7 @@ namespace {
 // ---- item layout (bytes from the start of one (chunk, head) item) ------------------
 constexpr uint32_t kItemQW = 0;          // [-W; Qt] tile, 64 KB
 constexpr uint32_t kItemP = 65536;       // P: rows 64..127 of K blocks 0 and 1, 2 x 8 KB
-constexpr uint32_t kItemKHT = 81920;     // Kh^T tile, 32 KB
+constexpr uint32_t kItemKHT = 81920;     // Kh (the MN-major A operand Kh^T), 32 KB
 constexpr uint32_t kItemU = 114688;      // U~ 64 x 128 fp32 in the 64-row tile layout, 32 KB
 constexpr uint32_t kItemGamma = 147456;  // e^g_last [128] fp32
 static_assert(kItemGamma + 512 == kItemBytes, "item layout");
@@ -112,8 +113,10 @@ __global__ void __launch_bounds__(1024) kda_plan_kernel(const int32_t* __restric
 // ================================ pass 1 =============================================
 // Persistent: each CTA walks the items it = blockIdx.x + k * gridDim.x (item = global
 // chunk it / H, head it % H). Two warp groups work on consecutive items at once:
-//   front (warps 0..7):  gate inputs, [Kt; Qt] and Kh, the [A; P] MMA, Kt^T      (item k+1)
-//   back  (warps 8..15): A and P out of TMEM, the triangular inverse, T into TMEM, V^T,
+//   front (warps 0..7):  gate inputs, [Kt; Qt] and Kh, the [A; P] MMA, Kt (and V) as
+//                        MN-major operand lines                                   (item k+1)
+//   back  (warps 8..15): A and P out of TMEM, the triangular inverse, T into TMEM (V for
+//                        the mixer),
 //                        the W / U~ MMA with A read from TMEM, -W, U~, P into the item (item k)
 // Each buffer the groups share is handed over through an mbarrier (bounded waits).
 constexpr int kIntraThreads = 512;
@@ -123,9 +126,10 @@ constexpr uint32_t kBarFront = 1, kBarBack = 2;  // named barrier ids of the two
 //  region  size     holds
 //  KQ      64 KB    [Kt; Qt] (128 x 128); the gate pass's decay totals first     (front)
 //  KH      32 KB    Kh (64 tok x 128 ch)                                         (front)
-//  KTT     32 KB    Kt^T (128 ch x 64 tok): front writes, back's W MMA reads; then staged -W
-//  VT      32 KB    V^T (128 dv x 64 tok), then staged U~                        (back)
-//  KHT     32 KB    Kh^T staged for the bulk store into the item                 (front)
+//  KTT     32 KB    Kt as MN-major lines (64 tok x 128 ch): front writes, back's W MMA
+//                   reads; then staged -W
+//  VT      32 KB    V as MN-major lines (64 tok x 128 dv), then staged U~
+//  KHT     32 KB    Kh as MN-major lines, staged for the bulk store into the item (front)
 //  SCR     25.5 KB  inverse scratch: A/X [64][kLd] + Y [32][kLd]                  (back)
 struct IntraSmem {
   static constexpr int kKQ = 0;
@@ -147,7 +151,7 @@ struct IntraSmem {
 enum : int {
   kBApFull = 0,  // [A; P] MMA done: back may read it, front may rewrite KQ / KH   (commit)
   kBApFree,      // back has read [A; P] out of TMEM                                (back arrives)
-  kBVtFull,      // front has written Kt^T                                          (front arrives)
+  kBVtFull,      // front has written Kt (and V)                                    (front arrives)
   kBWuDone,      // W / U~ MMA done                                                 (commit)
   kBWFree,       // back is done with KTT (W MMA read it, staged -W stored from it)  (back arrives)
   kBDrain        // teardown after a lost wait
@@ -472,7 +476,7 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
 #pragma unroll
         for (int g = 0; g < 16; ++g) gl += sTot[g * kD + ftid];
       }
-      if (ftid == 0) bulk_wait_read();  // the previous item's Qt and Kh^T have left KQ and KHT
+      if (ftid == 0) bulk_wait_read();  // the previous item's Qt and Kh have left KQ and KHT
       // The totals are read (KQ may be written) and the group votes: a chunk whose decay
       // passes kMaxChunkDecay in some channel is handed to the recurrence as its raw rows
       // (k, q after conv / L2, log_alpha, v, beta) and walked there token by token;
@@ -603,7 +607,7 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       }  // factorised form
       fence_proxy_async_smem();
       fsync();
-      if (ftid == 0 && !strong) {  // Qt: rows 64..127 of each 32-column block of the tile; Kh^T whole
+      if (ftid == 0 && !strong) {  // Qt: rows 64..127 of each 32-column block of the tile; Kh whole
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb)
           bulk_store(item + kItemQW + kb * 16384 + 8192, sm + SM::kKQ + kb * 16384 + 8192, 8192);
@@ -904,7 +908,7 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       bsync();
       tc_fence_after_sync();
 
-      // -- -W, U~ (over Kt^T and V^T, which the MMA has read) and P (over the scratch) staged
+      // -- -W, U~ (over the Kt and V tiles, which the MMA has read) and P (over the scratch) staged
       //    as 64-row tiles, then bulk-stored into the item --------------------------------------
       if (lq < 2) {
         const int r = row;
@@ -944,7 +948,7 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         bulk_store(item + kItemU, sm + SM::kVT, 32768);
         bulk_store(item + kItemP, sm + SM::kScr, 16384);
         bulk_commit_group();
-        bulk_wait_read();  // Kt^T, V^T and the scratch are free again
+        bulk_wait_read();  // the Kt and V tiles and the scratch are free again
         mbar_arrive(bars + kBWFree);
       }
       if (group_any(kBarBack, kGroupThreads, lost)) {
@@ -982,7 +986,7 @@ constexpr uint32_t kRecBarU = 1;  // named barrier: U^T written (epilogue warps 
 //  QW       64 KB       [-W; Qt] of the current chunk
 //  PT       2 x 32 KB   P of chunks i, i+1 (alternating) in rows 64..127 (K blocks at +8K,
 //                       +24K); the chunk's e^g_last in the unused rows at +0
-//  KHT      32 KB       Kh^T
+//  KHT      32 KB       Kh (the MN-major A operand Kh^T)
 //  ST       DV*512 B    S^T (DV x 128), the B operand of group 1
 //  UT       DV*256 B    U^T (DV x 64), the B operand of group 2
 template <int DV>
