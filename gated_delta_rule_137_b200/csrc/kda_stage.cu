@@ -17,15 +17,6 @@ namespace kda {
 namespace {
 
 template <typename T>
-__device__ __forceinline__ float ld_f32(const T* p, size_t i);
-template <>
-__device__ __forceinline__ float ld_f32<float>(const float* p, size_t i) { return p[i]; }
-template <>
-__device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
-  return __bfloat162float(p[i]);
-}
-
-template <typename T>
 __device__ __forceinline__ T zero_of();
 template <>
 __device__ __forceinline__ float zero_of<float>() { return 0.f; }
