@@ -825,6 +825,31 @@ def run_profile_tokens(args):
                       "bytes_per_call": mixer_decode_tokens_bytes(Nd, Kt)}), flush=True)
 
 
+def run_profile_mixer(args):
+    """The full mixer (conv4 + L2 + KDA + gate) on 2 x 8192 tokens of 32 heads — the config-2
+    shape with a quarter of its tokens (about 2 GB on the device), W + K calls, then one
+    line with the CUDA-event time per call; for kernel captures."""
+    import torch
+    import gated_delta_rule_137_b200 as kda
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(device)
+    lib = kda.load_library()
+    Bm, Tm = 2, 8192
+    mi = device_prefill_inputs(Bm * Tm, H, D, 1370002, device, normalise=False, mixer=True)
+    mo = torch.empty(Bm * Tm, H, D, dtype=torch.bfloat16, device=device)
+    mf = torch.empty(Bm, H, D, D, dtype=torch.float32, device=device)
+    mws = torch.empty(lib.kda_mixer_fwd_workspace(Bm * Tm, Bm, H, D, D), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def call(i):
+        kda.mixer_fwd(mi["q"], mi["k"], mi["v"], mi["conv_w"], mi["log_alpha"], mi["beta"], mi["gate"], None,
+                      None, N=Bm, out=mo, final_state=mf, workspace=mws, stream=stream)
+
+    per, tot = time_region(call, args.steps, args.warmup, stream, device)
+    print(json.dumps({"case": f"full mixer {Bm} x {Tm} tokens, H={H} d={D}", "ms_per_call": tot / args.steps,
+                      "bytes_per_call": prefill_bytes(Bm * Tm, Bm, with_h0=False, mixer=True)}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -838,6 +863,8 @@ def main(argv=None):
                     help="only a mid-size single-pass prefill (8 x 4096 tokens, 32 heads), for kernel captures")
     ap.add_argument("--profile-tokens", action="store_true",
                     help="only the 4-token serving decode (256 sequences, 32 heads), for kernel captures")
+    ap.add_argument("--profile-mixer", action="store_true",
+                    help="only the full mixer on 2 x 8192 tokens (32 heads), for kernel captures")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per headline call to report instead of profiles/traffic.json")
     args = ap.parse_args(argv)
@@ -849,6 +876,8 @@ def main(argv=None):
         run_profile_case(args)
     elif args.profile_tokens:
         run_profile_tokens(args)
+    elif args.profile_mixer:
+        run_profile_mixer(args)
     else:
         run_gpu(args)
 
