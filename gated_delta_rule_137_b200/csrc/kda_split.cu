@@ -495,16 +495,26 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         RawRowsFront rr{a.q, a.k, a.log_alpha, a.a_pre, a.a_scale, a.conv_w, item, t0, bos, len, h, H, fw};
         raw_rows_front<TIn, kConv, kPre>(rr);
       } else {
+        // q/k row m of group s is chunk row r0 - kHist + m; rows outside [bos, t0 + len) read
+        // row t0 (always in bounds) and are replaced by zero where used. With the conv, the
+        // second group's history rows are the first group's last rows: carried, not reloaded.
+        uint32_t kraw[kGRows][sizeof(TIn)], qraw[kGRows][sizeof(TIn)];
+        bool rin[kGRows];
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           const int r0 = 4 * (2 * fw + s);
-          // q/k row m is chunk row r0 - kHist + m; rows outside [bos, t0 + len) read row t0
-          // (always in bounds) and are replaced by zero where used
-          uint32_t kraw[kGRows][sizeof(TIn)], qraw[kGRows][sizeof(TIn)];
-          bool rin[kGRows];
 #pragma unroll
           for (int m = 0; m < kGRows; ++m) {
             const int rr = r0 - kHist + m;
+            if (kConv && s == 1 && m < kHist) {
+#pragma unroll
+              for (int w = 0; w < static_cast<int>(sizeof(TIn)); ++w) {
+                kraw[m][w] = kraw[m + 4][w];
+                qraw[m][w] = qraw[m + 4][w];
+              }
+              rin[m] = rin[m + 4];
+              continue;
+            }
             rin[m] = rr < len && t0 + rr >= bos;
             if constexpr (!kConv) {
 #pragma unroll
@@ -811,9 +821,14 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         const TIn* vh = static_cast<const TIn*>(a.v) + static_cast<size_t>(ip.h) * kD;
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
-          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+          const int t4 = 4 * (2 * (btid >> 5) + bb), j4 = 4 * (btid & 31);  // two consecutive groups
 #pragma unroll
           for (int m = 0; m < kGRows; ++m) {
+            if (bb == 1 && m < kHist) {  // the second group's history rows: the first group's last
+#pragma unroll
+              for (int w = 0; w < kWb; ++w) vraw[1][m][w] = vraw[0][m + 4][w];
+              continue;
+            }
             const int rr = t4 - kHist + m;
             const bool in = rr < ip.len && ip.t0 + rr >= ip.bos;
             const TIn* src = vh + static_cast<size_t>(in ? ip.t0 + rr : ip.t0) * tok_stride + j4;
@@ -853,7 +868,7 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
       if constexpr (!kVFront) {
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
-          const int blk = btid + bb * kGroupThreads, t4 = 4 * (blk >> 5), j4 = 4 * (blk & 31);
+          const int t4 = 4 * (2 * (btid >> 5) + bb), j4 = 4 * (btid & 31);  // two consecutive groups
           auto elem = [&](int jr, int m) -> float {  // column j4 + jr of loaded row m
             if constexpr (kWb == 2) {
               const uint32_t x = vraw[bb][m][jr >> 1];
