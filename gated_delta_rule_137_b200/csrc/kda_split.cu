@@ -1333,7 +1333,7 @@ __device__ __forceinline__ void recur_body(const PrefillArgs& a, const SplitPlan
           float ws[8];
           tmem_ld8(d1 + lane_off + cc, ws);
           tmem_ld_wait();
-          // U row `row` as a line of the MN-major B operand of group 2
+          // U row `row` into the U^T operand of group 2
 #pragma unroll
           for (int e = 0; e < 8; ++e) st_tf32(sm + SM::kUT, f32_offset(cc + e, row, DV), ut[j + e] + ws[e]);
         }
