@@ -125,12 +125,13 @@ constexpr uint32_t kBarFront = 1, kBarBack = 2;  // named barrier ids of the two
 
 //  region  size     holds
 //  KQ      64 KB    [Kt; Qt] (128 x 128); the gate pass's decay totals first     (front)
-//  KH      32 KB    Kh (64 tok x 128 ch)                                         (front)
+//  KH      32 KB    Kh (64 tok x 128 ch); the mixer's decay running sums first   (front)
 //  KTT     32 KB    Kt as MN-major lines (64 tok x 128 ch): front writes, back's W MMA
 //                   reads; then staged -W
 //  VT      32 KB    V as MN-major lines (64 tok x 128 dv), then staged U~
 //  KHT     32 KB    Kh as MN-major lines, staged for the bulk store into the item (front)
 //  SCR     25.5 KB  inverse scratch: A/X [64][kLd] + Y [32][kLd]                  (back)
+//  CONVW   4 KB     the mixer's q, k conv taps of the item's head                 (front)
 struct IntraSmem {
   static constexpr int kKQ = 0;
   static constexpr int kKH = 65536;
@@ -144,7 +145,8 @@ struct IntraSmem {
   static constexpr int kNumBars = 8;
   static constexpr int kTmemSlot = kBar + 8 * kNumBars;
   static constexpr int kStrong = kTmemSlot + 16;     // int [2]: the item is walked token by token
-  static constexpr int kTotal = kStrong + 16;
+  static constexpr int kConvW = kStrong + 16;       // fp32 [2][4][128]: q, k conv taps (tap, channel)
+  static constexpr int kTotal = kConvW + 4096;
   static constexpr int kAlloc = kTotal + 1024;
   static_assert(kAlloc <= 232448, "shared memory plan exceeds the per-block limit");
 };
@@ -326,6 +328,10 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
   // which group builds the V rows: the front one, except for the mixer, whose gate pass
   // (conv and L2 norm of q and k) already makes the front group the longer one
   constexpr bool kVFront = !kConv;
+  // the conv's gate pass holds its taps and 7 raw rows per group in registers: the decay's
+  // running sums wait in shared memory meanwhile, in the bytes of KH that the same thread's
+  // Kh rows overwrite later (no other thread touches them in between)
+  constexpr bool kParkLa = kConv;
 
   const int H = a.H;
   const int total_chunks = __ldg(p.chunk_start + a.N);
@@ -408,6 +414,9 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
         fsync();
       }
       if (ftid < 64) sB[ftid] = ftid < len ? __ldg(a.beta + (t0 + ftid) * H + h) : 0.f;
+      float4 wtap;  // the conv taps of channel ftid & 127 of q (ftid < 128) or k
+      if constexpr (kConv)
+        wtap = __ldg(reinterpret_cast<const float4*>(a.conv_w + (((ftid >> 7) * H + h) * kD + (ftid & 127)) * 4));
 
       // raw q/k rows of both 4-token groups, in flight together with log_alpha (no conv:
       // the conv's extra history rows are loaded per group below)
@@ -461,7 +470,16 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) { tot[s][e] += la[s][i][e]; la[s][i][e] = tot[s][e]; }
         }
+        if constexpr (kParkLa) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            st4_f32(sm + SM::kKH, f32_offset(r0 + i, c0, 64), la[s][i][0], la[s][i][1], la[s][i][2], la[s][i][3]);
+        }
         *reinterpret_cast<float4*>(sTot + (2 * fw + s) * kD + c0) = make_float4(tot[s][0], tot[s][1], tot[s][2], tot[s][3]);
+      }
+      if constexpr (kConv) {
+        float* w = reinterpret_cast<float*>(sm + SM::kConvW) + (ftid >> 7) * 512 + (ftid & 127);
+        w[0] = wtap.x; w[128] = wtap.y; w[256] = wtap.z; w[384] = wtap.w;
       }
       fsync();
       float pre[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -548,13 +566,15 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
           if constexpr (kConv) {
             // y[t, c] = sum_j w[c, j] x[t - 3 + j, c] (x = 0 before the sequence start), then
             // x / sqrt(sum_c y^2 + 1e-6) over the head's 128 channels (this warp holds them all)
+            // taps from shared memory, [tensor][tap][channel]
+            const float* sw = reinterpret_cast<const float*>(sm + SM::kConvW) + c0;
             float wq[4][4], wk[4][4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float4 a4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((0 * H + h) * kD + c0 + e) * 4));
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.conv_w + ((1 * H + h) * kD + c0 + e) * 4));
-              wq[e][0] = a4.x; wq[e][1] = a4.y; wq[e][2] = a4.z; wq[e][3] = a4.w;
-              wk[e][0] = b4.x; wk[e][1] = b4.y; wk[e][2] = b4.z; wk[e][3] = b4.w;
+            for (int j = 0; j < 4; ++j) {
+              const float4 a4 = *reinterpret_cast<const float4*>(sw + j * 128);
+              const float4 b4 = *reinterpret_cast<const float4*>(sw + 512 + j * 128);
+              wq[0][j] = a4.x; wq[1][j] = a4.y; wq[2][j] = a4.z; wq[3][j] = a4.w;
+              wk[0][j] = b4.x; wk[1][j] = b4.y; wk[2][j] = b4.z; wk[3][j] = b4.w;
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -598,15 +618,23 @@ __global__ void __launch_bounds__(kIntraThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float kt[4], qt[4], kh[4];
+            const int r = r0 + i;
+            float lr[4];
+            if constexpr (kParkLa) {
+              const float4 l4 = *reinterpret_cast<const float4*>(sm + SM::kKH + f32_offset(r, c0, 64));
+              lr[0] = l4.x; lr[1] = l4.y; lr[2] = l4.z; lr[3] = l4.w;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) lr[e] = la[s][i][e];
+            }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float g = pre[s][e] + la[s][i][e];
+              const float g = pre[s][e] + lr[e];
               const float eg = __expf(g), eng = __expf(-g);
               kt[e] = kv[i][e] * eg;
               kh[e] = to_tf32(kv[i][e] * eng);
               qt[e] = to_tf32(qv[i][e] * eg);
             }
-            const int r = r0 + i;
             st4_f32(sm + SM::kKQ, f32_offset(r, c0, 128), kt[0], kt[1], kt[2], kt[3]);       // Kt [tok][ch]
             st4_f32(sm + SM::kKQ, f32_offset(64 + r, c0, 128), qt[0], qt[1], qt[2], qt[3]);  // Qt [tok][ch]
             st4_f32(sm + SM::kKH, f32_offset(r, c0, 64), kh[0], kh[1], kh[2], kh[3]);        // Kh [tok][ch]
