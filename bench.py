@@ -106,6 +106,22 @@ def load_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+def headline_input_sets() -> int:
+    """Device copies of the headline inputs the timed calls rotate through: more than
+    3x the 126 MB L2 in all, so no call finds its inputs in L2."""
+    return max(2, math.ceil(3 * 126e6 / prefill_bytes(T1, 1)) + 1)
+
+
+def headline_config(world: int) -> dict:
+    """The workload of the headline line, the same for both arms (the reference arm
+    times the oracle on a bounded sample of it; its `cpu_baseline` says which)."""
+    n_sets = headline_input_sets()
+    return {"workload": "KDA chunked prefill B=1 T=4096 H=32 d_k=d_v=128 (bf16 q/k/v, fp32 log_alpha/beta/state)",
+            "global_batch": world, "seq_len": T1, "heads": H, "head_dim": D, "chunk": CHUNK,
+            "parallelism": f"replicas x{world} (independent (sequence, head) chains, no collective)",
+            "l2": f"inputs rotate through {n_sets} device copies ({n_sets * prefill_bytes(T1, 1) / 1e6:.0f} MB > L2)"}
+
+
 # The sources the headline call's kernels (plan, intra-chunk, recurrence) are compiled from.
 HEADLINE_KERNEL_SOURCES = ("kda_split.cu", "kda_tile.cuh", "sm100_ptx.cuh")
 
@@ -306,7 +322,7 @@ def run_gpu(args):
                 v=torch.from_numpy(w.v).to(torch.bfloat16), log_alpha=torch.from_numpy(w.log_alpha),
                 beta=torch.from_numpy(w.beta), initial_state=torch.from_numpy(w.initial_state))
     bytes_call = prefill_bytes(T1, 1)
-    n_sets = max(2, math.ceil(3 * 126e6 / bytes_call) + 1)  # rotate through > 3x L2
+    n_sets = headline_input_sets()
     sets = []
     for _ in range(n_sets):
         sets.append({k: t.to(device) for k, t in host.items()})
@@ -655,10 +671,7 @@ def run_gpu(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded NumPy generator; random inputs, no weights)",
-            "config": {"workload": "KDA chunked prefill B=1 T=4096 H=32 d_k=d_v=128 (bf16 q/k/v, fp32 log_alpha/beta/state)",
-                       "global_batch": world, "seq_len": T1, "heads": H, "head_dim": D, "chunk": CHUNK,
-                       "parallelism": f"replicas x{world} (independent (sequence, head) chains, no collective)",
-                       "l2": f"inputs rotate through {n_sets} device copies ({n_sets * bytes_call / 1e6:.0f} MB > L2)"},
+            "config": headline_config(world),
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved_gbs / hbm_peak, "traffic": load_traffic(args.traffic),
                          "kernel": "kda_chunk_fwd (plan + intra-chunk + recurrence kernels, one call)",
@@ -757,8 +770,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded NumPy generator)",
-        "config": {"workload": "KDA chunked prefill B=1 T=4096 H=32 d_k=d_v=128 (bf16 q/k/v, fp32 log_alpha/beta/state)",
-                   "global_batch": 1, "seq_len": T1, "parallelism": "host CPU, 1 core"},
+        "config": headline_config(world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": "each step: 1 of 32 heads x the first 1024 tokens (scaled to all heads)", **host},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

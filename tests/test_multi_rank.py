@@ -111,3 +111,24 @@ def test_backward_work_figure():
     assert per_tok == 3592
     assert bench.backward_bytes(4096, 1) == 4096 * 32 * per_tok + 3 * 32 * 128 * 128 * 4
     assert bench.backward_bytes(0, 2) == 3 * 2 * 32 * 128 * 128 * 4
+
+
+def test_reference_arm_line_on_the_host():
+    """`bench.py --impl reference` times the fp64 oracle on the host (no GPU) and prints
+    one line on the headline's metric, unit and config, with the sample it timed."""
+    import json
+    import subprocess
+    import sys
+    import bench
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0"],
+                       cwd=bench.ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["metric"] == bench.METRIC and j["unit"] == "tokens/s"
+    assert j["higher_is_better"] is True and j["steps"] == 1 and j["n_gpus"] == 1
+    assert j["config"] == bench.headline_config(1)
+    assert j["value"] > 0 and j["cpu_baseline"]["value"] == j["value"]
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1 and j["cpu_baseline"]["sample"]
+    assert j["e2e"] == {"value": j["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
